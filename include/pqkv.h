@@ -1,0 +1,242 @@
+/*
+ * pqkv.h -- C ABI of the paged, quantized KV-cache decode-attention library.
+ *
+ * The operations follow the method described on three public web pages:
+ *   [P1] "vLLM 0.7 Ships Unified KV Cache Compression: 3.4x Higher Concurrency
+ *        on Enterprise Clusters" (dailyaiworld.com), sections "Technical
+ *        Breakdown: Dynamic Quantization with Outlier Retention" (steps 1-4) and
+ *        the architecture diagram (512-token chunks, FP16 outlier buffer,
+ *        Flash-Decoding kernel).
+ *   [P2] "vLLM v0.7.2" field report (xonoai.com/?p=2844), section
+ *        "Deconstructing the v0.7.2 Architecture" (FP8 E4M3/E5M2 KV cache,
+ *        16-token blocks, page tables) and "Field Observations & Production
+ *        Failure Modes" (block pool exhaustion).
+ *   [P3] "vLLM" glossary (inferensys.com), entries "PagedAttention" (fixed-size
+ *        blocks, logical-to-physical mapping, sharing across sequences),
+ *        "Continuous batching" (blocks returned to the pool), "KV cache
+ *        quantization" (FP8 just-in-time quantization).
+ * Number formats follow the public OCP 8-bit Floating Point Specification
+ * (OFP8: E4M3 "fn" with max 448 and no infinities, E5M2 with max 57344) and the
+ * OCP Microscaling Formats specification (E2M1: values 0, .5, 1, 1.5, 2, 3, 4, 6).
+ *
+ * General conventions
+ *  - Every pointer argument named "device" must point to GPU memory owned by the
+ *    caller; every "host" pointer to CPU memory owned by the caller. The library
+ *    never allocates, frees or retains device memory.
+ *  - GPU entry points are asynchronous on `stream` (a cudaStream_t, 0 = legacy
+ *    default stream). A return of PQKV_OK means the work was enqueued.
+ *  - Problems found on the device never trap: the offending item is skipped and
+ *    a PQKV_DEVERR_* bit is ORed into the caller's device int32 *err_flag (which
+ *    the caller zeroes and reads back when it synchronizes).
+ *  - Integer arguments are validated on the host first; invalid ones return
+ *    PQKV_ERR_ARG and launch nothing.
+ *
+ * Cache layout (num_blocks = nb, num_kv_heads = H, head_dim = D, block = 16):
+ *  One (block, head) pair holds its K tile and then its V tile contiguously, so
+ *  one gathered block of one KV head is one contiguous region of the cache.
+ *   FP16 / BF16 : cache  [nb][H][2 (K,V)][16][D] 2-byte elements (bit copy of input)
+ *   FP8 E4M3/E5M2: cache [nb][H][2][16][D] one code per byte
+ *                 scales [nb][H][4] float32 = {scale_K, scale_V, 0, 0}
+ *                 (value = decode(code) * scale; 16-byte granule per pair)
+ *   FP4 E2M1    : cache  [nb][H][2][16][D/2] bytes, channel 2i in the low nibble,
+ *                 channel 2i+1 in the high nibble
+ *                 scales [nb][H][2][16][D/16] unsigned E4M3 codes, one per
+ *                 16 consecutive channels of one token
+ *                 outliers_idx [nb][H][2][8] uint8: slots 0..3 hold the outlier
+ *                 channels in ascending order, 0xFF = empty; slots 4..7 = 0xFF
+ *                 outliers_val [nb][H][2][16][4] IEEE fp16, value of outlier
+ *                 slot r for token offset t (+0 for empty slots)
+ *                 (value = channel in slot r ? outliers_val : e2m1(code)*e4m3(scale);
+ *                 an outlier channel's own code is 0)
+ *  Slot s addresses token offset s % 16 of physical block s / 16.
+ */
+#ifndef PQKV_H
+#define PQKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* cudaStream_t-compatible handle, declared here so that this header does not
+ * need the CUDA headers. */
+typedef struct CUstream_st* pqkv_stream_t;
+
+/* ---- return codes ---------------------------------------------------------- */
+enum {
+  PQKV_OK = 0,
+  PQKV_ERR_ARG = 1,   /* null pointer, bad enum, unsupported size, small buffer */
+  PQKV_ERR_OOM = 2,   /* block pool cannot satisfy an allocation (no change made) */
+  PQKV_ERR_STATE = 3, /* refcount underflow / freeing or sharing a free block */
+  PQKV_ERR_CUDA = 4   /* a CUDA runtime call or launch failed */
+};
+
+/* ---- element types ---------------------------------------------------------- */
+enum {
+  PQKV_DTYPE_FP16 = 0,
+  PQKV_DTYPE_BF16 = 1,
+  PQKV_DTYPE_FP8_E4M3 = 2,
+  PQKV_DTYPE_FP8_E5M2 = 3,
+  PQKV_DTYPE_FP4_E2M1 = 4
+};
+
+/* ---- device error bits (ORed into *err_flag) -------------------------------- */
+enum {
+  PQKV_DEVERR_SLOT = 1,      /* write: slot >= 16 * num_blocks; token skipped */
+  PQKV_DEVERR_BLOCK_ID = 2,  /* decode: table entry outside [0, num_blocks); block skipped */
+  PQKV_DEVERR_SEQ_LEN = 4,   /* decode: seq_len < 0 or > 16 * max_blocks_per_seq; sequence
+                                skipped and its output rows written as zeros */
+  PQKV_DEVERR_RUN = 8,       /* write (FP8/FP4): two adjacent tokens map to the same block
+                                with non-consecutive offsets */
+  PQKV_DEVERR_TIMEOUT = 16   /* a bounded wait on an asynchronous copy gave up */
+};
+
+#define PQKV_BLOCK_SIZE 16
+#define PQKV_FP4_GROUP 16
+#define PQKV_FP4_OUTLIER_SLOTS 4
+#define PQKV_FP4_IDX_STRIDE 8
+#define PQKV_FP4_SIGMA 3.2
+#define PQKV_MAX_BATCH 4096
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int pqkv_version(void);
+
+/* Human-readable name of a PQKV_* return code. Never NULL. */
+const char* pqkv_status_string(int status);
+
+/*
+ * Byte sizes of the four cache arrays for `kv_dtype`: out_bytes[0] = cache,
+ * [1] = scales, [2] = outliers_idx, [3] = outliers_val (0 where the format has
+ * no such array). Layout as in the header comment. Sizing the pool is the
+ * caller's decision (vLLM's --gpu-memory-utilization in [P1]/[P2] launch
+ * configurations). head_dim must be 64 or 128; num_blocks, num_kv_heads >= 1.
+ */
+int pqkv_cache_layout(int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                      size_t out_bytes[4]);
+
+/*
+ * Quantizing cache write ([P1] steps 1-3; [P2] FP8 KV cache; [P3] "KV cache
+ * quantization"). Token i (0 <= i < num_tokens) of k and v, each
+ * [num_tokens][num_kv_heads][head_dim] contiguous device arrays of `in_dtype`
+ * (FP16 or BF16), is stored at slot slot_mapping[i] (device int32; < 0 = skip).
+ *   16-bit kv_dtype: bit copy; requires in_dtype == kv_dtype.
+ *   FP8: tokens are grouped into runs (maximal chains of consecutive tokens
+ *     whose slots increase by one inside one block). Per run, head and K|V:
+ *     a = max |x| over the run; s_run = fp32(a / FPMAX) (448 or 57344). If the
+ *     run starts at offset 0 the block scale becomes s_run; otherwise
+ *     s = max(s_old, s_run) and, if it grew, the existing codes at offsets below
+ *     the run are re-encoded as enc(fp32(fp32(dec(c) * s_old) / s)). New codes
+ *     are enc(fp32(x / s)) (all +0 when s == 0); enc rounds to nearest even and
+ *     saturates to +-FPMAX, keeping the sign of zero.
+ *   FP4: for a run starting at offset 0, per head and K|V: channel norm
+ *     n_c = max_t |x_tc| over the run; mu and sigma (population) of the D norms
+ *     in fp64; channels with n_c >= mu + 3.2 sigma are outliers, at most 4 kept
+ *     (largest n_c first, ties to the lower channel), stored ascending. Runs
+ *     starting later reuse the stored set. Per token: outlier values -> fp16
+ *     (round to nearest even); per 16-channel group over non-outlier channels,
+ *     scale code = e4m3(fp32(absmax / 6)) and codes e2m1(fp32(x / dec(scale)))
+ *     (code +0 for outlier channels and when the decoded scale is 0).
+ * A block must not receive tokens from two different runs in one call, and a
+ * run not starting at offset 0 must append to a block written earlier. Inputs
+ * must be finite. err_flag: device int32, never NULL.
+ */
+int pqkv_kv_cache_write(const void* k, const void* v, int in_dtype, int num_tokens,
+                        const int32_t* slot_mapping, void* cache, void* scales,
+                        void* outliers_idx, void* outliers_val, int kv_dtype,
+                        int num_blocks, int num_kv_heads, int head_dim,
+                        int32_t* err_flag, pqkv_stream_t stream);
+
+/*
+ * Device workspace needed by pqkv_paged_decode_attention for these sizes, on
+ * the current device. split_blocks as in pqkv_paged_decode_attention. Returns 0
+ * for invalid sizes.
+ */
+size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
+                                   int head_dim, int max_blocks_per_seq,
+                                   int split_blocks);
+
+/*
+ * Split-K paged decode attention with log-sum-exp merge ([P1] steps 3-4 and the
+ * "Flash-Decoding Kernel" of its diagram; [P3] "PagedAttention").
+ * For sequence b and query head hq (kv head h = hq / (num_q_heads/num_kv_heads)):
+ *   L = seq_lens[b]; token t < L lives at offset t % 16 of physical block
+ *   block_tables[b * max_blocks_per_seq + t / 16];
+ *   out[b][hq] = sum_t softmax_t(scale * q[b][hq] . k_t) * v_t
+ * with k_t, v_t dequantized from the cache. q and out: [batch][num_q_heads]
+ * [head_dim] device arrays of q_dtype (FP16 or BF16); BF16/FP16 caches need
+ * q_dtype == kv_dtype. num_q_heads / num_kv_heads must be an integer 1..8.
+ * Table entries at and beyond ceil(L/16) are never read; a physical block may
+ * appear in several tables. L == 0 gives zero output rows.
+ * split_blocks: 0 = balance the work of all sequences and heads evenly over the
+ * GPU; > 0 = process the KV of all (sequence, head) pairs, laid end to end, in
+ * chunks of exactly that many 16-token blocks. Results differ only by rounding.
+ * workspace: device buffer of at least pqkv_decode_workspace_bytes(...) bytes,
+ * zero-filled before its first use (pqkv_decode_workspace_init); every call
+ * leaves it ready for the next. Calls that share a workspace must be ordered.
+ * batch <= PQKV_MAX_BATCH.
+ */
+int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads,
+                                const void* cache, const void* scales,
+                                const void* outliers_idx, const void* outliers_val,
+                                int kv_dtype, int num_blocks, int num_kv_heads,
+                                int head_dim, const int32_t* block_tables,
+                                int max_blocks_per_seq, const int32_t* seq_lens,
+                                float scale, int split_blocks, void* out,
+                                void* workspace, size_t workspace_bytes,
+                                int32_t* err_flag, pqkv_stream_t stream);
+
+/* Zero-fill a decode workspace on `stream` (needed once per new buffer). */
+int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
+                               pqkv_stream_t stream);
+
+/*
+ * Element-wise encoder used by the cache write: n float32 values (device) to
+ * codes (device, one byte each) of FP8 E4M3, FP8 E5M2 or E2M1 (low nibble),
+ * round to nearest even with saturation to the largest finite value, sign of
+ * zero kept. Inputs must be finite.
+ */
+int pqkv_encode(const float* x, int64_t n, int code_dtype, uint8_t* codes,
+                pqkv_stream_t stream);
+
+/* ---- block pool ([P3] PagedAttention / continuous batching; [P2] pool
+ *      exhaustion) ------------------------------------------------------------
+ * Host-only allocator of physical block ids 0..num_blocks-1 with reference
+ * counts, so that one block can sit in several block tables. O(1) per block.
+ * Not thread-safe: one scheduler thread owns a pool. */
+typedef struct pqkv_pool pqkv_pool;
+
+/* Create a pool with all blocks free. Allocation hands out the lowest free ids
+ * first on a fresh pool, then reuses freed ids last-in first-out. */
+int pqkv_pool_create(int32_t num_blocks, pqkv_pool** out_pool);
+void pqkv_pool_destroy(pqkv_pool* pool);
+/* Allocate n blocks into ids_out (host), refcount 1 each. All or nothing:
+ * PQKV_ERR_OOM leaves the pool unchanged. */
+int pqkv_pool_alloc(pqkv_pool* pool, int n, int32_t* ids_out);
+/* Add one reference to each of ids[0..n) (host). Every id must be allocated;
+ * otherwise PQKV_ERR_STATE (or ERR_ARG for an id out of range), no change. */
+int pqkv_pool_share(pqkv_pool* pool, const int32_t* ids, int n);
+/* Drop one reference from each of ids[0..n) (host); blocks reaching 0 return to
+ * the pool. Dropping more references than an id holds (counting repeats in
+ * ids) gives PQKV_ERR_STATE and no change. */
+int pqkv_pool_free(pqkv_pool* pool, const int32_t* ids, int n);
+int32_t pqkv_pool_num_free(const pqkv_pool* pool);
+/* Reference count of `id`, or -1 if out of range. */
+int32_t pqkv_pool_refcount(const pqkv_pool* pool, int32_t id);
+
+/*
+ * Host helper: slot mapping for appending tokens. For each sequence b, tokens
+ * at positions start_pos[b] .. start_pos[b] + num_new[b] - 1 get
+ * slot = block_tables[b][pos / 16] * 16 + pos % 16, written consecutively into
+ * slots_out (host int32, sum(num_new) entries). Returns PQKV_ERR_ARG if a
+ * position needs a table entry outside [0, max_blocks_per_seq) or a negative id.
+ */
+int pqkv_build_slot_mapping(const int32_t* block_tables, int batch,
+                            int max_blocks_per_seq, const int32_t* start_pos,
+                            const int32_t* num_new, int32_t* slots_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PQKV_H */
