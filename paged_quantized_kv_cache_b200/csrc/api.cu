@@ -1,0 +1,259 @@
+// api.cu -- C ABI entry points: argument validation, TMA descriptors, launches.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstring>
+#include <mutex>
+
+#include "decode.cuh"
+#include "write.cuh"
+
+namespace pqkv {
+cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap, const DecodeParams& p,
+                          int grid, cudaStream_t st);
+size_t decode_smem_bytes(int kv_dtype, int D, int B);
+}  // namespace pqkv
+
+using namespace pqkv;
+
+namespace {
+
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded wait on one asynchronous copy
+
+bool is_kv_dtype(int t) { return t >= PQKV_DTYPE_FP16 && t <= PQKV_DTYPE_FP4_E2M1; }
+bool is_16(int t) { return t == PQKV_DTYPE_FP16 || t == PQKV_DTYPE_BF16; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int sms = 0;
+  int max_smem = 0;
+};
+
+bool device_info(DeviceInfo& out) {
+  static std::mutex mu;
+  static DeviceInfo cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev].sms == 0) {
+    int sms = 0, smem = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return false;
+    if (cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) return false;
+    cache[dev].sms = sms;
+    cache[dev].max_smem = smem;
+  }
+  out = cache[dev];
+  return true;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// TMA descriptor over the cache viewed as rows of one token's K or V:
+// [num_blocks * H * 2 * 16 rows][row bytes]; one box = 32 rows (K and V of one
+// (block, head) pair) x up to 128 bytes, swizzled to the box row width.
+bool make_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb, int H, int D) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const int row = row_bytes(kv_dtype, D);
+  const int box_row = std::min(row, 128);
+  const int esz = is_16(kv_dtype) ? 2 : 1;
+  const CUtensorMapDataType dt = is_16(kv_dtype) ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const cuuint64_t dims[2] = {(cuuint64_t)(row / esz), (cuuint64_t)nb * H * 2 * 16};
+  const cuuint64_t strides[1] = {(cuuint64_t)row};
+  const cuuint32_t box[2] = {(cuuint32_t)(box_row / esz), 32};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle sw = box_row == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                                : box_row == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                : CU_TENSOR_MAP_SWIZZLE_32B;
+  const CUresult r = fn(map, dt, 2, const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Most recent descriptor per thread (the cache buffer rarely changes).
+bool cached_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb, int H, int D) {
+  struct Key {
+    const void* p;
+    int dt, nb, H, D, dev;
+  };
+  thread_local Key key{nullptr, -1, 0, 0, 0, -1};
+  thread_local CUtensorMap last;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (key.p == cache && key.dt == kv_dtype && key.nb == nb && key.H == H && key.D == D && key.dev == dev) {
+    *map = last;
+    return true;
+  }
+  if (!make_cache_map(&last, cache, kv_dtype, nb, H, D)) return false;
+  key = Key{cache, kv_dtype, nb, H, D, dev};
+  *map = last;
+  return true;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" {
+
+int pqkv_version(void) { return 10000; }
+
+const char* pqkv_status_string(int status) {
+  switch (status) {
+    case PQKV_OK: return "ok";
+    case PQKV_ERR_ARG: return "invalid argument";
+    case PQKV_ERR_OOM: return "block pool exhausted";
+    case PQKV_ERR_STATE: return "invalid block state";
+    case PQKV_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int pqkv_cache_layout(int kv_dtype, int num_blocks, int num_kv_heads, int head_dim, size_t out_bytes[4]) {
+  if (!out_bytes || !is_kv_dtype(kv_dtype) || num_blocks < 1 || num_kv_heads < 1 ||
+      (head_dim != 64 && head_dim != 128))
+    return PQKV_ERR_ARG;
+  const size_t pairs = (size_t)num_blocks * num_kv_heads;
+  out_bytes[0] = pairs * 2 * PQKV_BLOCK_SIZE * (size_t)row_bytes(kv_dtype, head_dim);
+  out_bytes[1] = out_bytes[2] = out_bytes[3] = 0;
+  if (kv_dtype == PQKV_DTYPE_FP8_E4M3 || kv_dtype == PQKV_DTYPE_FP8_E5M2) out_bytes[1] = pairs * 4 * sizeof(float);
+  if (kv_dtype == PQKV_DTYPE_FP4_E2M1) {
+    out_bytes[1] = pairs * 2 * PQKV_BLOCK_SIZE * (size_t)(head_dim / PQKV_FP4_GROUP);
+    out_bytes[2] = pairs * 2 * PQKV_FP4_IDX_STRIDE;
+    out_bytes[3] = pairs * 2 * PQKV_BLOCK_SIZE * PQKV_FP4_OUTLIER_SLOTS * 2;
+  }
+  return PQKV_OK;
+}
+
+int pqkv_kv_cache_write(const void* k, const void* v, int in_dtype, int num_tokens, const int32_t* slot_mapping,
+                        void* cache, void* scales, void* outliers_idx, void* outliers_val, int kv_dtype,
+                        int num_blocks, int num_kv_heads, int head_dim, int32_t* err_flag, pqkv_stream_t stream) {
+  if (!is_kv_dtype(kv_dtype) || (in_dtype != PQKV_DTYPE_FP16 && in_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
+  if (is_16(kv_dtype) && in_dtype != kv_dtype) return PQKV_ERR_ARG;
+  if (num_tokens < 0 || num_blocks < 1 || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128))
+    return PQKV_ERR_ARG;
+  if ((int64_t)num_blocks * PQKV_BLOCK_SIZE > INT32_MAX) return PQKV_ERR_ARG;
+  if (num_tokens == 0) return PQKV_OK;
+  if (!k || !v || !slot_mapping || !cache || !err_flag) return PQKV_ERR_ARG;
+  if (!aligned16(k) || !aligned16(v) || !aligned16(cache)) return PQKV_ERR_ARG;
+  if (!is_16(kv_dtype) && !scales) return PQKV_ERR_ARG;
+  if (kv_dtype == PQKV_DTYPE_FP4_E2M1 && (!outliers_idx || !outliers_val)) return PQKV_ERR_ARG;
+  WriteParams p;
+  p.k = k;
+  p.v = v;
+  p.slots = slot_mapping;
+  p.cache = static_cast<uint8_t*>(cache);
+  p.scales = static_cast<uint8_t*>(scales);
+  p.oidx = static_cast<uint8_t*>(outliers_idx);
+  p.oval = static_cast<uint8_t*>(outliers_val);
+  p.err = err_flag;
+  p.T = num_tokens;
+  p.nb = num_blocks;
+  p.Hkv = num_kv_heads;
+  const cudaError_t e = launch_write(kv_dtype, in_dtype, head_dim, p, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads, int head_dim,
+                                   int max_blocks_per_seq, int split_blocks) {
+  if (batch < 1 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+      (head_dim != 64 && head_dim != 128) || max_blocks_per_seq < 1 || split_blocks < 0)
+    return 0;
+  const int G = num_q_heads / num_kv_heads;
+  if (G > 8) return 0;
+  DeviceInfo di;
+  if (!device_info(di)) return 0;
+  const size_t counters = round_up((size_t)batch * num_kv_heads * 4, 256);
+  const size_t slot = round_up((size_t)G * head_dim + 2 * G, 4) * 4;
+  const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
+  const size_t chunks = split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks
+                                         : (size_t)di.sms * kDecodeWarps;
+  return counters + 2 * chunks * slot;
+}
+
+int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_stream_t stream) {
+  if (!workspace && workspace_bytes) return PQKV_ERR_ARG;
+  if (!workspace_bytes) return PQKV_OK;
+  return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? PQKV_OK
+             : PQKV_ERR_CUDA;
+}
+
+int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads, const void* cache,
+                                const void* scales, const void* outliers_idx, const void* outliers_val,
+                                int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                                float scale, int split_blocks, void* out, void* workspace,
+                                size_t workspace_bytes, int32_t* err_flag, pqkv_stream_t stream) {
+  if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
+  if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
+  if (batch < 0 || batch > PQKV_MAX_BATCH || num_kv_heads < 1 || num_q_heads < 1 ||
+      num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > 8 || (head_dim != 64 && head_dim != 128) ||
+      num_blocks < 1 || max_blocks_per_seq < 1 || split_blocks < 0)
+    return PQKV_ERR_ARG;
+  if (batch == 0) return PQKV_OK;
+  if (!q || !cache || !block_tables || !seq_lens || !out || !workspace || !err_flag) return PQKV_ERR_ARG;
+  if (!is_16(kv_dtype) && !scales) return PQKV_ERR_ARG;
+  if (kv_dtype == PQKV_DTYPE_FP4_E2M1 && (!outliers_idx || !outliers_val)) return PQKV_ERR_ARG;
+  if (!aligned16(cache) || (scales && !aligned16(scales)) || (outliers_idx && !aligned16(outliers_idx)) ||
+      (outliers_val && !aligned16(outliers_val)) || !aligned16(q) || !aligned16(out))
+    return PQKV_ERR_ARG;
+  // flat block indices and TMA row coordinates must fit in int32
+  if ((int64_t)batch * num_kv_heads * max_blocks_per_seq >= INT32_MAX ||
+      (int64_t)num_blocks * num_kv_heads * 32 >= INT32_MAX)
+    return PQKV_ERR_ARG;
+  const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                                                  split_blocks);
+  if (need == 0 || workspace_bytes < need) return PQKV_ERR_ARG;
+  DeviceInfo di;
+  if (!device_info(di)) return PQKV_ERR_CUDA;
+  if (decode_smem_bytes(kv_dtype, head_dim, batch) > (size_t)di.max_smem) return PQKV_ERR_ARG;
+  CUtensorMap tmap;
+  if (!cached_cache_map(&tmap, cache, kv_dtype, num_blocks, num_kv_heads, head_dim)) return PQKV_ERR_CUDA;
+  DecodeParams p;
+  p.q = q;
+  p.out = out;
+  p.scales = static_cast<const uint8_t*>(scales);
+  p.oidx = static_cast<const uint8_t*>(outliers_idx);
+  p.oval = static_cast<const uint8_t*>(outliers_val);
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.err = err_flag;
+  p.counters = static_cast<int32_t*>(workspace);
+  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                        round_up((size_t)batch * num_kv_heads * 4, 256));
+  p.B = batch;
+  p.Hq = num_q_heads;
+  p.Hkv = num_kv_heads;
+  p.G = num_q_heads / num_kv_heads;
+  p.nb = num_blocks;
+  p.maxblk = max_blocks_per_seq;
+  p.split_blocks = split_blocks;
+  p.slot_floats = (int)round_up((size_t)p.G * head_dim + 2 * p.G, 4);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  const cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms,
+                                      reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+int pqkv_encode(const float* x, int64_t n, int code_dtype, uint8_t* codes, pqkv_stream_t stream) {
+  if (n < 0 || (n > 0 && (!x || !codes))) return PQKV_ERR_ARG;
+  if (code_dtype != PQKV_DTYPE_FP8_E4M3 && code_dtype != PQKV_DTYPE_FP8_E5M2 && code_dtype != PQKV_DTYPE_FP4_E2M1)
+    return PQKV_ERR_ARG;
+  const cudaError_t e = launch_encode(code_dtype, x, n, codes, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,229 @@
+// common.cuh -- device helpers shared by the cache-write and decode kernels:
+// inline-PTX wrappers for sm_100a (mbarrier, TMA bulk / tensor copies,
+// FP8 / E2M1 conversions, warp-level MMA) and the cache geometry.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/pqkv.h"
+
+namespace pqkv {
+
+constexpr int kBlock = PQKV_BLOCK_SIZE;          // tokens per cache block
+constexpr int kGroup = PQKV_FP4_GROUP;           // channels per FP4 scale
+constexpr int kOutSlots = PQKV_FP4_OUTLIER_SLOTS;
+constexpr int kIdxStride = PQKV_FP4_IDX_STRIDE;
+
+// Bytes of one K (or V) row of one token in the cache.
+__host__ __device__ constexpr int row_bytes(int kv_dtype, int D) {
+  return (kv_dtype == PQKV_DTYPE_FP16 || kv_dtype == PQKV_DTYPE_BF16) ? 2 * D
+         : (kv_dtype == PQKV_DTYPE_FP4_E2M1)                          ? D / 2
+                                                                      : D;
+}
+
+// ---------------------------------------------------------------------------
+// error flag
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_flag(int32_t* err, int bits) { atomicOr(err, bits); }
+
+// ---------------------------------------------------------------------------
+// small float conversions (hardware cvt, round to nearest even, satfinite)
+// ---------------------------------------------------------------------------
+
+// Two floats -> two E4M3 / E5M2 codes, `lo` in the low byte. A zero result
+// keeps the sign of its input (the cache stores -0 as sign bit + zero).
+template <int KVF>
+__device__ __forceinline__ uint32_t enc_fp8x2(float lo, float hi) {
+  uint16_t r;
+  if constexpr (KVF == PQKV_DTYPE_FP8_E4M3)
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  else
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  uint32_t c = r;
+  if ((c & 0x7Fu) == 0) c = (c & ~0xFFu) | ((__float_as_uint(lo) >> 24) & 0x80u);
+  if ((c & 0x7F00u) == 0) c = (c & 0xFFu) | ((__float_as_uint(hi) >> 16) & 0x8000u);
+  return c;
+}
+
+// Two floats -> two E2M1 codes packed in one byte, `lo` in the low nibble.
+__device__ __forceinline__ uint32_t enc_e2m1x2(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  if ((r & 0x7u) == 0) r = (r & 0xF0u) | ((__float_as_uint(lo) >> 28) & 0x8u);
+  if ((r & 0x70u) == 0) r = (r & 0x0Fu) | ((__float_as_uint(hi) >> 24) & 0x80u);
+  return r;
+}
+
+// Two FP8 codes (low byte first) -> f16x2 (exact).
+template <int KVF>
+__device__ __forceinline__ uint32_t dec_fp8x2(uint32_t two_codes) {
+  uint32_t r;
+  uint16_t c = (uint16_t)two_codes;
+  if constexpr (KVF == PQKV_DTYPE_FP8_E4M3)
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(c));
+  else
+    asm("cvt.rn.f16x2.e5m2x2 %0, %1;" : "=r"(r) : "h"(c));
+  return r;
+}
+
+// Two E2M1 codes in one byte (low nibble first) -> f16x2 (exact).
+__device__ __forceinline__ uint32_t dec_e2m1x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+  return r;
+}
+
+__device__ __forceinline__ float lo_half(uint32_t h2) {
+  return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
+}
+__device__ __forceinline__ float hi_half(uint32_t h2) {
+  return __half2float(__ushort_as_half((unsigned short)(h2 >> 16)));
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier + TMA (cp.async.bulk) wrappers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait until the phase with `parity` of `bar` completes, giving up after
+// `limit_ns` nanoseconds. Returns false on timeout.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// 2-D tiled TMA load of box {x .. x+box0, y .. y+box1} into shared memory.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Untiled bulk copy of `bytes` (multiple of 16, both addresses 16-byte aligned).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// warp-level matrix helpers
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+  return r;
+}
+
+// D += A * B, m16n8k16, fp32 accumulate. IS_BF16 selects bf16 vs f16 operands.
+template <bool IS_BF16>
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  if constexpr (IS_BF16)
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f32x2(float lo, float hi, bool bf16) {
+  if (bf16) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+  __half2 v = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float unpack_lo(uint32_t v, bool bf16) {
+  return bf16 ? __uint_as_float(v << 16) : __half2float(__ushort_as_half((unsigned short)(v & 0xFFFFu)));
+}
+__device__ __forceinline__ float unpack_hi(uint32_t v, bool bf16) {
+  return bf16 ? __uint_as_float(v & 0xFFFF0000u) : __half2float(__ushort_as_half((unsigned short)(v >> 16)));
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t r;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+  return r;
+}
+
+
+}  // namespace pqkv

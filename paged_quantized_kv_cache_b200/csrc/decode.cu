@@ -1,0 +1,767 @@
+// decode.cu -- the paged decode-attention kernel (see decode.cuh for the design).
+#include <atomic>
+#include <cfloat>
+
+#include "decode.cuh"
+
+namespace pqkv {
+
+namespace {
+
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+// Zero the low (token t0) / high (token t0 + 1) half of a packed pair when the
+// token lies past the end of the sequence (its bytes may hold anything).
+__device__ __forceinline__ uint32_t mask_pair(uint32_t v, int t0, int valid) {
+  if (t0 >= valid) v &= 0xFFFF0000u;
+  if (t0 + 1 >= valid) v &= 0x0000FFFFu;
+  return v;
+}
+
+__device__ __forceinline__ uint32_t f16x2_from(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <bool QBF16>
+__device__ __forceinline__ float q_at(const void* q, size_t i) {
+  if constexpr (QBF16)
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(q)[i]);
+  else
+    return __half2float(reinterpret_cast<const __half*>(q)[i]);
+}
+
+template <bool QBF16>
+__device__ __forceinline__ void store_out(void* out, size_t i, float v) {
+  if constexpr (QBF16)
+    reinterpret_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
+}
+
+// Row `rr` (0..15) of output m-tile `mt` -> head-dimension index. The order
+// of d inside a tile follows how each format's dequantization lays out the
+// V^T fragment (see the PV steps below).
+template <int KVF>
+__device__ __forceinline__ int dmap(int mt, int rr) {
+  if constexpr (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16) {
+    return 16 * mt + rr;
+  } else if constexpr (KVF == PQKV_DTYPE_FP4_E2M1) {
+    // tiles (2c, 2c+1) cover d in [32c, 32c + 32): tile 2c+e, row g -> 32c + 4g + 2e,
+    // row g + 8 -> 32c + 4g + 2e + 1
+    const int c = mt >> 1, e = mt & 1;
+    return 32 * c + 4 * (rr & 7) + 2 * e + (rr >> 3);
+  } else {
+    // FP8: tile c covers [16c, 16c + 16): row g -> 16c + 2g, row g + 8 -> 16c + 2g + 1
+    return 16 * mt + 2 * (rr & 7) + (rr >> 3);
+  }
+}
+
+}  // namespace
+
+template <int KVF, int D, bool QBF16>
+__global__ void __launch_bounds__(kDecodeWarps * 32, 1)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
+  using Gm = DecodeGeom<KVF, D>;
+  using Sm = DecodeSmem<KVF, D>;
+  constexpr int NS = Gm::kStages;
+  constexpr int KT = D / 16;  // k-steps of QK^T and m-tiles of PV
+  constexpr bool kBf16Mma = (KVF == PQKV_DTYPE_BF16);
+  constexpr float kNegInf = -INFINITY;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* tiles = smem;
+  uint8_t* sides = tiles + Sm::kTilesBytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sides + Sm::kSideBytes);
+  uint16_t* qcopy = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(bars) + Sm::kBarBytes);
+  int* P = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(qcopy) + Sm::kQBytes);
+  __shared__ int warp_sums[kDecodeWarps];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int B = p.B, Hkv = p.Hkv, G = p.G, Hq = p.Hq;
+  const int g = lane >> 2, qd = lane & 3;
+  uint64_t* wbar = bars + warp * NS;
+  uint8_t* wtile = tiles + warp * NS * Gm::kTile;
+  uint8_t* wside = sides + warp * NS * Gm::kSideStride;
+  uint16_t* wq = qcopy + warp * 8 * D;
+
+  if (lane == 0) {
+    for (int s = 0; s < NS; ++s) mbar_init(&wbar[s], 1);
+    fence_mbar_init();
+  }
+  if (tid == 0) prefetch_tensormap(&tmap);
+
+  // ---- prefix sums of blocks per sequence: P[b] = sum of ceil(L/16) below b ----
+  {
+    const int nthr = blockDim.x;
+    const int per = (B + nthr - 1) / nthr;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    const int lim = kBlock * p.maxblk;
+    int local = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      const bool bad = (L < 0 || L > lim);
+      if (bad && blockIdx.x == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
+      local += bad ? 0 : (L + kBlock - 1) / kBlock;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < warp; ++w) run += warp_sums[w];
+    if (tid == 0) P[0] = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      const bool bad = (L < 0 || L > lim);
+      run += bad ? 0 : (L + kBlock - 1) / kBlock;
+      P[i + 1] = run;
+    }
+  }
+  __syncthreads();
+
+  // ---- sequences without blocks (empty or rejected): zero output rows ----
+  for (int b = blockIdx.x; b < B; b += gridDim.x) {
+    if (P[b + 1] != P[b]) continue;
+    for (int i = tid; i < Hq * D; i += blockDim.x) store_out<QBF16>(p.out, (size_t)b * Hq * D + i, 0.f);
+  }
+
+  const int T = Hkv * P[B];
+  const int W = gridDim.x * kDecodeWarps;
+  const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + W - 1) / W);
+  const int K = T > 0 ? (T + Qc - 1) / Qc : 0;
+
+  uint32_t phase = 0;      // parity bit per stage
+  uint32_t inflight = 0;   // stages with an issued, unconsumed copy
+  bool aborted = false;
+
+  // flat block index -> (b, h, j) of its (sequence, head, block)
+  auto locate = [&](int f, int& b, int& h, int& j) {
+    int lo = 0, hi = B;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (Hkv * P[mid] <= f) lo = mid; else hi = mid;
+    }
+    const int n = P[lo + 1] - P[lo];
+    const int rel = f - Hkv * P[lo];
+    b = lo;
+    h = rel / n;
+    j = rel - h * n;
+  };
+
+  for (int k = warp * gridDim.x + blockIdx.x; k < K && !aborted; k += W) {
+    const int f0 = k * Qc;
+    const int f1 = min(T, f0 + Qc);
+
+    // Per-lane window of TMA row coordinates: lane l holds flat block wbase + l.
+    auto load_coord = [&](int f) -> int {
+      if (f >= f1) return -2;
+      int b, h, j;
+      locate(f, b, h, j);
+      const int id = __ldg(p.block_tables + (size_t)b * p.maxblk + j);
+      if (id < 0 || id >= p.nb) {
+        raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
+        return -1;
+      }
+      return (id * Hkv + h) * 32;
+    };
+    int wbase = f0;
+    int wcur = load_coord(f0 + lane);
+    int wnxt = load_coord(f0 + 32 + lane);
+    auto coord_of = [&](int f) -> int {
+      while (f - wbase >= 32) {
+        wbase += 32;
+        wcur = wnxt;
+        wnxt = load_coord(wbase + 32 + lane);
+      }
+      return __shfl_sync(kFull, wcur, f - wbase);
+    };
+    uint32_t skip = 0;
+    auto issue = [&](int s, int coord) {
+      inflight |= 1u << s;
+      if (coord < 0) skip |= 1u << s; else skip &= ~(1u << s);
+      if (lane == 0) {
+        uint64_t* bar = &wbar[s];
+        if (coord < 0) {
+          mbar_arrive(bar);
+        } else {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          mbar_arrive_expect_tx(bar, Gm::kTx);
+          uint8_t* dst = wtile + s * Gm::kTile;
+          constexpr int kElem = Gm::k16 ? 2 : 1;
+#pragma unroll
+          for (int bx = 0; bx < Gm::kBoxes; ++bx)
+            tma_load_2d(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar);
+          const size_t pair = (size_t)(coord >> 5);
+          uint8_t* side = wside + s * Gm::kSideStride;
+          if constexpr (Gm::kFp8) {
+            bulk_load(side, p.scales + pair * 16, 16, bar);
+          } else if constexpr (Gm::kFp4) {
+            bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, bar);
+            bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, bar);
+            bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, bar);
+          }
+        }
+      }
+    };
+
+    const int npre = min(NS, f1 - f0);
+    for (int i = 0; i < npre; ++i) issue(i, coord_of(f0 + i));
+
+    // ---- consumer state of the current (sequence, head) piece ----
+    int b, h, j;
+    locate(f0, b, h, j);
+    int nblk = P[b + 1] - P[b];
+    int Lb = p.seq_lens[b];
+    bool started_before = j > 0;
+    uint32_t qf[KT][2];
+    float acc[KT][4];
+    float m0, m1, l0, l1, vref;
+
+    auto begin_piece = [&]() {
+      m0 = m1 = kNegInf;
+      l0 = l1 = 0.f;
+      vref = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+      const size_t qrow = ((size_t)b * Hq + (size_t)h * G + g) * D;
+      const bool has = g < G;
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk) {
+        if constexpr (Gm::k16) {
+          const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
+          qf[kk][0] = has ? __ldg(q32 + (qrow + 16 * kk + 2 * qd) / 2) : 0u;
+          qf[kk][1] = has ? __ldg(q32 + (qrow + 16 * kk + 8 + 2 * qd) / 2) : 0u;
+        } else {
+          // k-slot order of the dequantized K fragments: FP8 k-step kk holds
+          // d = 16kk + 4qd + {0,1 | 2,3}; FP4 k-step (c, s) = (kk/2, kk%2) holds
+          // d = 32c + 8qd + 4s + {0,1 | 2,3}.
+          const int d0 = Gm::kFp8 ? 16 * kk + 4 * qd : 32 * (kk >> 1) + 8 * qd + 4 * (kk & 1);
+          float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
+          if (has) {
+            v0 = q_at<QBF16>(p.q, qrow + d0);
+            v1 = q_at<QBF16>(p.q, qrow + d0 + 1);
+            v2 = q_at<QBF16>(p.q, qrow + d0 + 2);
+            v3 = q_at<QBF16>(p.q, qrow + d0 + 3);
+          }
+          qf[kk][0] = f16x2_from(v0, v1);
+          qf[kk][1] = f16x2_from(v2, v3);
+        }
+      }
+      if constexpr (Gm::kFp4) {
+        // f16 copy of this warp's query rows for the outlier channels
+        __syncwarp();
+        for (int i = lane; i < 8 * D; i += 32) {
+          const int n = i / D;
+          const float v = (n < G) ? q_at<QBF16>(p.q, ((size_t)b * Hq + (size_t)h * G + n) * D + (i % D)) : 0.f;
+          wq[i] = __half_as_ushort(__float2half_rn(v));
+        }
+        __syncwarp();
+      }
+    };
+
+    auto merge = [&](int k0, int k1) {
+      constexpr int DPL = D / 32;
+      float M[8], Ls[8], o[8][DPL];
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        M[n] = kNegInf;
+        Ls[n] = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) o[n][e] = 0.f;
+      }
+      for (int kk = k0; kk <= k1; ++kk) {
+        const float* base = p.partials + (size_t)(kk == k0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
+#pragma unroll
+        for (int n = 0; n < 8; ++n)
+          if (n < G) M[n] = fmaxf(M[n], __ldcg(base + G * D + n));
+      }
+      for (int kk = k0; kk <= k1; ++kk) {
+        const float* base = p.partials + (size_t)(kk == k0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+          if (n >= G) continue;
+          const float mj = __ldcg(base + G * D + n);
+          const float w = (M[n] == kNegInf) ? 0.f : exp2f(mj - M[n]);
+          Ls[n] += w * __ldcg(base + G * D + G + n);
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) o[n][e] += w * __ldcg(base + n * D + lane * DPL + e);
+        }
+      }
+#pragma unroll
+      for (int n = 0; n < 8; ++n) {
+        if (n >= G) continue;
+        const float inv = Ls[n] > 0.f ? 1.f / Ls[n] : 0.f;
+        const size_t orow = ((size_t)b * Hq + (size_t)h * G + n) * D + lane * DPL;
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, o[n][e] * inv);
+      }
+    };
+
+    auto finish_piece = [&](bool ends_after) {
+      float lt0 = l0, lt1 = l1;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) {
+        lt0 += __shfl_xor_sync(kFull, lt0, o);
+        lt1 += __shfl_xor_sync(kFull, lt1, o);
+      }
+      const float vs = Gm::kFp8 ? vref : 1.f;
+      const int n0 = 2 * qd, n1 = 2 * qd + 1;
+      if (!started_before && !ends_after) {
+        const float i0 = lt0 > 0.f ? vs / lt0 : 0.f;
+        const float i1 = lt1 > 0.f ? vs / lt1 : 0.f;
+        const size_t ob = ((size_t)b * Hq + (size_t)h * G) * D;
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) {
+          const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
+          if (n0 < G) {
+            store_out<QBF16>(p.out, ob + (size_t)n0 * D + da, acc[mt][0] * i0);
+            store_out<QBF16>(p.out, ob + (size_t)n0 * D + db, acc[mt][2] * i0);
+          }
+          if (n1 < G) {
+            store_out<QBF16>(p.out, ob + (size_t)n1 * D + da, acc[mt][1] * i1);
+            store_out<QBF16>(p.out, ob + (size_t)n1 * D + db, acc[mt][3] * i1);
+          }
+        }
+        return;
+      }
+      const int slot = started_before ? 2 * k : 2 * k + 1;
+      float* base = p.partials + (size_t)slot * p.slot_floats;
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt) {
+        const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
+        if (n0 < G) {
+          base[n0 * D + da] = acc[mt][0] * vs;
+          base[n0 * D + db] = acc[mt][2] * vs;
+        }
+        if (n1 < G) {
+          base[n1 * D + da] = acc[mt][1] * vs;
+          base[n1 * D + db] = acc[mt][3] * vs;
+        }
+      }
+      if (g == 0) {
+        if (n0 < G) {
+          base[G * D + n0] = m0;
+          base[G * D + G + n0] = lt0;
+        }
+        if (n1 < G) {
+          base[G * D + n1] = m1;
+          base[G * D + G + n1] = lt1;
+        }
+      }
+      __syncwarp();
+      __threadfence();
+      const int s0 = Hkv * P[b] + h * nblk;
+      const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
+      int last = 0;
+      if (lane == 0) {
+        int* ctr = p.counters + (size_t)b * Hkv + h;
+        const int prev = atomicAdd(ctr, 1);
+        last = (prev == k1 - k0);
+        if (last) atomicExch(ctr, 0);
+      }
+      last = __shfl_sync(kFull, last, 0);
+      if (last) {
+        __threadfence();
+        merge(k0, k1);
+      }
+    };
+
+    begin_piece();
+    int s = 0;
+    for (int f = f0; f < f1; ++f) {
+      const bool ok = __all_sync(kFull, mbar_wait_bounded(&wbar[s], (phase >> s) & 1u, p.timeout_ns));
+      phase ^= 1u << s;
+      inflight &= ~(1u << s);
+      if (!ok) {
+        if (lane == 0) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+        aborted = true;
+        break;
+      }
+      const int valid = min(kBlock, Lb - kBlock * j);
+      if (!((skip >> s) & 1u)) {
+        const uint32_t tb = smem_u32(wtile + s * Gm::kTile);
+        const uint8_t* side = wside + s * Gm::kSideStride;
+        const int mi = lane >> 3, ri = lane & 7;
+        float sk = 1.f, sv = 1.f;
+        if constexpr (Gm::kFp8) {
+          sk = reinterpret_cast<const float*>(side)[0];
+          sv = reinterpret_cast<const float*>(side)[1];
+        }
+
+        // ---- S^T = K Q^T (16 tokens x 8 query heads) ----
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (Gm::k16) {
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk) {
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * kk + (mi >> 1)) * 16), a0, a1, a2, a3);
+            mma16816<kBf16Mma>(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+          }
+        } else if constexpr (Gm::kFp8) {
+          // ldmatrix on byte data: lane (g, qd) receives bytes 4qd..4qd+3 of a
+          // token row's 16-byte chunk, i.e. 4 consecutive d of one k-step.
+#pragma unroll
+          for (int cp = 0; cp < KT / 2; ++cp) {
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
+            mma16816<false>(sc, dec_fp8x2<KVF>(r0), dec_fp8x2<KVF>(r1), dec_fp8x2<KVF>(r0 >> 16),
+                            dec_fp8x2<KVF>(r1 >> 16), qf[2 * cp][0], qf[2 * cp][1]);
+            mma16816<false>(sc, dec_fp8x2<KVF>(r2), dec_fp8x2<KVF>(r3), dec_fp8x2<KVF>(r2 >> 16),
+                            dec_fp8x2<KVF>(r3 >> 16), qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+          }
+        } else {
+          // FP4: one 16-byte chunk = 32 d; lane (g, qd) receives 8 codes
+          // d = 32c + 8qd .. +7 of token rows g and g + 8 and multiplies them by
+          // the token's E4M3 scale of group 2c + qd/2 (exact in f16).
+          const uint32_t* srow = reinterpret_cast<const uint32_t*>(side);  // K scales [16][D/16]
+          constexpr int SPR = D / 16;                                       // scale bytes per token
+          uint32_t s_lo, s_hi;  // scale codes of this lane's groups, tokens g and g+8
+          {
+            const uint8_t* sb = side;
+            uint32_t ca = 0, cb = 0;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              ca |= (uint32_t)sb[g * SPR + 2 * c + (qd >> 1)] << (8 * c);
+              cb |= (uint32_t)sb[(g + 8) * SPR + 2 * c + (qd >> 1)] << (8 * c);
+            }
+            s_lo = ca;
+            s_hi = cb;
+            (void)srow;
+          }
+#pragma unroll
+          for (int cp = 0; cp < D / 64; ++cp) {
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
+            const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int c = 2 * cp + e;
+              const uint32_t sca = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_lo >> (8 * c)) & 0xFFu);
+              const uint32_t scb = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_hi >> (8 * c)) & 0xFFu);
+              const __half2 sa = __low2half2(*reinterpret_cast<const __half2*>(&sca));
+              const __half2 sb2 = __low2half2(*reinterpret_cast<const __half2*>(&scb));
+              uint32_t ha[4], hb[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                uint32_t x = dec_e2m1x2((rr[e][0] >> (8 * i)) & 0xFFu);
+                uint32_t y = dec_e2m1x2((rr[e][1] >> (8 * i)) & 0xFFu);
+                __half2 xa = __hmul2(*reinterpret_cast<__half2*>(&x), sa);
+                __half2 yb = __hmul2(*reinterpret_cast<__half2*>(&y), sb2);
+                ha[i] = *reinterpret_cast<uint32_t*>(&xa);
+                hb[i] = *reinterpret_cast<uint32_t*>(&yb);
+              }
+              mma16816<false>(sc, ha[0], hb[0], ha[1], hb[1], qf[2 * c][0], qf[2 * c][1]);
+              mma16816<false>(sc, ha[2], hb[2], ha[3], hb[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
+            }
+          }
+          // outlier channels: S^T += Kout (16 tokens x R) * Qout^T (R x n)
+          {
+            const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;  // K idx [8]
+            const uint16_t* kv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);  // K vals [16][4]
+            uint32_t a0 = 0, a1 = 0, b0 = 0;
+            if (qd < 2) {
+              const int r0i = idx[2 * qd], r1i = idx[2 * qd + 1];
+              a0 = (uint32_t)kv[g * 4 + 2 * qd] | ((uint32_t)kv[g * 4 + 2 * qd + 1] << 16);
+              a1 = (uint32_t)kv[(g + 8) * 4 + 2 * qd] | ((uint32_t)kv[(g + 8) * 4 + 2 * qd + 1] << 16);
+              const uint32_t q0 = (r0i < D) ? wq[g * D + r0i] : 0u;
+              const uint32_t q1 = (r1i < D) ? wq[g * D + r1i] : 0u;
+              b0 = q0 | (q1 << 16);
+              if (r0i >= D) { a0 &= 0xFFFF0000u; a1 &= 0xFFFF0000u; }
+              if (r1i >= D) { a0 &= 0x0000FFFFu; a1 &= 0x0000FFFFu; }
+            }
+            mma16816<false>(sc, a0, a1, 0u, 0u, b0, 0u);
+          }
+        }
+
+        // ---- online softmax over this block (log2 domain) ----
+        const float mult = p.scale_log2 * sk;
+        float x0 = sc[0] * mult, x1 = sc[1] * mult, x2 = sc[2] * mult, x3 = sc[3] * mult;
+        if (g >= valid) x0 = x1 = kNegInf;
+        if (g + 8 >= valid) x2 = x3 = kNegInf;
+        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
+          bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
+        }
+        const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+        const float al0 = (mn0 == kNegInf) ? 1.f : exp2f(m0 - mn0);
+        const float al1 = (mn1 == kNegInf) ? 1.f : exp2f(m1 - mn1);
+        const float p0 = (mn0 == kNegInf) ? 0.f : exp2f(x0 - mn0);
+        const float p2 = (mn0 == kNegInf) ? 0.f : exp2f(x2 - mn0);
+        const float p1 = (mn1 == kNegInf) ? 0.f : exp2f(x1 - mn1);
+        const float p3 = (mn1 == kNegInf) ? 0.f : exp2f(x3 - mn1);
+        l0 = l0 * al0 + p0 + p2;
+        l1 = l1 * al1 + p1 + p3;
+        m0 = mn0;
+        m1 = mn1;
+
+        // FP8 V scale: O is kept in units of vref = largest V scale so far; a
+        // block with a smaller scale enters with P scaled by sv / vref <= 1.
+        float f0c = al0, f1c = al1, pr = 1.f;
+        bool do_pv = true;
+        if constexpr (Gm::kFp8) {
+          if (sv > vref) {
+            const float rs = vref / sv;
+            f0c *= rs;
+            f1c *= rs;
+            vref = sv;
+          } else if (sv > 0.f) {
+            pr = sv / vref;
+          } else {
+            do_pv = false;
+          }
+        }
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) {
+          acc[mt][0] *= f0c;
+          acc[mt][1] *= f1c;
+          acc[mt][2] *= f0c;
+          acc[mt][3] *= f1c;
+        }
+
+        if (do_pv) {
+          // P = P_hi + P_lo, each rounded to the MMA operand type, so the
+          // probabilities keep ~16 significant bits through the PV product.
+          uint32_t b0, b1, c0, c1;
+          {
+            const float w0 = p0 * pr, w1 = p1 * pr, w2 = p2 * pr, w3 = p3 * pr;
+            const uint32_t pA = pack_f32x2(w0, w1, kBf16Mma);
+            const uint32_t pB = pack_f32x2(w2, w3, kBf16Mma);
+            const uint32_t lA = pack_f32x2(w0 - unpack_lo(pA, kBf16Mma), w1 - unpack_hi(pA, kBf16Mma), kBf16Mma);
+            const uint32_t lB = pack_f32x2(w2 - unpack_lo(pB, kBf16Mma), w3 - unpack_hi(pB, kBf16Mma), kBf16Mma);
+            b0 = movmatrix_t(pA);
+            b1 = movmatrix_t(pB);
+            c0 = movmatrix_t(lA);
+            c1 = movmatrix_t(lB);
+          }
+          auto mma_pv = [&](float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+            mma16816<kBf16Mma>(d, a0, a1, a2, a3, b0, b1);
+            mma16816<kBf16Mma>(d, a0, a1, a2, a3, c0, c1);
+          };
+          const int t0 = 2 * qd, t1 = 2 * qd + 8;
+
+          // ---- O^T += V^T P^T ----
+          if constexpr (Gm::k16) {
+#pragma unroll
+            for (int mt = 0; mt < KT; ++mt) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_t(tb + Gm::off(16 + ((mi >> 1) << 3) + ri, (2 * mt + (mi & 1)) * 16), a0, a1, a2, a3);
+              if (valid < kBlock) {
+                a0 = mask_pair(a0, t0, valid);
+                a1 = mask_pair(a1, t0, valid);
+                a2 = mask_pair(a2, t1, valid);
+                a3 = mask_pair(a3, t1, valid);
+              }
+              mma_pv(acc[mt], a0, a1, a2, a3);
+            }
+          } else if constexpr (Gm::kFp8) {
+            // ldmatrix.trans on byte data: lane (g, qd) receives d0 = 16c + 2g and
+            // d0 + 1 of tokens 2qd and 2qd + 1; one byte permute pairs the tokens.
+#pragma unroll
+            for (int cp = 0; cp < KT / 2; ++cp) {
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4_t(tb + Gm::off(16 + ((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
+              const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const uint32_t xa = prmt(rr[e][0], 0u, 0x3120u);
+                const uint32_t xb = prmt(rr[e][1], 0u, 0x3120u);
+                uint32_t a0 = dec_fp8x2<KVF>(xa), a1 = dec_fp8x2<KVF>(xa >> 16);
+                uint32_t a2 = dec_fp8x2<KVF>(xb), a3 = dec_fp8x2<KVF>(xb >> 16);
+                if (valid < kBlock) {
+                  a0 = mask_pair(a0, t0, valid);
+                  a1 = mask_pair(a1, t0, valid);
+                  a2 = mask_pair(a2, t1, valid);
+                  a3 = mask_pair(a3, t1, valid);
+                }
+                mma_pv(acc[2 * cp + e], a0, a1, a2, a3);
+              }
+            }
+          } else {
+            // FP4: ldmatrix.trans gives lane (g, qd) the codes d0 = 32c + 4g .. +3
+            // of tokens 2qd, 2qd + 1; a nibble transpose pairs the tokens per d.
+            constexpr int SPR = D / 16;
+            const uint8_t* vs = side + 16 * SPR;  // V scales [16][D/16]
+            const int gs = g >> 2;
+            uint32_t sp[2][D / 32];  // scale pairs (tokens t, t+1) per chunk c, f16x2
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              const int ta = 2 * qd + 8 * hh;
+#pragma unroll
+              for (int c = 0; c < D / 32; ++c) {
+                const uint32_t two = (uint32_t)vs[ta * SPR + 2 * c + gs] | ((uint32_t)vs[(ta + 1) * SPR + 2 * c + gs] << 8);
+                sp[hh][c] = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(two);
+              }
+            }
+#pragma unroll
+            for (int cp = 0; cp < D / 64; ++cp) {
+              uint32_t r0, r1, r2, r3;
+              ldsm_x4_t(tb + Gm::off(16 + ((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
+              const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int c = 2 * cp + e;
+                uint32_t fa[4], fb[4];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                  const uint32_t x = rr[e][hh];
+                  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+                  const uint32_t A = prmt(lo, hi, 0x5140u), Bv = prmt(lo, hi, 0x7362u);
+                  const uint32_t nib = A | (Bv << 4);  // bytes: d0, d0+1, d0+2, d0+3 (token pair)
+                  const __half2 scl = *reinterpret_cast<const __half2*>(&sp[hh][c]);
+                  uint32_t* dst = hh ? fb : fa;
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    uint32_t v = dec_e2m1x2((nib >> (8 * i)) & 0xFFu);
+                    __half2 w = __hmul2(*reinterpret_cast<__half2*>(&v), scl);
+                    dst[i] = *reinterpret_cast<uint32_t*>(&w);
+                  }
+                }
+                if (valid < kBlock) {
+#pragma unroll
+                  for (int i = 0; i < 4; ++i) {
+                    fa[i] = mask_pair(fa[i], t0, valid);
+                    fb[i] = mask_pair(fb[i], t1, valid);
+                  }
+                }
+                // tile 2c: rows g -> d0, g+8 -> d0+1; tile 2c+1: rows g -> d0+2, g+8 -> d0+3
+                mma_pv(acc[2 * c], fa[0], fa[1], fb[0], fb[1]);
+                mma_pv(acc[2 * c + 1], fa[2], fa[3], fb[2], fb[3]);
+              }
+            }
+            // outlier channels: O^T[idx_r] += Vout^T (R x 16 tokens) P^T
+            {
+              const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes + 8;             // V idx
+              const uint16_t* vv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes + 128);  // V vals
+              uint32_t a0 = 0, a2 = 0;
+              if (g < 4) {
+                a0 = (uint32_t)vv[t0 * 4 + g] | ((uint32_t)vv[(t0 + 1) * 4 + g] << 16);
+                a2 = (uint32_t)vv[t1 * 4 + g] | ((uint32_t)vv[(t1 + 1) * 4 + g] << 16);
+                if (valid < kBlock) {
+                  a0 = mask_pair(a0, t0, valid);
+                  a2 = mask_pair(a2, t1, valid);
+                }
+              }
+              float ex[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_pv(ex, a0, 0u, a2, 0u);
+              // ex[0], ex[1]: slot r = g (g < 4), query heads 2qd, 2qd+1
+#pragma unroll
+              for (int r = 0; r < kOutSlots; ++r) {
+                const int dch = idx[r];
+                const float e0 = __shfl_sync(kFull, ex[0], r * 4 + qd);
+                const float e1 = __shfl_sync(kFull, ex[1], r * 4 + qd);
+                if (dch >= D) continue;  // warp-uniform
+                const int c = dch >> 5, rem = dch & 31;
+                const int tile = 2 * c + ((rem & 3) >> 1), half = rem & 1;
+                if (g == (rem >> 2)) {
+#pragma unroll
+                  for (int mt = 0; mt < KT; ++mt) {
+                    if (mt == tile) {
+                      acc[mt][2 * half] += e0;
+                      acc[mt][2 * half + 1] += e1;
+                    }
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+      __syncwarp();
+      if (f + NS < f1) issue(s, coord_of(f + NS));
+      s = (s + 1 == NS) ? 0 : s + 1;
+
+      // ---- advance through (sequence, head, block) ----
+      ++j;
+      const bool seg_end = (j == nblk);
+      const bool chunk_end = (f + 1 == f1);
+      if (seg_end || chunk_end) {
+        finish_piece(!seg_end);
+        if (!chunk_end) {
+          j = 0;
+          if (++h == Hkv) {
+            h = 0;
+            do { ++b; } while (P[b + 1] == P[b]);
+            nblk = P[b + 1] - P[b];
+            Lb = p.seq_lens[b];
+          }
+          started_before = false;
+          begin_piece();
+        }
+      }
+    }
+  }
+
+  // after a timeout: let copies still in flight land before the CTA exits
+  if (aborted) {
+    for (int s2 = 0; s2 < NS; ++s2)
+      if ((inflight >> s2) & 1u) (void)mbar_wait_bounded(&wbar[s2], (phase >> s2) & 1u, p.timeout_ns);
+  }
+}
+
+// ---- instantiation + launch --------------------------------------------------
+
+template <int KVF, int D, bool QBF16>
+static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& p, int grid, cudaStream_t st) {
+  auto kern = paged_decode_kernel<KVF, D, QBF16>;
+  const size_t smem = DecodeSmem<KVF, D>::bytes(p.B);
+  // opt in once per device to the largest size any batch can need
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)DecodeSmem<KVF, D>::bytes(PQKV_MAX_BATCH));
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  kern<<<grid, kDecodeWarps * 32, smem, st>>>(tmap, p);
+  return cudaGetLastError();
+}
+
+size_t decode_smem_bytes(int kv_dtype, int D, int B) {
+  switch (kv_dtype) {
+    case PQKV_DTYPE_FP16:
+    case PQKV_DTYPE_BF16:
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_BF16, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_BF16, 64>::bytes(B);
+    case PQKV_DTYPE_FP8_E4M3:
+    case PQKV_DTYPE_FP8_E5M2:
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP8_E4M3, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_FP8_E4M3, 64>::bytes(B);
+    default:
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP4_E2M1, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_FP4_E2M1, 64>::bytes(B);
+  }
+}
+
+cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap, const DecodeParams& p,
+                          int grid, cudaStream_t st) {
+#define PQKV_DEC(KVF, DD, QB) \
+  if (kv_dtype == KVF && D == DD && q_bf16 == QB) return launch_decode_t<KVF, DD, QB>(tmap, p, grid, st);
+  PQKV_DEC(PQKV_DTYPE_FP16, 128, false)
+  PQKV_DEC(PQKV_DTYPE_FP16, 64, false)
+  PQKV_DEC(PQKV_DTYPE_BF16, 128, true)
+  PQKV_DEC(PQKV_DTYPE_BF16, 64, true)
+  PQKV_DEC(PQKV_DTYPE_FP8_E4M3, 128, true)
+  PQKV_DEC(PQKV_DTYPE_FP8_E4M3, 128, false)
+  PQKV_DEC(PQKV_DTYPE_FP8_E4M3, 64, true)
+  PQKV_DEC(PQKV_DTYPE_FP8_E4M3, 64, false)
+  PQKV_DEC(PQKV_DTYPE_FP8_E5M2, 128, true)
+  PQKV_DEC(PQKV_DTYPE_FP8_E5M2, 128, false)
+  PQKV_DEC(PQKV_DTYPE_FP8_E5M2, 64, true)
+  PQKV_DEC(PQKV_DTYPE_FP8_E5M2, 64, false)
+  PQKV_DEC(PQKV_DTYPE_FP4_E2M1, 128, true)
+  PQKV_DEC(PQKV_DTYPE_FP4_E2M1, 128, false)
+  PQKV_DEC(PQKV_DTYPE_FP4_E2M1, 64, true)
+  PQKV_DEC(PQKV_DTYPE_FP4_E2M1, 64, false)
+#undef PQKV_DEC
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pqkv

@@ -1,0 +1,96 @@
+// decode.cuh -- split-K paged decode attention with in-register dequantization
+// and log-sum-exp merge, for sm_100a.
+//
+// Method ("vLLM 0.7 Ships Unified KV Cache Compression": architecture diagram
+// "Flash-Decoding Kernel" and step 4, "Flash-Decoding kernels fuse the outlier
+// and compressed representations"; "vLLM" glossary, "PagedAttention"):
+// every (sequence, KV head) pair reads its KV blocks through the block table,
+// the KV range is split across the GPU, each piece keeps an online softmax
+// (running max m, sum l, unnormalized output O) and the pieces of one pair are
+// merged by log-sum-exp.
+//
+// Work decomposition. The blocks of all (sequence b, KV head h) pairs are laid
+// end to end (b-major, then h, then block j) into one flat range of T blocks.
+// The grid is persistent (one CTA per SM, NW warps each); the flat range is cut
+// into chunks of Q blocks and warp w takes chunks w, w + W, ... (W = all warps).
+// A chunk covers whole pairs (written straight to `out`) and at most two
+// partial pairs at its ends (written to a workspace slot). The warp that
+// completes the last piece of a pair (an atomic counter per pair) merges the
+// pieces in chunk order, so results do not depend on timing.
+//
+// Per warp: a private ring of NS shared-memory stages, each holding the K and V
+// tiles of one (block, head) pair fetched by one TMA tensor copy (128/64/32-byte
+// swizzle so ldmatrix reads are conflict-free) plus small bulk copies of the
+// block's scales and outlier buffer. Lane 0 issues the copies NS blocks ahead.
+// GQA: the G = Hq/Hkv query heads of a KV head are the N = 8 columns of
+// m16n8k16 MMAs: S^T = K Q^T (M = 16 tokens of one block) and O^T += V^T P^T
+// (M = 16 head dims per tile, K = 16 tokens). Dequantization happens in
+// registers between ldmatrix and the MMA.
+#pragma once
+
+#include "common.cuh"
+
+namespace pqkv {
+
+constexpr int kDecodeWarps = 8;
+
+struct DecodeParams {
+  const void* q;
+  void* out;
+  const uint8_t* scales;        // FP8: float [nb][H][4]; FP4: u8 [nb][H][2][16][D/16]
+  const uint8_t* oidx;          // FP4: u8 [nb][H][2][8]
+  const uint8_t* oval;          // FP4: fp16 [nb][H][2][16][4]
+  const int32_t* block_tables;  // [B][maxblk]
+  const int32_t* seq_lens;      // [B]
+  int32_t* err;
+  int32_t* counters;            // [B * Hkv], zero between calls
+  float* partials;              // [2 * chunks][slot_floats]
+  int B, Hq, Hkv, G, nb, maxblk;
+  int split_blocks;
+  int slot_floats;
+  float scale_log2;             // softmax scale * log2(e)
+  uint64_t timeout_ns;
+};
+
+// Compile-time geometry of one format.
+template <int KVF, int D>
+struct DecodeGeom {
+  static constexpr bool k16 = (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16);
+  static constexpr bool kFp8 = (KVF == PQKV_DTYPE_FP8_E4M3 || KVF == PQKV_DTYPE_FP8_E5M2);
+  static constexpr bool kFp4 = (KVF == PQKV_DTYPE_FP4_E2M1);
+  static constexpr int kRow = row_bytes(KVF, D);               // bytes per token row
+  static constexpr int kBoxRow = kRow > 128 ? 128 : kRow;       // bytes per TMA box row
+  static constexpr int kBoxes = kRow / kBoxRow;                 // TMA boxes per tile
+  static constexpr int kTile = 32 * kRow;                       // K (16 rows) + V (16 rows)
+  static constexpr int kScaleBytes = kFp8 ? 16 : (kFp4 ? 2 * 16 * (D / 16) : 0);
+  static constexpr int kValBytes = kFp4 ? 2 * 16 * 4 * 2 : 0;
+  static constexpr int kIdxBytes = kFp4 ? 16 : 0;
+  static constexpr int kSide = kScaleBytes + kValBytes + kIdxBytes;  // multiple of 16
+  static constexpr int kSideStride = kSide == 0 ? 0 : ((kSide + 127) / 128) * 128;
+  static constexpr int kStages = k16 ? (D == 128 ? 3 : 5) : (kFp8 ? (D == 128 ? 5 : 8) : (D == 128 ? 8 : 10));
+  static constexpr uint32_t kTx = kTile + kSide;
+  // byte offset in a tile of (row r, byte b of that row); rows 0-15 K, 16-31 V.
+  __device__ static __forceinline__ uint32_t off(int r, int b) {
+    const int box = b / kBoxRow;
+    const int inner = b % kBoxRow;
+    int chunk = inner >> 4;
+    if constexpr (kBoxRow == 128) chunk ^= (r & 7);
+    else if constexpr (kBoxRow == 64) chunk ^= ((r >> 1) & 3);
+    else chunk ^= ((r >> 2) & 1);
+    return (uint32_t)(box * 32 * kBoxRow + r * kBoxRow + (chunk << 4) + (inner & 15));
+  }
+};
+
+template <int KVF, int D>
+struct DecodeSmem {
+  using Gm = DecodeGeom<KVF, D>;
+  static constexpr int kTilesBytes = kDecodeWarps * Gm::kStages * Gm::kTile;
+  static constexpr int kSideBytes = kDecodeWarps * Gm::kStages * Gm::kSideStride;
+  static constexpr int kBarBytes = kDecodeWarps * Gm::kStages * 8;
+  static constexpr int kQBytes = Gm::kFp4 ? kDecodeWarps * 8 * D * 2 : 0;  // per-warp f16 q copy
+  static size_t bytes(int B) {
+    return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + (size_t)(B + 1) * 4;
+  }
+};
+
+}  // namespace pqkv
