@@ -1,0 +1,584 @@
+#!/usr/bin/env python
+"""Benchmark of the paged, quantized KV-cache decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--kv-dtype bf16|fp16|fp8_e4m3|fp8_e5m2|fp4] [--impl ours|reference]
+
+One step = one decode step of one attention layer over the whole batch:
+kv_cache_write of one new token per sequence, then paged_decode_attention of
+every sequence over its cache (the write, the split-K decode and its
+log-sum-exp merge). Inputs are seeded synthetic data of the workload's shapes,
+resident in HBM when timing starts. Prints one JSON line (rank 0).
+
+N > 1 (torchrun, one process per GPU): every rank runs its own replica of the
+workload (weak scaling, no collective on the data path); the timed region is
+bracketed by barriers and the time taken is the maximum over ranks.
+
+--impl reference times the CPU oracle (the fp64 restatement used by the tests)
+on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "paged decode-attn KV GB/s (frac of B200 HBM peak); decode tok/s per layer"
+UNIT = "GB/s"
+KV_NAMES = {"fp16": W.DT_FP16, "bf16": W.DT_BF16, "fp8_e4m3": W.DT_FP8_E4M3, "fp8_e5m2": W.DT_FP8_E5M2,
+            "fp4": W.DT_FP4}
+DT_LABEL = {W.DT_FP16: "fp16", W.DT_BF16: "bf16", W.DT_FP8_E4M3: "fp8_e4m3", W.DT_FP8_E5M2: "fp8_e5m2",
+            W.DT_FP4: "fp4_e2m1"}
+DESCR = {
+    "tiny": "tiny decode step: 4 seqs, ctx {17,33,64,100}, 8 q / 2 kv heads, head_dim 64, fp16 KV",
+    "llama8b": "Llama-3-8B-shaped decode layer: 64 seqs, ctx U[512,4096], 32 q / 8 kv heads, head_dim 128, "
+               "block 16, random blocks of a 40k-block pool",
+    "fp8": "Llama-3-8B-shaped decode layer, FP8 KV with per-block-per-head absmax scales: 128 seqs, "
+           "ctx U[1024,8192]",
+    "llama70b": "Llama-3.1-70B-shaped layer: 16 seqs, ctx U[24576,40960], 64 q / 8 kv heads, head_dim 128, "
+                "seqs 0-3 share a 4096-token prefix",
+    "fp4": "FP4 E2M1 KV with 3.2-sigma fp16 outlier channels: 256 seqs, ctx log-uniform [1024,65536], "
+           "32 q / 8 kv heads, head_dim 128, prefill written in 512-token chunks",
+}
+L2_BYTES = 126 * 1024 * 1024
+
+
+# ---------------------------------------------------------------------------
+# workload on the device
+# ---------------------------------------------------------------------------
+
+def bench_spec(name: str, kv_name: str | None) -> W.Spec:
+    s = W.spec(name, kv_dtype=KV_NAMES[kv_name] if kv_name else None)
+    s.append_tokens = 1  # every step appends one token per sequence
+    if s.kv_dtype in (W.DT_FP16, W.DT_BF16):
+        s.q_dtype = s.kv_dtype  # 16-bit caches take queries of their own type
+    return s
+
+
+def per_token_bytes(s: W.Spec) -> int:
+    """Algorithmic KV bytes of one token (all KV heads, K and V, with its share of
+    the scales / outlier buffers of the cache layout)."""
+    H, D = s.num_kv_heads, s.head_dim
+    if s.kv_dtype in (W.DT_FP16, W.DT_BF16):
+        return H * 2 * D * 2
+    if s.kv_dtype in (W.DT_FP8_E4M3, W.DT_FP8_E5M2):
+        return H * 2 * D + H * 16 // 16
+    return H * 2 * (D // 2 + D // 16 + 4 * 2) + H * 16 // 16
+
+
+def generate_kv(s: W.Spec, seqs, threads: int = 0, ahead: int = 8):
+    """Yield seq_kv(s, b) for b in seqs, in order, computed by a few threads ahead."""
+    import concurrent.futures as cf
+    seqs = list(seqs)
+    threads = threads or max(1, min(16, (os.cpu_count() or 2) - 1))
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        futs = {}
+        for i, b in enumerate(seqs):
+            for jj in range(i, min(len(seqs), i + ahead)):
+                if jj not in futs:
+                    futs[jj] = ex.submit(W.seq_kv, s, seqs[jj])
+            yield futs.pop(i).result()
+
+
+class Setup:
+    """Cache prefilled with the workload, plus one decode step's inputs, on `device`."""
+
+    def __init__(self, s: W.Spec, device, split_blocks: int):
+        import paged_quantized_kv_cache_b200 as pq
+        self.pq = pq
+        self.s = s
+        self.device = device
+        tab = W.tables(s)
+        self.tab = tab
+        self.lens0 = W.seq_lens(s)
+        self.lens = W.decode_lens(s)
+        self.cache = pq.allocate_cache(s.kv_dtype, tab.num_blocks, s.num_kv_heads, s.head_dim, device=device,
+                                       fill=0xFF)
+        self.err = torch.zeros(1, dtype=torch.int32, device=device)
+        in_dt = W.TORCH_DTYPE[W.input_dtype(s)]
+        # prefill: generate per sequence on the host (seeded, a few threads
+        # ahead), write with the GPU in the workload's write-call sizes
+        newk, newv = [], []
+        for b, (k, v) in enumerate(generate_kv(s, range(s.batch))):
+            k = k.to(in_dt)
+            v = v.to(in_dt)
+            L0 = int(self.lens0[b])
+            lo = s.shared_prefix_tokens if (0 < b < s.shared_prefix_seqs) else 0
+            kd, vd = k.to(device), v.to(device)
+            step = s.chunk_tokens or L0
+            for c0 in range(lo, L0, step):
+                c1 = min(L0, c0 + step)
+                sl = torch.from_numpy(W.slots_for(tab.block_tables[b], c0, c1 - c0)).to(device)
+                pq.kv_cache_write(kd[c0:c1].contiguous(), vd[c0:c1].contiguous(), sl, self.cache, self.err)
+            newk.append(k[L0:L0 + 1])
+            newv.append(v[L0:L0 + 1])
+        torch.cuda.synchronize(device)
+        if int(self.err.item()) != 0:
+            raise RuntimeError("prefill raised device error bits %d" % int(self.err.item()))
+        self.k_new = torch.cat(newk).contiguous()
+        self.v_new = torch.cat(newv).contiguous()
+        self.slots_new = np.array([W.slots_for(tab.block_tables[b], int(self.lens0[b]), 1)[0]
+                                   for b in range(s.batch)], np.int32)
+        self.q = W.query(s)
+        self.split_blocks = split_blocks
+        self.scale = W.softmax_scale(s)
+        # The step's inputs (q, new k / v, slots, block tables, lengths) live in
+        # one packed buffer so the end-to-end leg moves them with one copy.
+        parts = [("q", self.q), ("k", self.k_new), ("v", self.v_new),
+                 ("slots", torch.from_numpy(self.slots_new)), ("bt", torch.from_numpy(tab.block_tables)),
+                 ("lens", torch.from_numpy(self.lens))]
+        offs, total = {}, 0
+        for name, t in parts:
+            offs[name] = total
+            total += (t.numel() * t.element_size() + 255) // 256 * 256
+        self.h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
+        self.d_in = torch.empty(total, dtype=torch.uint8, device=device)
+        views = {}
+        for name, t in parts:
+            n = t.numel() * t.element_size()
+            self.h_in[offs[name]:offs[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
+            views[name] = self.d_in[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+        self.d_in.copy_(self.h_in)
+        self.d_q, self.d_k, self.d_v = views["q"], views["k"], views["v"]
+        self.d_slots, self.d_bt, self.d_lens = views["slots"], views["bt"], views["lens"]
+        self.h2d_bytes = sum(t.numel() * t.element_size() for _, t in parts)
+        self.d_out = torch.empty_like(self.d_q)
+        self.ws = pq.decode_workspace(s.batch, s.num_q_heads, s.num_kv_heads, s.head_dim, tab.max_blocks,
+                                      split_blocks, device=device)
+
+    def write(self):
+        self.pq.kv_cache_write(self.d_k, self.d_v, self.d_slots, self.cache, self.err)
+
+    def decode(self):
+        self.pq.paged_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale, self.d_out,
+                                       self.ws, self.err, split_blocks=self.split_blocks)
+
+    def unique_tokens(self) -> int:
+        s = self.s
+        tot = int(self.lens.sum())
+        if s.shared_prefix_seqs:
+            tot -= s.shared_prefix_tokens * (min(s.shared_prefix_seqs, s.batch) - 1)
+        return tot
+
+    def step_bytes(self) -> dict:
+        s = self.s
+        kv = self.unique_tokens() * per_token_bytes(s)
+        qo = 2 * s.batch * s.num_q_heads * s.head_dim * 2
+        tables = int(sum(W.nblocks(int(L)) for L in self.lens)) * 4 + s.batch * 4
+        return {"kv": kv, "q_out": qo, "tables": tables, "decode_total": kv + qo + tables}
+
+
+# ---------------------------------------------------------------------------
+# clocks (NVML, sampled during the timed region)
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+        "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index: int, period_s: float = 0.01):
+        self.ok = False
+        self.samples = []
+        self.reasons = 0
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+
+    def _sample_once(self):
+        self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+        try:
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            r = self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        self.reasons |= int(r) & ~0x1
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample_once()
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+        if self.ok and len(self.samples) < 3:
+            for _ in range(3):
+                try:
+                    self._sample_once()
+                except Exception:
+                    pass
+
+    def summary(self) -> dict:
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"]}
+        names = [n for n, bit in self.REASONS.items() if self.reasons & bit]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("decode.cu", "decode.cuh", "common.cuh"):
+        with open(os.path.join(ROOT, "paged_quantized_kv_cache_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(workload: str, kv_name: str) -> int | None:
+    """DRAM bytes per decode launch from a committed ncu summary, if it was
+    taken from the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "decode_traffic_%s_%s.txt" % (workload, kv_name))
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    for line in open(p):
+        if "=" in line and not line.startswith("#"):
+            k, v = line.strip().split("=", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_hash") != decode_source_hash():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reference arm and cpu_baseline)
+# ---------------------------------------------------------------------------
+
+class OracleSample:
+    """The oracle's decode (gather through the tables, dequantize, fp64
+    attention) over a bounded sample of the workload's sequences, with the
+    sample's cache written by the oracle itself."""
+
+    def __init__(self, s: W.Spec, nseq: int):
+        import oracle
+        self.oracle = oracle
+        self.s = s
+        lens = W.decode_lens(s)
+        tab = W.tables(s)
+        order = [int(i) for i in np.argsort(lens, kind="stable")]
+        # a spread of lengths: shortest, longest, then alternating inwards
+        pick, lo, hi = [], 0, len(order) - 1
+        while lo <= hi:
+            pick.append(order[lo]); lo += 1
+            if lo <= hi:
+                pick.append(order[hi]); hi -= 1
+        sample = sorted(pick[:max(1, min(nseq, len(pick)))])
+        need = sum(W.nblocks(int(lens[b])) for b in sample)
+        self.c = oracle.Cache(s.kv_dtype, need, s.num_kv_heads, s.head_dim)
+        self.bt = np.full((len(sample), tab.max_blocks), -1, np.int32)
+        nxt = 0
+        for i, b in enumerate(sample):
+            nb = W.nblocks(int(lens[b]))
+            self.bt[i, :nb] = np.arange(nxt, nxt + nb, dtype=np.int32)
+            nxt += nb
+            k, v = W.seq_kv(s, b)
+            L = int(lens[b])
+            step = s.chunk_tokens or L
+            for c0 in range(0, L, step):
+                c1 = min(L, c0 + step)
+                oracle.kv_cache_write(self.c, k[c0:c1].contiguous(), v[c0:c1].contiguous(),
+                                      W.slots_for(self.bt[i], c0, c1 - c0))
+        self.q = W.query(s)[sample].contiguous()
+        self.lens = lens[sample].astype(np.int32)
+        self.sample = sample
+        self.tokens = int(self.lens.sum())
+
+    def step(self):
+        self.oracle.paged_decode(self.c, self.q, self.bt, self.lens, W.softmax_scale(self.s))
+
+    def describe(self, reps: int, per: float) -> str:
+        return ("%d of %d sequences (%d tokens, lengths %d..%d); oracle decode (gather, dequantize, fp64 "
+                "attention) timed %d times, %.3f s each" % (len(self.sample), self.s.batch, self.tokens,
+                                                            int(self.lens.min()), int(self.lens.max()), reps, per))
+
+
+def oracle_baseline(s: W.Spec, budget_s: float, nseq: int) -> dict:
+    """cpu_baseline: the oracle as it stands, timed for about budget_s seconds."""
+    o = OracleSample(s, nseq)
+    t_total, reps = 0.0, 0
+    while reps < 1 or (t_total < budget_s and reps < 100):
+        t0 = time.perf_counter()
+        o.step()
+        t_total += time.perf_counter() - t0
+        reps += 1
+    per = t_total / reps
+    return {"value": o.tokens * per_token_bytes(s) / per / 1e9, "unit": UNIT, "cores": o.oracle.num_threads(),
+            "kind": "oracle", "sample": o.describe(reps, per)}
+
+
+def run_reference(args) -> None:
+    """The oracle on the host cores, same metric and workload; each step is the
+    oracle decode over a sample small enough for W + K steps to take minutes."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    s = bench_spec(args.workload, args.kv_dtype)
+    nseq = args.ref_seqs
+    budget = 150.0
+    while True:
+        o = OracleSample(s, nseq)
+        t0 = time.perf_counter()
+        o.step()
+        one = time.perf_counter() - t0
+        if (args.steps + args.warmup) * one <= budget or nseq == 1:
+            break
+        nseq = max(1, nseq // 2)
+    for _ in range(args.warmup):
+        o.step()
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        o.step()
+        times.append(time.perf_counter() - t0)
+    per = statistics.mean(times)
+    value = o.tokens * per_token_bytes(s) / per / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(args, s, None),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.oracle.num_threads(), "kind": "oracle",
+                         "sample": o.describe(args.steps, per)},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_dict(args, s: W.Spec, st: Setup | None) -> dict:
+    d = {"workload": args.workload + ": " + DESCR[args.workload] + "; KV " + DT_LABEL[s.kv_dtype] +
+         "; step = append 1 token per sequence + paged decode", "batch": s.batch,
+         "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
+         "block_size": 16, "kv_dtype": DT_LABEL[s.kv_dtype], "split_blocks": args.split_blocks,
+         "parallelism": "replicas (one independent batch per GPU)"}
+    if st is not None:
+        b = st.step_bytes()
+        d["context_tokens"] = int(st.lens.sum())
+        d["kv_bytes_per_step"] = b["kv"]
+        d["l2"] = ("inputs larger than L2: %.0f MB of KV read per step vs 126 MB L2; no flush"
+                   % (b["kv"] / 1e6)) if b["kv"] > 2 * L2_BYTES else \
+            "KV smaller than L2 (%.1f MB): numbers include L2 hits" % (b["kv"] / 1e6)
+    return d
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+
+def run_ours(args) -> None:
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    s = bench_spec(args.workload, args.kv_dtype)
+    st = Setup(s, device, args.split_blocks)
+    stream = torch.cuda.current_stream(device)
+
+    for _ in range(max(args.warmup, 3)):
+        st.write()
+        st.decode()
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    e0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        st.write()
+        ev[i][1].record(stream)
+        st.decode()
+        ev[i][2].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    clocks.stop()
+    barrier(world)
+    if int(st.err.item()) != 0:
+        raise RuntimeError("device error bits %d during the timed steps" % int(st.err.item()))
+    total_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    ms_step = total_ms / K
+    dec_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
+    wr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+
+    b = st.step_bytes()
+    value = b["kv"] * world / (ms_step * 1e-3) / 1e9
+    tok_s = s.batch * world / (ms_step * 1e-3)
+    peaks = measured_peaks()
+    achieved = b["decode_total"] / (dec_ms * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"],
+                "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype]),
+                "kernel": "paged_decode_kernel", "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, "
+                "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms}
+
+    e2e = run_e2e(st, args, world) if not args.no_e2e else None
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = oracle_baseline(s, args.cpu_budget, args.ref_seqs)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if s.kv_dtype == W.DT_BF16 else ("fp16" if s.kv_dtype == W.DT_FP16 else
+                                                             DT_LABEL[s.kv_dtype] + "->f16"),
+            "data": "synthetic", "config": config_dict(args, s, st),
+            "frac_of_hbm_peak": value / world / peaks["hbm_gbs"],
+            "frac_of_8tbs_spec": value / world / 8000.0,
+            "decode_tok_s_per_layer": tok_s,
+            "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * K, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_e2e(st: Setup, args, world: int) -> dict:
+    """Same step through the public API from pinned host buffers: copy the
+    step's inputs in (q, the new tokens' k / v, slots, block tables, lengths),
+    write + decode, copy the output back, every step."""
+    dev = st.device
+    stream = torch.cuda.current_stream(dev)
+    h_out = torch.empty(st.d_out.shape, dtype=st.d_out.dtype).pin_memory()
+    h2d = st.h2d_bytes
+    d2h = h_out.numel() * h_out.element_size()
+
+    def step():
+        st.d_in.copy_(st.h_in, non_blocking=True)
+        st.write()
+        st.decode()
+        h_out.copy_(st.d_out, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    K = max(1, args.steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+    b = st.step_bytes()
+    return {"value": b["kv"] * world / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(DESCR), default="llama8b")
+    ap.add_argument("--kv-dtype", choices=sorted(KV_NAMES), default=None)
+    ap.add_argument("--split-blocks", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle timing")
+    ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.ref_seqs is None:
+        args.ref_seqs = {"tiny": 4, "llama8b": 16, "fp8": 16, "llama70b": 4, "fp4": 16}[args.workload]
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -9,6 +9,11 @@ namespace pqkv {
 namespace {
 
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr float kNegInf = -INFINITY;
+// The running max m is only moved (and O, l rescaled) when a block's max
+// exceeds it by more than this many log2 units, so most blocks skip the
+// rescale; probabilities then stay below 2^kLazy, well inside f16 / bf16.
+constexpr float kLazy = 8.f;
 
 // Zero the low (token t0) / high (token t0 + 1) half of a packed pair when the
 // token lies past the end of the sequence (its bytes may hold anything).
@@ -21,6 +26,13 @@ __device__ __forceinline__ uint32_t mask_pair(uint32_t v, int t0, int valid) {
 __device__ __forceinline__ uint32_t f16x2_from(float a, float b) {
   __half2 h = __floats2half2_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// 2^x with the hardware approximation (relative error ~2^-22, denormal results flushed).
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 template <bool QBF16>
@@ -39,9 +51,49 @@ __device__ __forceinline__ void store_out(void* out, size_t i, float v) {
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
+// Four FP8 codes of a word -> f16x2 of bytes (0,1) and of bytes (2,3), exact.
+// E5M2 codes are the high byte of the binary16 of the same value, so they are
+// placed, not converted.
+template <int KVF>
+__device__ __forceinline__ void dec4(uint32_t r, uint32_t& lo, uint32_t& hi) {
+  if constexpr (KVF == PQKV_DTYPE_FP8_E5M2) {
+    lo = prmt(r, 0u, 0x1404u);
+    hi = prmt(r, 0u, 0x3424u);
+  } else {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(r));
+  }
+}
+
+// Per-lane shared-memory offsets (bytes, within a stage) of the ldmatrix rows
+// of one block: K reads of k-step group i and V reads of m-tile group i. The
+// swizzle depends on the lane, so these are computed once per kernel.
+template <int KVF, int D>
+struct LdsmOffsets {
+  using Gm = DecodeGeom<KVF, D>;
+  // 16-bit: one x4 per 16 head dims; FP8: per 32 dims; FP4: per 64 dims
+  static constexpr int kN = Gm::k16 ? D / 16 : (Gm::kFp8 ? D / 32 : D / 64);
+  uint32_t k[kN], v[kN];
+  __device__ __forceinline__ explicit LdsmOffsets(int lane) {
+    const int mi = lane >> 3, ri = lane & 7;
+#pragma unroll
+    for (int i = 0; i < kN; ++i) {
+      if constexpr (Gm::k16) {
+        k[i] = Gm::off(((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
+        v[i] = Gm::off(16 + ((mi >> 1) << 3) + ri, (2 * i + (mi & 1)) * 16);
+      } else {
+        k[i] = Gm::off(((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
+        v[i] = Gm::off(16 + ((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
+      }
+    }
+  }
+};
+
 // Row `rr` (0..15) of output m-tile `mt` -> head-dimension index. The order
 // of d inside a tile follows how each format's dequantization lays out the
-// V^T fragment (see the PV steps below).
+// V^T fragment (see block_pv).
 template <int KVF>
 __device__ __forceinline__ int dmap(int mt, int rr) {
   if constexpr (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16) {
@@ -57,17 +109,258 @@ __device__ __forceinline__ int dmap(int mt, int rr) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// S^T (16 tokens x 8 query heads) += K Q^T for one block in shared memory.
+// Lane (g, qd) ends with rows (tokens) g, g + 8 and columns (heads) 2qd, 2qd + 1.
+// ---------------------------------------------------------------------------
+template <int KVF, int D>
+__device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, const uint32_t (&qf)[D / 16][2],
+                                             const uint16_t* wq, const LdsmOffsets<KVF, D>& lo, int lane,
+                                             float (&sc)[4]) {
+  using Gm = DecodeGeom<KVF, D>;
+  constexpr int KT = D / 16;
+  const int g = lane >> 2, qd = lane & 3;
+  float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};  // two independent chains
+  if constexpr (Gm::k16) {
+    constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
+#pragma unroll
+    for (int kk = 0; kk < KT; ++kk) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4(tb + lo.k[kk], a0, a1, a2, a3);
+      if (kk & 1) mma16816<kBf>(so, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+      else mma16816<kBf>(se, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+    }
+  } else if constexpr (Gm::kFp8) {
+    // ldmatrix on byte data: lane (g, qd) receives bytes 4qd..4qd+3 of a token
+    // row's 16-byte chunk, i.e. 4 consecutive d of one k-step.
+#pragma unroll
+    for (int cp = 0; cp < KT / 2; ++cp) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4(tb + lo.k[cp], r0, r1, r2, r3);
+      uint32_t x0l, x0h, x1l, x1h, x2l, x2h, x3l, x3h;
+      dec4<KVF>(r0, x0l, x0h);
+      dec4<KVF>(r1, x1l, x1h);
+      dec4<KVF>(r2, x2l, x2h);
+      dec4<KVF>(r3, x3l, x3h);
+      mma16816<false>(se, x0l, x1l, x0h, x1h, qf[2 * cp][0], qf[2 * cp][1]);
+      mma16816<false>(so, x2l, x3l, x2h, x3h, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+    }
+  } else {
+    // FP4: one 16-byte chunk = 32 d; lane (g, qd) receives the 8 codes
+    // d = 32c + 8qd .. +7 of token rows g and g + 8 and multiplies them by the
+    // token's E4M3 scale of group 2c + qd/2 (the product is exact in f16).
+    constexpr int SPR = D / 16;  // scale bytes per token row
+    uint32_t s_lo = 0, s_hi = 0;
+#pragma unroll
+    for (int c = 0; c < D / 32; ++c) {
+      s_lo |= (uint32_t)side[g * SPR + 2 * c + (qd >> 1)] << (8 * c);
+      s_hi |= (uint32_t)side[(g + 8) * SPR + 2 * c + (qd >> 1)] << (8 * c);
+    }
+#pragma unroll
+    for (int cp = 0; cp < D / 64; ++cp) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4(tb + lo.k[cp], r0, r1, r2, r3);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = 2 * cp + e;
+        const uint32_t ra = e ? r2 : r0, rb = e ? r3 : r1;
+        const uint32_t sca = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_lo >> (8 * c)) & 0xFFu);
+        const uint32_t scb = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_hi >> (8 * c)) & 0xFFu);
+        const __half2 sa = __low2half2(*reinterpret_cast<const __half2*>(&sca));
+        const __half2 sb = __low2half2(*reinterpret_cast<const __half2*>(&scb));
+        uint32_t ha[4], hb[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          uint32_t x = dec_e2m1x2((ra >> (8 * i)) & 0xFFu);
+          uint32_t y = dec_e2m1x2((rb >> (8 * i)) & 0xFFu);
+          __half2 xa = __hmul2(*reinterpret_cast<__half2*>(&x), sa);
+          __half2 yb = __hmul2(*reinterpret_cast<__half2*>(&y), sb);
+          ha[i] = *reinterpret_cast<uint32_t*>(&xa);
+          hb[i] = *reinterpret_cast<uint32_t*>(&yb);
+        }
+        mma16816<false>(se, ha[0], hb[0], ha[1], hb[1], qf[2 * c][0], qf[2 * c][1]);
+        mma16816<false>(so, ha[2], hb[2], ha[3], hb[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
+      }
+    }
+    // outlier channels (their codes are 0): S^T += Kout (16 tokens x 4 slots) Qout^T
+    {
+      const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;                      // K idx [8]
+      const uint16_t* kv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);   // K vals [16][4]
+      uint32_t a0 = 0, a1 = 0, b0 = 0;
+      if (qd < 2) {
+        const int r0i = idx[2 * qd], r1i = idx[2 * qd + 1];
+        a0 = (uint32_t)kv[g * 4 + 2 * qd] | ((uint32_t)kv[g * 4 + 2 * qd + 1] << 16);
+        a1 = (uint32_t)kv[(g + 8) * 4 + 2 * qd] | ((uint32_t)kv[(g + 8) * 4 + 2 * qd + 1] << 16);
+        const uint32_t q0 = (r0i < D) ? wq[g * D + r0i] : 0u;
+        const uint32_t q1 = (r1i < D) ? wq[g * D + r1i] : 0u;
+        b0 = q0 | (q1 << 16);
+        if (r0i >= D) { a0 &= 0xFFFF0000u; a1 &= 0xFFFF0000u; }
+        if (r1i >= D) { a0 &= 0x0000FFFFu; a1 &= 0x0000FFFFu; }
+      }
+      mma16816<false>(so, a0, a1, 0u, 0u, b0, 0u);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) sc[i] = se[i] + so[i];
+}
+
+// ---------------------------------------------------------------------------
+// O^T (D x 8 query heads) += V^T P^T for one block. P^T arrives as two B
+// fragments (hi and lo parts, P = P_hi + P_lo rounded to the operand type).
+// ---------------------------------------------------------------------------
+template <int KVF, int D>
+__device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const LdsmOffsets<KVF, D>& lo, int lane,
+                                         int valid, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
+                                         float (&acc)[D / 16][4]) {
+  using Gm = DecodeGeom<KVF, D>;
+  constexpr int KT = D / 16;
+  constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
+  const int g = lane >> 2, qd = lane & 3;
+  const int t0 = 2 * qd, t1 = 2 * qd + 8;
+  auto mma_pv = [&](float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+    mma16816<kBf>(d, a0, a1, a2, a3, b0, b1);
+    mma16816<kBf>(d, a0, a1, a2, a3, c0, c1);
+  };
+  if constexpr (Gm::k16) {
+#pragma unroll
+    for (int mt = 0; mt < KT; ++mt) {
+      uint32_t a0, a1, a2, a3;
+      ldsm_x4_t(tb + lo.v[mt], a0, a1, a2, a3);
+      if (valid < kBlock) {
+        a0 = mask_pair(a0, t0, valid);
+        a1 = mask_pair(a1, t0, valid);
+        a2 = mask_pair(a2, t1, valid);
+        a3 = mask_pair(a3, t1, valid);
+      }
+      mma_pv(acc[mt], a0, a1, a2, a3);
+    }
+  } else if constexpr (Gm::kFp8) {
+    // ldmatrix.trans on byte data: lane (g, qd) receives d0 = 16c + 2g and d0 + 1
+    // of tokens 2qd and 2qd + 1; one byte permute pairs the tokens per d.
+#pragma unroll
+    for (int cp = 0; cp < KT / 2; ++cp) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(tb + lo.v[cp], r0, r1, r2, r3);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const uint32_t xa = prmt(e ? r2 : r0, 0u, 0x3120u);
+        const uint32_t xb = prmt(e ? r3 : r1, 0u, 0x3120u);
+        uint32_t a0, a1, a2, a3;
+        dec4<KVF>(xa, a0, a1);
+        dec4<KVF>(xb, a2, a3);
+        if (valid < kBlock) {
+          a0 = mask_pair(a0, t0, valid);
+          a1 = mask_pair(a1, t0, valid);
+          a2 = mask_pair(a2, t1, valid);
+          a3 = mask_pair(a3, t1, valid);
+        }
+        mma_pv(acc[2 * cp + e], a0, a1, a2, a3);
+      }
+    }
+  } else {
+    // FP4: ldmatrix.trans gives lane (g, qd) the codes d0 = 32c + 4g .. +3 of
+    // tokens 2qd, 2qd + 1; a nibble transpose pairs the tokens per d, and each
+    // pair is multiplied by the two tokens' E4M3 scales of group 2c + g/4.
+    constexpr int SPR = D / 16;
+    const uint8_t* vs = side + 16 * SPR;  // V scales [16][D/16]
+    const int gs = g >> 2;
+    uint32_t sp[2][D / 32];
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const int ta = 2 * qd + 8 * hh;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        const uint32_t two =
+            (uint32_t)vs[ta * SPR + 2 * c + gs] | ((uint32_t)vs[(ta + 1) * SPR + 2 * c + gs] << 8);
+        sp[hh][c] = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(two);
+      }
+    }
+#pragma unroll
+    for (int cp = 0; cp < D / 64; ++cp) {
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(tb + lo.v[cp], r0, r1, r2, r3);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int c = 2 * cp + e;
+        uint32_t fa[4], fb[4];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const uint32_t x = hh ? (e ? r3 : r1) : (e ? r2 : r0);
+          const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
+          const uint32_t A = prmt(lo, hi, 0x5140u), Bv = prmt(lo, hi, 0x7362u);
+          const uint32_t nib = A | (Bv << 4);  // bytes: d0, d0+1, d0+2, d0+3 (token pair)
+          const __half2 scl = *reinterpret_cast<const __half2*>(&sp[hh][c]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t v = dec_e2m1x2((nib >> (8 * i)) & 0xFFu);
+            __half2 w = __hmul2(*reinterpret_cast<__half2*>(&v), scl);
+            if (hh) fb[i] = *reinterpret_cast<uint32_t*>(&w);
+            else fa[i] = *reinterpret_cast<uint32_t*>(&w);
+          }
+        }
+        if (valid < kBlock) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            fa[i] = mask_pair(fa[i], t0, valid);
+            fb[i] = mask_pair(fb[i], t1, valid);
+          }
+        }
+        // tile 2c: rows g -> d0, g+8 -> d0+1; tile 2c+1: rows g -> d0+2, g+8 -> d0+3
+        mma_pv(acc[2 * c], fa[0], fa[1], fb[0], fb[1]);
+        mma_pv(acc[2 * c + 1], fa[2], fa[3], fb[2], fb[3]);
+      }
+    }
+    // outlier channels: O^T[idx_r] += Vout^T (4 slots x 16 tokens) P^T; the
+    // result of slot r sits in lanes 4r..4r+3 and moves to the lanes owning d = idx_r
+    {
+      const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes + 8;                         // V idx
+      const uint16_t* vv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes + 128);    // V vals
+      uint32_t a0 = 0, a2 = 0;
+      if (g < 4) {
+        a0 = (uint32_t)vv[t0 * 4 + g] | ((uint32_t)vv[(t0 + 1) * 4 + g] << 16);
+        a2 = (uint32_t)vv[t1 * 4 + g] | ((uint32_t)vv[(t1 + 1) * 4 + g] << 16);
+        if (valid < kBlock) {
+          a0 = mask_pair(a0, t0, valid);
+          a2 = mask_pair(a2, t1, valid);
+        }
+      }
+      float ex[4] = {0.f, 0.f, 0.f, 0.f};
+      mma_pv(ex, a0, 0u, a2, 0u);
+#pragma unroll
+      for (int r = 0; r < kOutSlots; ++r) {
+        const int dch = idx[r];
+        const float e0 = __shfl_sync(kFull, ex[0], r * 4 + qd);
+        const float e1 = __shfl_sync(kFull, ex[1], r * 4 + qd);
+        if (dch >= D) continue;  // warp-uniform
+        const int c = dch >> 5, rem = dch & 31;
+        const int tile = 2 * c + ((rem & 3) >> 1), half = rem & 1;
+        if (g == (rem >> 2)) {
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            if (mt == tile) {
+              acc[mt][0] += half ? 0.f : e0;
+              acc[mt][1] += half ? 0.f : e1;
+              acc[mt][2] += half ? e0 : 0.f;
+              acc[mt][3] += half ? e1 : 0.f;
+            }
+          }
+        }
+      }
+    }
+  }
+}
+
 }  // namespace
 
 template <int KVF, int D, bool QBF16>
-__global__ void __launch_bounds__(kDecodeWarps * 32, 1)
+__global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
   using Gm = DecodeGeom<KVF, D>;
   using Sm = DecodeSmem<KVF, D>;
+  constexpr int NW = Gm::kWarps;
   constexpr int NS = Gm::kStages;
   constexpr int KT = D / 16;  // k-steps of QK^T and m-tiles of PV
   constexpr bool kBf16Mma = (KVF == PQKV_DTYPE_BF16);
-  constexpr float kNegInf = -INFINITY;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -76,7 +369,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(sides + Sm::kSideBytes);
   uint16_t* qcopy = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(bars) + Sm::kBarBytes);
   int* P = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(qcopy) + Sm::kQBytes);
-  __shared__ int warp_sums[kDecodeWarps];
+  __shared__ int warp_sums[NW];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = p.B, Hkv = p.Hkv, G = p.G, Hq = p.Hq;
@@ -85,6 +378,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
   uint16_t* wq = qcopy + warp * 8 * D;
+  const LdsmOffsets<KVF, D> lofs(lane);
 
   if (lane == 0) {
     for (int s = 0; s < NS; ++s) mbar_init(&wbar[s], 1);
@@ -132,12 +426,12 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
   }
 
   const int T = Hkv * P[B];
-  const int W = gridDim.x * kDecodeWarps;
+  const int W = gridDim.x * NW;
   const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + W - 1) / W);
   const int K = T > 0 ? (T + Qc - 1) / Qc : 0;
 
-  uint32_t phase = 0;      // parity bit per stage
-  uint32_t inflight = 0;   // stages with an issued, unconsumed copy
+  uint32_t phase = 0;     // parity bit per stage
+  uint32_t inflight = 0;  // stages with an issued, unconsumed copy
   bool aborted = false;
 
   // flat block index -> (b, h, j) of its (sequence, head, block)
@@ -158,46 +452,48 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
     const int f0 = k * Qc;
     const int f1 = min(T, f0 + Qc);
 
-    // Per-lane window of TMA row coordinates: lane l holds flat block wbase + l.
-    auto load_coord = [&](int f) -> int {
-      if (f >= f1) return -2;
-      int b, h, j;
-      locate(f, b, h, j);
-      const int id = __ldg(p.block_tables + (size_t)b * p.maxblk + j);
-      if (id < 0 || id >= p.nb) {
-        raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
-        return -1;
+    // Per-lane window of (physical id, head) for flat blocks wbase + lane and,
+    // loaded ahead, wbase + 32 + lane. Values are only inspected when issued.
+    auto load_entry = [&](int f, int& id, int& hh) {
+      id = -1;
+      hh = 0;
+      if (f < f1) {
+        int b, h, j;
+        locate(f, b, h, j);
+        id = __ldg(p.block_tables + (size_t)b * p.maxblk + j);
+        hh = h;
       }
-      return (id * Hkv + h) * 32;
     };
-    int wbase = f0;
-    int wcur = load_coord(f0 + lane);
-    int wnxt = load_coord(f0 + 32 + lane);
-    auto coord_of = [&](int f) -> int {
+    int wbase = f0, wid, wh, nid, nh;
+    load_entry(f0 + lane, wid, wh);
+    load_entry(f0 + 32 + lane, nid, nh);
+    uint32_t skip = 0;
+    auto issue = [&](int s, int f) {
       while (f - wbase >= 32) {
         wbase += 32;
-        wcur = wnxt;
-        wnxt = load_coord(wbase + 32 + lane);
+        wid = nid;
+        wh = nh;
+        load_entry(wbase + 32 + lane, nid, nh);
       }
-      return __shfl_sync(kFull, wcur, f - wbase);
-    };
-    uint32_t skip = 0;
-    auto issue = [&](int s, int coord) {
+      const int id = __shfl_sync(kFull, wid, f - wbase);
+      const int hh = __shfl_sync(kFull, wh, f - wbase);
+      const bool bad = (id < 0 || id >= p.nb);
       inflight |= 1u << s;
-      if (coord < 0) skip |= 1u << s; else skip &= ~(1u << s);
+      if (bad) skip |= 1u << s; else skip &= ~(1u << s);
       if (lane == 0) {
         uint64_t* bar = &wbar[s];
-        if (coord < 0) {
+        if (bad) {
+          raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
           mbar_arrive(bar);
         } else {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          const int coord = (id * Hkv + hh) * 32;
           mbar_arrive_expect_tx(bar, Gm::kTx);
           uint8_t* dst = wtile + s * Gm::kTile;
           constexpr int kElem = Gm::k16 ? 2 : 1;
 #pragma unroll
           for (int bx = 0; bx < Gm::kBoxes; ++bx)
             tma_load_2d(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar);
-          const size_t pair = (size_t)(coord >> 5);
+          const size_t pair = (size_t)id * Hkv + hh;
           uint8_t* side = wside + s * Gm::kSideStride;
           if constexpr (Gm::kFp8) {
             bulk_load(side, p.scales + pair * 16, 16, bar);
@@ -211,7 +507,7 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
     };
 
     const int npre = min(NS, f1 - f0);
-    for (int i = 0; i < npre; ++i) issue(i, coord_of(f0 + i));
+    for (int i = 0; i < npre; ++i) issue(i, f0 + i);
 
     // ---- consumer state of the current (sequence, head) piece ----
     int b, h, j;
@@ -372,152 +668,85 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
       }
     };
 
-    begin_piece();
-    int s = 0;
-    for (int f = f0; f < f1; ++f) {
+    auto wait_stage = [&](int s) -> bool {
       const bool ok = __all_sync(kFull, mbar_wait_bounded(&wbar[s], (phase >> s) & 1u, p.timeout_ns));
       phase ^= 1u << s;
       inflight &= ~(1u << s);
+      return ok;
+    };
+
+    begin_piece();
+    int s = 0;
+    int f = f0;
+    while (f < f1) {
+      // two consecutive blocks of the same piece when available, else one
+      const int n2 = (f + 1 < f1 && j + 1 < nblk) ? 2 : 1;
+      const int sA = s, sB = (s + 1 == NS) ? 0 : s + 1;
+      bool ok = wait_stage(sA);
+      if (n2 == 2) ok = wait_stage(sB) && ok;
       if (!ok) {
         if (lane == 0) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
         aborted = true;
         break;
       }
-      const int valid = min(kBlock, Lb - kBlock * j);
-      if (!((skip >> s) & 1u)) {
-        const uint32_t tb = smem_u32(wtile + s * Gm::kTile);
-        const uint8_t* side = wside + s * Gm::kSideStride;
-        const int mi = lane >> 3, ri = lane & 7;
-        float sk = 1.f, sv = 1.f;
-        if constexpr (Gm::kFp8) {
-          sk = reinterpret_cast<const float*>(side)[0];
-          sv = reinterpret_cast<const float*>(side)[1];
-        }
+      const bool useA = !((skip >> sA) & 1u);
+      const bool useB = (n2 == 2) && !((skip >> sB) & 1u);
+      const int validA = min(kBlock, Lb - kBlock * j);
+      const int validB = min(kBlock, Lb - kBlock * (j + 1));
+      const uint32_t tbA = smem_u32(wtile + sA * Gm::kTile), tbB = smem_u32(wtile + sB * Gm::kTile);
+      const uint8_t* sdA = wside + sA * Gm::kSideStride;
+      const uint8_t* sdB = wside + sB * Gm::kSideStride;
 
-        // ---- S^T = K Q^T (16 tokens x 8 query heads) ----
-        float sc[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (Gm::k16) {
-#pragma unroll
-          for (int kk = 0; kk < KT; ++kk) {
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * kk + (mi >> 1)) * 16), a0, a1, a2, a3);
-            mma16816<kBf16Mma>(sc, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-          }
-        } else if constexpr (Gm::kFp8) {
-          // ldmatrix on byte data: lane (g, qd) receives bytes 4qd..4qd+3 of a
-          // token row's 16-byte chunk, i.e. 4 consecutive d of one k-step.
-#pragma unroll
-          for (int cp = 0; cp < KT / 2; ++cp) {
-            uint32_t r0, r1, r2, r3;
-            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
-            mma16816<false>(sc, dec_fp8x2<KVF>(r0), dec_fp8x2<KVF>(r1), dec_fp8x2<KVF>(r0 >> 16),
-                            dec_fp8x2<KVF>(r1 >> 16), qf[2 * cp][0], qf[2 * cp][1]);
-            mma16816<false>(sc, dec_fp8x2<KVF>(r2), dec_fp8x2<KVF>(r3), dec_fp8x2<KVF>(r2 >> 16),
-                            dec_fp8x2<KVF>(r3 >> 16), qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
-          }
-        } else {
-          // FP4: one 16-byte chunk = 32 d; lane (g, qd) receives 8 codes
-          // d = 32c + 8qd .. +7 of token rows g and g + 8 and multiplies them by
-          // the token's E4M3 scale of group 2c + qd/2 (exact in f16).
-          const uint32_t* srow = reinterpret_cast<const uint32_t*>(side);  // K scales [16][D/16]
-          constexpr int SPR = D / 16;                                       // scale bytes per token
-          uint32_t s_lo, s_hi;  // scale codes of this lane's groups, tokens g and g+8
-          {
-            const uint8_t* sb = side;
-            uint32_t ca = 0, cb = 0;
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              ca |= (uint32_t)sb[g * SPR + 2 * c + (qd >> 1)] << (8 * c);
-              cb |= (uint32_t)sb[(g + 8) * SPR + 2 * c + (qd >> 1)] << (8 * c);
-            }
-            s_lo = ca;
-            s_hi = cb;
-            (void)srow;
-          }
-#pragma unroll
-          for (int cp = 0; cp < D / 64; ++cp) {
-            uint32_t r0, r1, r2, r3;
-            ldsm_x4(tb + Gm::off(((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
-            const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int c = 2 * cp + e;
-              const uint32_t sca = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_lo >> (8 * c)) & 0xFFu);
-              const uint32_t scb = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_hi >> (8 * c)) & 0xFFu);
-              const __half2 sa = __low2half2(*reinterpret_cast<const __half2*>(&sca));
-              const __half2 sb2 = __low2half2(*reinterpret_cast<const __half2*>(&scb));
-              uint32_t ha[4], hb[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                uint32_t x = dec_e2m1x2((rr[e][0] >> (8 * i)) & 0xFFu);
-                uint32_t y = dec_e2m1x2((rr[e][1] >> (8 * i)) & 0xFFu);
-                __half2 xa = __hmul2(*reinterpret_cast<__half2*>(&x), sa);
-                __half2 yb = __hmul2(*reinterpret_cast<__half2*>(&y), sb2);
-                ha[i] = *reinterpret_cast<uint32_t*>(&xa);
-                hb[i] = *reinterpret_cast<uint32_t*>(&yb);
-              }
-              mma16816<false>(sc, ha[0], hb[0], ha[1], hb[1], qf[2 * c][0], qf[2 * c][1]);
-              mma16816<false>(sc, ha[2], hb[2], ha[3], hb[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
-            }
-          }
-          // outlier channels: S^T += Kout (16 tokens x R) * Qout^T (R x n)
-          {
-            const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;  // K idx [8]
-            const uint16_t* kv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);  // K vals [16][4]
-            uint32_t a0 = 0, a1 = 0, b0 = 0;
-            if (qd < 2) {
-              const int r0i = idx[2 * qd], r1i = idx[2 * qd + 1];
-              a0 = (uint32_t)kv[g * 4 + 2 * qd] | ((uint32_t)kv[g * 4 + 2 * qd + 1] << 16);
-              a1 = (uint32_t)kv[(g + 8) * 4 + 2 * qd] | ((uint32_t)kv[(g + 8) * 4 + 2 * qd + 1] << 16);
-              const uint32_t q0 = (r0i < D) ? wq[g * D + r0i] : 0u;
-              const uint32_t q1 = (r1i < D) ? wq[g * D + r1i] : 0u;
-              b0 = q0 | (q1 << 16);
-              if (r0i >= D) { a0 &= 0xFFFF0000u; a1 &= 0xFFFF0000u; }
-              if (r1i >= D) { a0 &= 0x0000FFFFu; a1 &= 0x0000FFFFu; }
-            }
-            mma16816<false>(sc, a0, a1, 0u, 0u, b0, 0u);
-          }
-        }
+      // ---- scores of both blocks (independent MMA chains) ----
+      float scA[4] = {0.f, 0.f, 0.f, 0.f}, scB[4] = {0.f, 0.f, 0.f, 0.f};
+      if (useA) block_scores<KVF, D>(tbA, sdA, qf, wq, lofs, lane, scA);
+      if (useB) block_scores<KVF, D>(tbB, sdB, qf, wq, lofs, lane, scB);
+      float skA = 1.f, skB = 1.f, svA = 1.f, svB = 1.f;
+      if constexpr (Gm::kFp8) {
+        if (useA) { skA = reinterpret_cast<const float*>(sdA)[0]; svA = reinterpret_cast<const float*>(sdA)[1]; }
+        if (useB) { skB = reinterpret_cast<const float*>(sdB)[0]; svB = reinterpret_cast<const float*>(sdB)[1]; }
+      }
 
-        // ---- online softmax over this block (log2 domain) ----
-        const float mult = p.scale_log2 * sk;
-        float x0 = sc[0] * mult, x1 = sc[1] * mult, x2 = sc[2] * mult, x3 = sc[3] * mult;
-        if (g >= valid) x0 = x1 = kNegInf;
-        if (g + 8 >= valid) x2 = x3 = kNegInf;
-        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+      // ---- online softmax over up to 32 tokens (log2 domain) ----
+      const float mA = p.scale_log2 * skA, mB = p.scale_log2 * skB;
+      float xA0 = scA[0] * mA, xA1 = scA[1] * mA, xA2 = scA[2] * mA, xA3 = scA[3] * mA;
+      float xB0 = scB[0] * mB, xB1 = scB[1] * mB, xB2 = scB[2] * mB, xB3 = scB[3] * mB;
+      if (!useA || g >= validA) xA0 = xA1 = kNegInf;
+      if (!useA || g + 8 >= validA) xA2 = xA3 = kNegInf;
+      if (!useB || g >= validB) xB0 = xB1 = kNegInf;
+      if (!useB || g + 8 >= validB) xB2 = xB3 = kNegInf;
+      float bm0 = fmaxf(fmaxf(xA0, xA2), fmaxf(xB0, xB2));
+      float bm1 = fmaxf(fmaxf(xA1, xA3), fmaxf(xB1, xB3));
 #pragma unroll
-        for (int o = 4; o < 32; o <<= 1) {
-          bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
-          bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
+      for (int o = 4; o < 32; o <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
+      }
+      const bool need0 = bm0 > m0 + kLazy, need1 = bm1 > m1 + kLazy;
+      float f0c = 1.f, f1c = 1.f;
+      bool rescale = __any_sync(kFull, need0 || need1);
+      if (rescale) {
+        if (need0) { f0c = ex2(m0 - bm0); m0 = bm0; }
+        if (need1) { f1c = ex2(m1 - bm1); m1 = bm1; }
+        l0 *= f0c;
+        l1 *= f1c;
+      }
+      // FP8 V scales: O is kept in units of vref, the largest V scale so far;
+      // a block with a smaller scale enters with P scaled by sv / vref <= 1.
+      float prA = 1.f, prB = 1.f;
+      if constexpr (Gm::kFp8) {
+        const float svm = fmaxf(useA ? svA : 0.f, useB ? svB : 0.f);
+        if (svm > vref) {
+          const float rs = vref / svm;
+          f0c *= rs;
+          f1c *= rs;
+          vref = svm;
+          rescale = true;
         }
-        const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-        const float al0 = (mn0 == kNegInf) ? 1.f : exp2f(m0 - mn0);
-        const float al1 = (mn1 == kNegInf) ? 1.f : exp2f(m1 - mn1);
-        const float p0 = (mn0 == kNegInf) ? 0.f : exp2f(x0 - mn0);
-        const float p2 = (mn0 == kNegInf) ? 0.f : exp2f(x2 - mn0);
-        const float p1 = (mn1 == kNegInf) ? 0.f : exp2f(x1 - mn1);
-        const float p3 = (mn1 == kNegInf) ? 0.f : exp2f(x3 - mn1);
-        l0 = l0 * al0 + p0 + p2;
-        l1 = l1 * al1 + p1 + p3;
-        m0 = mn0;
-        m1 = mn1;
-
-        // FP8 V scale: O is kept in units of vref = largest V scale so far; a
-        // block with a smaller scale enters with P scaled by sv / vref <= 1.
-        float f0c = al0, f1c = al1, pr = 1.f;
-        bool do_pv = true;
-        if constexpr (Gm::kFp8) {
-          if (sv > vref) {
-            const float rs = vref / sv;
-            f0c *= rs;
-            f1c *= rs;
-            vref = sv;
-          } else if (sv > 0.f) {
-            pr = sv / vref;
-          } else {
-            do_pv = false;
-          }
-        }
+        prA = (useA && vref > 0.f) ? svA / vref : 0.f;
+        prB = (useB && vref > 0.f) ? svB / vref : 0.f;
+      }
+      if (rescale) {
 #pragma unroll
         for (int mt = 0; mt < KT; ++mt) {
           acc[mt][0] *= f0c;
@@ -525,163 +754,39 @@ __global__ void __launch_bounds__(kDecodeWarps * 32, 1)
           acc[mt][2] *= f0c;
           acc[mt][3] *= f1c;
         }
-
-        if (do_pv) {
-          // P = P_hi + P_lo, each rounded to the MMA operand type, so the
-          // probabilities keep ~16 significant bits through the PV product.
-          uint32_t b0, b1, c0, c1;
-          {
-            const float w0 = p0 * pr, w1 = p1 * pr, w2 = p2 * pr, w3 = p3 * pr;
-            const uint32_t pA = pack_f32x2(w0, w1, kBf16Mma);
-            const uint32_t pB = pack_f32x2(w2, w3, kBf16Mma);
-            const uint32_t lA = pack_f32x2(w0 - unpack_lo(pA, kBf16Mma), w1 - unpack_hi(pA, kBf16Mma), kBf16Mma);
-            const uint32_t lB = pack_f32x2(w2 - unpack_lo(pB, kBf16Mma), w3 - unpack_hi(pB, kBf16Mma), kBf16Mma);
-            b0 = movmatrix_t(pA);
-            b1 = movmatrix_t(pB);
-            c0 = movmatrix_t(lA);
-            c1 = movmatrix_t(lB);
-          }
-          auto mma_pv = [&](float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-            mma16816<kBf16Mma>(d, a0, a1, a2, a3, b0, b1);
-            mma16816<kBf16Mma>(d, a0, a1, a2, a3, c0, c1);
-          };
-          const int t0 = 2 * qd, t1 = 2 * qd + 8;
-
-          // ---- O^T += V^T P^T ----
-          if constexpr (Gm::k16) {
-#pragma unroll
-            for (int mt = 0; mt < KT; ++mt) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_t(tb + Gm::off(16 + ((mi >> 1) << 3) + ri, (2 * mt + (mi & 1)) * 16), a0, a1, a2, a3);
-              if (valid < kBlock) {
-                a0 = mask_pair(a0, t0, valid);
-                a1 = mask_pair(a1, t0, valid);
-                a2 = mask_pair(a2, t1, valid);
-                a3 = mask_pair(a3, t1, valid);
-              }
-              mma_pv(acc[mt], a0, a1, a2, a3);
-            }
-          } else if constexpr (Gm::kFp8) {
-            // ldmatrix.trans on byte data: lane (g, qd) receives d0 = 16c + 2g and
-            // d0 + 1 of tokens 2qd and 2qd + 1; one byte permute pairs the tokens.
-#pragma unroll
-            for (int cp = 0; cp < KT / 2; ++cp) {
-              uint32_t r0, r1, r2, r3;
-              ldsm_x4_t(tb + Gm::off(16 + ((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
-              const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const uint32_t xa = prmt(rr[e][0], 0u, 0x3120u);
-                const uint32_t xb = prmt(rr[e][1], 0u, 0x3120u);
-                uint32_t a0 = dec_fp8x2<KVF>(xa), a1 = dec_fp8x2<KVF>(xa >> 16);
-                uint32_t a2 = dec_fp8x2<KVF>(xb), a3 = dec_fp8x2<KVF>(xb >> 16);
-                if (valid < kBlock) {
-                  a0 = mask_pair(a0, t0, valid);
-                  a1 = mask_pair(a1, t0, valid);
-                  a2 = mask_pair(a2, t1, valid);
-                  a3 = mask_pair(a3, t1, valid);
-                }
-                mma_pv(acc[2 * cp + e], a0, a1, a2, a3);
-              }
-            }
-          } else {
-            // FP4: ldmatrix.trans gives lane (g, qd) the codes d0 = 32c + 4g .. +3
-            // of tokens 2qd, 2qd + 1; a nibble transpose pairs the tokens per d.
-            constexpr int SPR = D / 16;
-            const uint8_t* vs = side + 16 * SPR;  // V scales [16][D/16]
-            const int gs = g >> 2;
-            uint32_t sp[2][D / 32];  // scale pairs (tokens t, t+1) per chunk c, f16x2
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-              const int ta = 2 * qd + 8 * hh;
-#pragma unroll
-              for (int c = 0; c < D / 32; ++c) {
-                const uint32_t two = (uint32_t)vs[ta * SPR + 2 * c + gs] | ((uint32_t)vs[(ta + 1) * SPR + 2 * c + gs] << 8);
-                sp[hh][c] = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(two);
-              }
-            }
-#pragma unroll
-            for (int cp = 0; cp < D / 64; ++cp) {
-              uint32_t r0, r1, r2, r3;
-              ldsm_x4_t(tb + Gm::off(16 + ((mi & 1) << 3) + ri, (2 * cp + (mi >> 1)) * 16), r0, r1, r2, r3);
-              const uint32_t rr[2][2] = {{r0, r1}, {r2, r3}};
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int c = 2 * cp + e;
-                uint32_t fa[4], fb[4];
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  const uint32_t x = rr[e][hh];
-                  const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
-                  const uint32_t A = prmt(lo, hi, 0x5140u), Bv = prmt(lo, hi, 0x7362u);
-                  const uint32_t nib = A | (Bv << 4);  // bytes: d0, d0+1, d0+2, d0+3 (token pair)
-                  const __half2 scl = *reinterpret_cast<const __half2*>(&sp[hh][c]);
-                  uint32_t* dst = hh ? fb : fa;
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    uint32_t v = dec_e2m1x2((nib >> (8 * i)) & 0xFFu);
-                    __half2 w = __hmul2(*reinterpret_cast<__half2*>(&v), scl);
-                    dst[i] = *reinterpret_cast<uint32_t*>(&w);
-                  }
-                }
-                if (valid < kBlock) {
-#pragma unroll
-                  for (int i = 0; i < 4; ++i) {
-                    fa[i] = mask_pair(fa[i], t0, valid);
-                    fb[i] = mask_pair(fb[i], t1, valid);
-                  }
-                }
-                // tile 2c: rows g -> d0, g+8 -> d0+1; tile 2c+1: rows g -> d0+2, g+8 -> d0+3
-                mma_pv(acc[2 * c], fa[0], fa[1], fb[0], fb[1]);
-                mma_pv(acc[2 * c + 1], fa[2], fa[3], fb[2], fb[3]);
-              }
-            }
-            // outlier channels: O^T[idx_r] += Vout^T (R x 16 tokens) P^T
-            {
-              const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes + 8;             // V idx
-              const uint16_t* vv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes + 128);  // V vals
-              uint32_t a0 = 0, a2 = 0;
-              if (g < 4) {
-                a0 = (uint32_t)vv[t0 * 4 + g] | ((uint32_t)vv[(t0 + 1) * 4 + g] << 16);
-                a2 = (uint32_t)vv[t1 * 4 + g] | ((uint32_t)vv[(t1 + 1) * 4 + g] << 16);
-                if (valid < kBlock) {
-                  a0 = mask_pair(a0, t0, valid);
-                  a2 = mask_pair(a2, t1, valid);
-                }
-              }
-              float ex[4] = {0.f, 0.f, 0.f, 0.f};
-              mma_pv(ex, a0, 0u, a2, 0u);
-              // ex[0], ex[1]: slot r = g (g < 4), query heads 2qd, 2qd+1
-#pragma unroll
-              for (int r = 0; r < kOutSlots; ++r) {
-                const int dch = idx[r];
-                const float e0 = __shfl_sync(kFull, ex[0], r * 4 + qd);
-                const float e1 = __shfl_sync(kFull, ex[1], r * 4 + qd);
-                if (dch >= D) continue;  // warp-uniform
-                const int c = dch >> 5, rem = dch & 31;
-                const int tile = 2 * c + ((rem & 3) >> 1), half = rem & 1;
-                if (g == (rem >> 2)) {
-#pragma unroll
-                  for (int mt = 0; mt < KT; ++mt) {
-                    if (mt == tile) {
-                      acc[mt][2 * half] += e0;
-                      acc[mt][2 * half + 1] += e1;
-                    }
-                  }
-                }
-              }
-            }
-          }
-        }
       }
+      const bool live0 = m0 != kNegInf, live1 = m1 != kNegInf;
+      const float pA0 = live0 ? ex2(xA0 - m0) : 0.f, pA2 = live0 ? ex2(xA2 - m0) : 0.f;
+      const float pA1 = live1 ? ex2(xA1 - m1) : 0.f, pA3 = live1 ? ex2(xA3 - m1) : 0.f;
+      const float pB0 = live0 ? ex2(xB0 - m0) : 0.f, pB2 = live0 ? ex2(xB2 - m0) : 0.f;
+      const float pB1 = live1 ? ex2(xB1 - m1) : 0.f, pB3 = live1 ? ex2(xB3 - m1) : 0.f;
+      l0 += (pA0 + pA2) + (pB0 + pB2);
+      l1 += (pA1 + pA3) + (pB1 + pB3);
+
+      // ---- O^T += V^T P^T; P = P_hi + P_lo so ~16 significant bits survive ----
+      auto pv = [&](uint32_t tb, const uint8_t* sd, int valid, float w0, float w1, float w2, float w3) {
+        const uint32_t hA = pack_f32x2(w0, w1, kBf16Mma), hB = pack_f32x2(w2, w3, kBf16Mma);
+        const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
+        const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
+        block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), movmatrix_t(lA), movmatrix_t(lB),
+                         acc);
+      };
+      if (useA && (!Gm::kFp8 || prA > 0.f))
+        pv(tbA, sdA, validA, pA0 * prA, pA1 * prA, pA2 * prA, pA3 * prA);
+      if (useB && (!Gm::kFp8 || prB > 0.f))
+        pv(tbB, sdB, validB, pB0 * prB, pB1 * prB, pB2 * prB, pB3 * prB);
+
       __syncwarp();
-      if (f + NS < f1) issue(s, coord_of(f + NS));
-      s = (s + 1 == NS) ? 0 : s + 1;
+      if (f + NS < f1) issue(sA, f + NS);
+      if (n2 == 2 && f + 1 + NS < f1) issue(sB, f + 1 + NS);
+      s = (sB + 1 == NS) ? 0 : sB + 1;
+      if (n2 == 1) s = sB;
 
       // ---- advance through (sequence, head, block) ----
-      ++j;
+      f += n2;
+      j += n2;
       const bool seg_end = (j == nblk);
-      const bool chunk_end = (f + 1 == f1);
+      const bool chunk_end = (f == f1);
       if (seg_end || chunk_end) {
         finish_piece(!seg_end);
         if (!chunk_end) {
@@ -723,7 +828,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<grid, kDecodeWarps * 32, smem, st>>>(tmap, p);
+  kern<<<grid, DecodeGeom<KVF, D>::kWarps * 32, smem, st>>>(tmap, p);
   return cudaGetLastError();
 }
 

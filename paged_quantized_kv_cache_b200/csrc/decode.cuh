@@ -32,7 +32,7 @@
 
 namespace pqkv {
 
-constexpr int kDecodeWarps = 8;
+constexpr int kDecodeWarps = 8;  // upper bound of warps per CTA over all formats
 
 struct DecodeParams {
   const void* q;
@@ -67,7 +67,10 @@ struct DecodeGeom {
   static constexpr int kIdxBytes = kFp4 ? 16 : 0;
   static constexpr int kSide = kScaleBytes + kValBytes + kIdxBytes;  // multiple of 16
   static constexpr int kSideStride = kSide == 0 ? 0 : ((kSide + 127) / 128) * 128;
-  static constexpr int kStages = k16 ? (D == 128 ? 3 : 5) : (kFp8 ? (D == 128 ? 5 : 8) : (D == 128 ? 8 : 10));
+  // Warps per CTA and shared-memory stages per warp (even: blocks are consumed
+  // in pairs while the next pair is in flight); about 192 KB of stages per SM.
+  static constexpr int kWarps = (k16 && D == 128) ? 6 : 8;
+  static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 6 : 8) : (D == 128 ? 8 : 10));
   static constexpr uint32_t kTx = kTile + kSide;
   // byte offset in a tile of (row r, byte b of that row); rows 0-15 K, 16-31 V.
   __device__ static __forceinline__ uint32_t off(int r, int b) {
@@ -84,10 +87,10 @@ struct DecodeGeom {
 template <int KVF, int D>
 struct DecodeSmem {
   using Gm = DecodeGeom<KVF, D>;
-  static constexpr int kTilesBytes = kDecodeWarps * Gm::kStages * Gm::kTile;
-  static constexpr int kSideBytes = kDecodeWarps * Gm::kStages * Gm::kSideStride;
-  static constexpr int kBarBytes = kDecodeWarps * Gm::kStages * 8;
-  static constexpr int kQBytes = Gm::kFp4 ? kDecodeWarps * 8 * D * 2 : 0;  // per-warp f16 q copy
+  static constexpr int kTilesBytes = Gm::kWarps * Gm::kStages * Gm::kTile;
+  static constexpr int kSideBytes = Gm::kWarps * Gm::kStages * Gm::kSideStride;
+  static constexpr int kBarBytes = Gm::kWarps * Gm::kStages * 8;
+  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 2 : 0;  // per-warp f16 q copy
   static size_t bytes(int B) {
     return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + (size_t)(B + 1) * 4;
   }

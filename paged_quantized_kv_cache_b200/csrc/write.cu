@@ -43,12 +43,12 @@ __device__ __forceinline__ float fp8_value(uint32_t code) {
 
 // Run discovery for the window of 32 tokens owned by this warp. Returns the
 // ballot of lanes whose token starts a run; raises SLOT / RUN error bits.
-__device__ __forceinline__ uint32_t run_starts(const WriteParams& p, int t, bool report) {
+__device__ __forceinline__ uint32_t run_starts(const WriteParams& p, int t, bool mine, bool report) {
   const int lim = p.nb * kBlock;
-  const int s = (t < p.T) ? p.slots[t] : -1;
+  const int s = (mine && t < p.T) ? p.slots[t] : -1;
   const bool valid = (s >= 0 && s < lim);
   if (report && s >= lim) raise_flag(p.err, PQKV_DEVERR_SLOT);
-  const int ps = (t > 0 && t - 1 < p.T) ? p.slots[t - 1] : -1;
+  const int ps = (mine && t > 0 && t - 1 < p.T) ? p.slots[t - 1] : -1;
   const bool pvalid = (ps >= 0 && ps < lim);
   const bool cont = valid && pvalid && s == ps + 1 && (s & (kBlock - 1)) != 0;
   const bool start = valid && !cont;
@@ -99,18 +99,18 @@ __global__ void __launch_bounds__(128) write_fp8_kernel(const WriteParams p) {
   constexpr float kMax = (KVF == PQKV_DTYPE_FP8_E4M3) ? 448.0f : 57344.0f;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int win = blockIdx.x * 4 + warp;
-  const int h = blockIdx.y;
-  const int t = win * 32 + lane;
-  uint32_t starts = run_starts(p, t, h == 0);
+  const int h = blockIdx.y, kv = blockIdx.z;
+  const int t = win * p.tpw + lane;
+  uint32_t starts = run_starts(p, t, lane < p.tpw, h == 0 && kv == 0);
   while (starts) {
     const int i = __ffs(starts) - 1;
     starts &= starts - 1;
-    const int ts = win * 32 + i;
+    const int ts = win * p.tpw + i;
     const int s0 = p.slots[ts];
     const int n = run_length(p, ts, s0, lane);
     const int blk = s0 >> 4, off0 = s0 & 15;
     const size_t pair = (size_t)blk * p.Hkv + h;
-    for (int kv = 0; kv < 2; ++kv) {
+    {
       const void* x = kv ? p.v : p.k;
       float xs[kBlock][CPL];
       float a = 0.f;
@@ -178,18 +178,18 @@ __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
   __shared__ float s_norm[4][D];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int win = blockIdx.x * 4 + warp;
-  const int h = blockIdx.y;
-  const int t = win * 32 + lane;
-  uint32_t starts = run_starts(p, t, h == 0);
+  const int h = blockIdx.y, kv = blockIdx.z;
+  const int t = win * p.tpw + lane;
+  uint32_t starts = run_starts(p, t, lane < p.tpw, h == 0 && kv == 0);
   while (starts) {
     const int i = __ffs(starts) - 1;
     starts &= starts - 1;
-    const int ts = win * 32 + i;
+    const int ts = win * p.tpw + i;
     const int s0 = p.slots[ts];
     const int n = run_length(p, ts, s0, lane);
     const int blk = s0 >> 4, off0 = s0 & 15;
     const size_t pair = (size_t)blk * p.Hkv + h;
-    for (int kv = 0; kv < 2; ++kv) {
+    {
       const void* x = kv ? p.v : p.k;
       const size_t tile = pair * 2 + kv;  // (block, head, K|V) index
       float xs[kBlock][CPL];
@@ -356,9 +356,12 @@ cudaError_t launch_write(int kv_dtype, int in_dtype, int D, const WriteParams& p
     else write16_kernel<64><<<grid, 256, 0, st>>>(p);
     return cudaGetLastError();
   }
-  const dim3 grid((unsigned)((p.T + 127) / 128), (unsigned)p.Hkv);
+  // a warp owns the runs starting in a window of tpw tokens of one (head, K|V)
+  WriteParams q = p;
+  q.tpw = (p.T <= 8192) ? 1 : 32;
+  const dim3 grid((unsigned)((p.T + 4 * q.tpw - 1) / (4 * q.tpw)), (unsigned)p.Hkv, 2u);
 #define PQKV_W8(F, DD, B) \
-  if (kv_dtype == F && D == DD && bf == B) { write_fp8_kernel<F, DD, B><<<grid, 128, 0, st>>>(p); return cudaGetLastError(); }
+  if (kv_dtype == F && D == DD && bf == B) { write_fp8_kernel<F, DD, B><<<grid, 128, 0, st>>>(q); return cudaGetLastError(); }
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 128, true)
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 128, false)
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 64, true)
@@ -370,11 +373,11 @@ cudaError_t launch_write(int kv_dtype, int in_dtype, int D, const WriteParams& p
 #undef PQKV_W8
   if (kv_dtype == PQKV_DTYPE_FP4_E2M1) {
     if (D == 128) {
-      if (bf) write_fp4_kernel<128, true><<<grid, 128, 0, st>>>(p);
-      else write_fp4_kernel<128, false><<<grid, 128, 0, st>>>(p);
+      if (bf) write_fp4_kernel<128, true><<<grid, 128, 0, st>>>(q);
+      else write_fp4_kernel<128, false><<<grid, 128, 0, st>>>(q);
     } else {
-      if (bf) write_fp4_kernel<64, true><<<grid, 128, 0, st>>>(p);
-      else write_fp4_kernel<64, false><<<grid, 128, 0, st>>>(p);
+      if (bf) write_fp4_kernel<64, true><<<grid, 128, 0, st>>>(q);
+      else write_fp4_kernel<64, false><<<grid, 128, 0, st>>>(q);
     }
     return cudaGetLastError();
   }

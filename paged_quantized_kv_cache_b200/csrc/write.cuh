@@ -15,6 +15,7 @@ struct WriteParams {
   uint8_t* oval;
   int32_t* err;
   int T, nb, Hkv;
+  int tpw;  // tokens per warp window (set by the launcher)
 };
 
 cudaError_t launch_write(int kv_dtype, int in_dtype, int D, const WriteParams& p, cudaStream_t st);

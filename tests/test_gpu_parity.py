@@ -226,11 +226,14 @@ def test_write_error_bits_match_oracle(kv_dtype):
     g, o = gh.new_pair(kv_dtype, 4, Hkv, D)
     rng = np.random.default_rng(8)
     k, v = _kv(rng, 4, Hkv, D, qdt)
-    ge, oe = gh.write_both(g, o, k, v, np.array([0, 4 * 16 + 3, -1, 1], np.int32))
+    # token 1 points past the pool: skipped and flagged; the others are written
+    ge, oe = gh.write_both(g, o, k, v, np.array([0, 4 * 16 + 3, -1, 16], np.int32))
     assert ge == oe and ge & pq.DEVERR_SLOT
     gh.assert_cache_equal(g, o, tag="slot error")
     if kv_dtype != pq.BF16:
-        ge, oe = gh.write_both(g, o, k[:2], v[:2], np.array([20, 23], np.int32))
+        # two adjacent tokens in one block with a gap in their offsets: flagged
+        # (their order in the block is unspecified, so no bytes are compared)
+        ge, oe = gh.write_both(g, o, k[:2], v[:2], np.array([36, 39], np.int32))
         assert ge & pq.DEVERR_RUN and oe & pq.DEVERR_RUN
     # empty call is a no-op
     pq.kv_cache_write(k[:0].cuda(), v[:0].cuda(), torch.zeros(0, dtype=torch.int32, device="cuda"), g,
