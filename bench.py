@@ -63,8 +63,11 @@ L2_BYTES = 126 * 1024 * 1024
 # workload on the device
 # ---------------------------------------------------------------------------
 
-def bench_spec(name: str, kv_name: str | None) -> W.Spec:
-    s = W.spec(name, kv_dtype=KV_NAMES[kv_name] if kv_name else None)
+def bench_spec(name: str, kv_name: str | None, batch: int | None = None, pool: int | None = None) -> W.Spec:
+    """The workload as bench.py runs it; batch / pool cut it down for profiling."""
+    s = W.spec(name, kv_dtype=KV_NAMES[kv_name] if kv_name else None, batch=batch)
+    if pool:
+        s.pool_blocks = pool
     s.append_tokens = 1  # every step appends one token per sequence
     if s.kv_dtype in (W.DT_FP16, W.DT_BF16):
         s.q_dtype = s.kv_dtype  # 16-bit caches take queries of their own type
@@ -386,7 +389,7 @@ def run_reference(args) -> None:
     rank, world, _ = dist_env()
     if rank != 0:
         return
-    s = bench_spec(args.workload, args.kv_dtype)
+    s = bench_spec(args.workload, args.kv_dtype, args.batch, args.pool_blocks)
     nseq = args.ref_seqs
     budget = 150.0
     while True:
@@ -448,7 +451,7 @@ def run_ours(args) -> None:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    s = bench_spec(args.workload, args.kv_dtype)
+    s = bench_spec(args.workload, args.kv_dtype, args.batch, args.pool_blocks)
     st = Setup(s, device, args.split_blocks)
     stream = torch.cuda.current_stream(device)
 
@@ -511,7 +514,8 @@ def run_ours(args) -> None:
             "decode_tok_s_per_layer": tok_s,
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": 2 * K, "clocks": clocks.summary(),
+            # per step: cache write, split decode, log-sum-exp merge
+            "gpu_launches": 3 * K, "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -565,6 +569,8 @@ def main():
     ap.add_argument("--workload", choices=sorted(DESCR), default="llama8b")
     ap.add_argument("--kv-dtype", choices=sorted(KV_NAMES), default=None)
     ap.add_argument("--split-blocks", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=None, help="first N sequences only (profiling subsets)")
+    ap.add_argument("--pool-blocks", type=int, default=None, help="smaller block pool (profiling subsets)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle timing")

@@ -173,9 +173,10 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
  * GPU; > 0 = process the KV of all (sequence, head) pairs, laid end to end, in
  * chunks of exactly that many 16-token blocks. Results differ only by rounding.
  * workspace: device buffer of at least pqkv_decode_workspace_bytes(...) bytes,
- * zero-filled before its first use (pqkv_decode_workspace_init); every call
- * leaves it ready for the next. Calls that share a workspace must be ordered.
- * batch <= PQKV_MAX_BATCH.
+ * scratch for the split pieces (no initialization needed). Two kernels run on
+ * `stream`: the split decode, then the log-sum-exp merge of split pairs
+ * (launched as a programmatic dependent of the first). Calls that share a
+ * workspace must be ordered. batch <= PQKV_MAX_BATCH.
  */
 int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads,
                                 const void* cache, const void* scales,
@@ -187,7 +188,8 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err_flag, pqkv_stream_t stream);
 
-/* Zero-fill a decode workspace on `stream` (needed once per new buffer). */
+/* Zero-fill a decode workspace on `stream` (optional; results never depend on
+ * the workspace's prior contents). */
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
                                pqkv_stream_t stream);
 

@@ -11,6 +11,7 @@
 namespace pqkv {
 cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st);
+cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
 size_t decode_smem_bytes(int kv_dtype, int D, int B);
 }  // namespace pqkv
 
@@ -103,6 +104,11 @@ bool cached_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb,
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Workspace = plan header (chunk length + block prefix per sequence, written by
+// the decode kernel, read by the merge kernel) followed by two partial-result
+// slots per chunk. Nothing in it needs to be initialized by the caller.
+size_t plan_bytes(int batch) { return round_up((size_t)(batch + 2) * 4, 256); }
+
 }  // namespace
 
 extern "C" {
@@ -174,12 +180,11 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
   if (G > 8) return 0;
   DeviceInfo di;
   if (!device_info(di)) return 0;
-  const size_t counters = round_up((size_t)batch * num_kv_heads * 4, 256);
   const size_t slot = round_up((size_t)G * head_dim + 2 * G, 4) * 4;
   const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
   const size_t chunks = split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks
                                          : (size_t)di.sms * kDecodeWarps;
-  return counters + 2 * chunks * slot;
+  return plan_bytes(batch) + 2 * chunks * slot;
 }
 
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_stream_t stream) {
@@ -230,9 +235,8 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   p.block_tables = block_tables;
   p.seq_lens = seq_lens;
   p.err = err_flag;
-  p.counters = static_cast<int32_t*>(workspace);
-  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                        round_up((size_t)batch * num_kv_heads * 4, 256));
+  p.plan = static_cast<int32_t*>(workspace);
+  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan_bytes(batch));
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
@@ -243,8 +247,19 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   p.slot_floats = (int)round_up((size_t)p.G * head_dim + 2 * p.G, 4);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
-  const cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms,
-                                      reinterpret_cast<cudaStream_t>(stream));
+  const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms, st);
+  if (e != cudaSuccess) return PQKV_ERR_CUDA;
+  MergeParams mp;
+  mp.plan = p.plan;
+  mp.partials = p.partials;
+  mp.out = out;
+  mp.B = batch;
+  mp.Hq = num_q_heads;
+  mp.Hkv = num_kv_heads;
+  mp.G = p.G;
+  mp.slot_floats = p.slot_floats;
+  e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
 }
 

@@ -79,6 +79,16 @@ __device__ __forceinline__ uint32_t dec_e2m1x2(uint32_t byte) {
   return r;
 }
 
+// Eight E2M1 codes of a word (byte i = codes 2i, 2i+1, low nibble first) ->
+// four f16x2 (exact), one per byte.
+__device__ __forceinline__ void dec_e2m1x8(uint32_t w, uint32_t (&o)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+
 __device__ __forceinline__ float lo_half(uint32_t h2) {
   return __half2float(__ushort_as_half((unsigned short)(h2 & 0xFFFFu)));
 }

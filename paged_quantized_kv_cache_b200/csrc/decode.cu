@@ -169,12 +169,12 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
         const __half2 sa = __low2half2(*reinterpret_cast<const __half2*>(&sca));
         const __half2 sb = __low2half2(*reinterpret_cast<const __half2*>(&scb));
         uint32_t ha[4], hb[4];
+        dec_e2m1x8(ra, ha);
+        dec_e2m1x8(rb, hb);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          uint32_t x = dec_e2m1x2((ra >> (8 * i)) & 0xFFu);
-          uint32_t y = dec_e2m1x2((rb >> (8 * i)) & 0xFFu);
-          __half2 xa = __hmul2(*reinterpret_cast<__half2*>(&x), sa);
-          __half2 yb = __hmul2(*reinterpret_cast<__half2*>(&y), sb);
+          __half2 xa = __hmul2(*reinterpret_cast<__half2*>(&ha[i]), sa);
+          __half2 yb = __hmul2(*reinterpret_cast<__half2*>(&hb[i]), sb);
           ha[i] = *reinterpret_cast<uint32_t*>(&xa);
           hb[i] = *reinterpret_cast<uint32_t*>(&yb);
         }
@@ -290,10 +290,11 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
           const uint32_t A = prmt(lo, hi, 0x5140u), Bv = prmt(lo, hi, 0x7362u);
           const uint32_t nib = A | (Bv << 4);  // bytes: d0, d0+1, d0+2, d0+3 (token pair)
           const __half2 scl = *reinterpret_cast<const __half2*>(&sp[hh][c]);
+          uint32_t dv[4];
+          dec_e2m1x8(nib, dv);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            uint32_t v = dec_e2m1x2((nib >> (8 * i)) & 0xFFu);
-            __half2 w = __hmul2(*reinterpret_cast<__half2*>(&v), scl);
+            __half2 w = __hmul2(*reinterpret_cast<__half2*>(&dv[i]), scl);
             if (hh) fb[i] = *reinterpret_cast<uint32_t*>(&w);
             else fa[i] = *reinterpret_cast<uint32_t*>(&w);
           }
@@ -351,6 +352,70 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
 }
 
 }  // namespace
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of split pairs ("Flash-Decoding": the partial softmaxes of
+// the pieces are combined as M = max_j m_j, L = sum_j l_j 2^(m_j - M),
+// out = sum_j O_j 2^(m_j - M) / L, in fixed piece order). One warp per
+// (sequence b, KV head h, query head n of the group). Launched as a
+// programmatic dependent of the decode kernel: it waits for that grid before
+// reading the plan and the partials it wrote.
+// ---------------------------------------------------------------------------
+template <int D, bool QBF16>
+__global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int DPL = D / 32;
+  const int lane = threadIdx.x & 31;
+  const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= (long)p.B * p.Hq) return;
+  const int b = (int)(wid / p.Hq), hq = (int)(wid % p.Hq);
+  const int h = hq / p.G, n = hq % p.G;
+  const int Qc = p.plan[0];
+  const int Pb = p.plan[1 + b], nblk = p.plan[2 + b] - Pb;
+  if (nblk == 0) return;
+  const int s0 = p.Hkv * Pb + h * nblk;
+  const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
+  if (k0 == k1) return;  // the pair was finished inside one chunk
+  const int np = k1 - k0 + 1;
+  auto slot_base = [&](int i) {  // piece i (0-based) of the pair
+    const int kk = k0 + i;
+    return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
+  };
+  // weights: lanes over pieces
+  float M = kNegInf;
+  for (int i = lane; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  float L = 0.f;
+  for (int i = lane; i < np; i += 32) {
+    const float* bs = slot_base(i);
+    const float m = __ldcg(bs + p.G * D + n);
+    L += (M == kNegInf) ? 0.f : exp2f(m - M) * __ldcg(bs + p.G * D + p.G + n);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+  // outputs: lanes over head dims, pieces in order
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+#pragma unroll 4
+  for (int i = 0; i < np; ++i) {
+    const float* bs = slot_base(i);
+    const float m = __ldcg(bs + p.G * D + n);
+    const float w = (M == kNegInf) ? 0.f : exp2f(m - M);
+    if constexpr (DPL == 4) {
+      const float4 v = __ldcg(reinterpret_cast<const float4*>(bs + n * D + lane * 4));
+      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] += w * __ldcg(bs + n * D + lane * DPL + e);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const size_t orow = ((size_t)b * p.Hq + hq) * D + lane * DPL;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
+}
 
 template <int KVF, int D, bool QBF16>
 __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
@@ -429,6 +494,11 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   const int W = gridDim.x * NW;
   const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + W - 1) / W);
   const int K = T > 0 ? (T + Qc - 1) / Qc : 0;
+  if (blockIdx.x == 0) {  // the plan the merge kernel reads
+    if (tid == 0) p.plan[0] = Qc;
+    for (int i = tid; i <= B; i += blockDim.x) p.plan[1 + i] = P[i];
+  }
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   uint32_t phase = 0;     // parity bit per stage
   uint32_t inflight = 0;  // stages with an issued, unconsumed copy
@@ -561,44 +631,6 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       }
     };
 
-    auto merge = [&](int k0, int k1) {
-      constexpr int DPL = D / 32;
-      float M[8], Ls[8], o[8][DPL];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        M[n] = kNegInf;
-        Ls[n] = 0.f;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) o[n][e] = 0.f;
-      }
-      for (int kk = k0; kk <= k1; ++kk) {
-        const float* base = p.partials + (size_t)(kk == k0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-          if (n < G) M[n] = fmaxf(M[n], __ldcg(base + G * D + n));
-      }
-      for (int kk = k0; kk <= k1; ++kk) {
-        const float* base = p.partials + (size_t)(kk == k0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
-#pragma unroll
-        for (int n = 0; n < 8; ++n) {
-          if (n >= G) continue;
-          const float mj = __ldcg(base + G * D + n);
-          const float w = (M[n] == kNegInf) ? 0.f : exp2f(mj - M[n]);
-          Ls[n] += w * __ldcg(base + G * D + G + n);
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) o[n][e] += w * __ldcg(base + n * D + lane * DPL + e);
-        }
-      }
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        if (n >= G) continue;
-        const float inv = Ls[n] > 0.f ? 1.f / Ls[n] : 0.f;
-        const size_t orow = ((size_t)b * Hq + (size_t)h * G + n) * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, o[n][e] * inv);
-      }
-    };
-
     auto finish_piece = [&](bool ends_after) {
       float lt0 = l0, lt1 = l1;
 #pragma unroll
@@ -649,22 +681,6 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
           base[G * D + n1] = m1;
           base[G * D + G + n1] = lt1;
         }
-      }
-      __syncwarp();
-      __threadfence();
-      const int s0 = Hkv * P[b] + h * nblk;
-      const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
-      int last = 0;
-      if (lane == 0) {
-        int* ctr = p.counters + (size_t)b * Hkv + h;
-        const int prev = atomicAdd(ctr, 1);
-        last = (prev == k1 - k0);
-        if (last) atomicExch(ctr, 0);
-      }
-      last = __shfl_sync(kFull, last, 0);
-      if (last) {
-        __threadfence();
-        merge(k0, k1);
       }
     };
 
@@ -830,6 +846,28 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
   }
   kern<<<grid, DecodeGeom<KVF, D>::kWarps * 32, smem, st>>>(tmap, p);
   return cudaGetLastError();
+}
+
+// The merge kernel is launched right behind the decode kernel on the same
+// stream as a programmatic dependent (its launch overlaps the decode's tail;
+// griddepcontrol.wait inside it orders it after the decode grid).
+cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st) {
+  const long warps = (long)p.B * p.Hq;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128)
+    return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, true>, p)
+                  : cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, false>, p);
+  return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, true>, p)
+                : cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, false>, p);
 }
 
 size_t decode_smem_bytes(int kv_dtype, int D, int B) {

@@ -14,9 +14,9 @@
 // The grid is persistent (one CTA per SM, NW warps each); the flat range is cut
 // into chunks of Q blocks and warp w takes chunks w, w + W, ... (W = all warps).
 // A chunk covers whole pairs (written straight to `out`) and at most two
-// partial pairs at its ends (written to a workspace slot). The warp that
-// completes the last piece of a pair (an atomic counter per pair) merges the
-// pieces in chunk order, so results do not depend on timing.
+// partial pairs at its ends (written to a workspace slot). A second kernel,
+// launched as a programmatic dependent of the first, merges the pieces of each
+// split pair in chunk order, so results do not depend on timing.
 //
 // Per warp: a private ring of NS shared-memory stages, each holding the K and V
 // tiles of one (block, head) pair fetched by one TMA tensor copy (128/64/32-byte
@@ -32,7 +32,7 @@
 
 namespace pqkv {
 
-constexpr int kDecodeWarps = 8;  // upper bound of warps per CTA over all formats
+constexpr int kDecodeWarps = 12;  // upper bound of warps per CTA over all formats
 
 struct DecodeParams {
   const void* q;
@@ -43,13 +43,21 @@ struct DecodeParams {
   const int32_t* block_tables;  // [B][maxblk]
   const int32_t* seq_lens;      // [B]
   int32_t* err;
-  int32_t* counters;            // [B * Hkv], zero between calls
+  int32_t* plan;                // workspace header: [0] = chunk length, [1..B+1] = block prefix P
   float* partials;              // [2 * chunks][slot_floats]
   int B, Hq, Hkv, G, nb, maxblk;
   int split_blocks;
   int slot_floats;
   float scale_log2;             // softmax scale * log2(e)
   uint64_t timeout_ns;
+};
+
+struct MergeParams {
+  const int32_t* plan;
+  const float* partials;
+  void* out;
+  int B, Hq, Hkv, G;
+  int slot_floats;
 };
 
 // Compile-time geometry of one format.
@@ -69,8 +77,8 @@ struct DecodeGeom {
   static constexpr int kSideStride = kSide == 0 ? 0 : ((kSide + 127) / 128) * 128;
   // Warps per CTA and shared-memory stages per warp (even: blocks are consumed
   // in pairs while the next pair is in flight); about 192 KB of stages per SM.
-  static constexpr int kWarps = (k16 && D == 128) ? 6 : 8;
-  static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 6 : 8) : (D == 128 ? 8 : 10));
+  static constexpr int kWarps = k16 ? (D == 128 ? 6 : 8) : 12;
+  static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 4 : 6) : (D == 128 ? 4 : 6));
   static constexpr uint32_t kTx = kTile + kSide;
   // byte offset in a tile of (row r, byte b of that row); rows 0-15 K, 16-31 V.
   __device__ static __forceinline__ uint32_t off(int r, int b) {

@@ -179,15 +179,15 @@ def test_repeated_calls_are_deterministic_and_reuse_the_workspace():
     ws = pq.decode_workspace(len(lens), case[3], case[4], case[2], bt.shape[1])
     qd = q.cuda()
     first = None
-    for _ in range(5):
+    for it in range(5):
         out = torch.empty_like(qd)
         e = gh.err_flag()
+        if it == 3:
+            ws.fill_(0xAB)  # results do not depend on what the workspace held
         pq.paged_decode_attention(qd, g, bt_d, sl, 0.1, out, ws, e)
         if first is None:
             first = out
         assert torch.equal(out, first) and int(e.item()) == 0
-    # the workspace's counters are back to zero after every call
-    assert int(ws[: 4 * len(lens) * case[4]].view(torch.int32).abs().sum().item()) == 0
 
 
 def test_edge_lengths_and_error_bits():
