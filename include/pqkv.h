@@ -70,7 +70,8 @@ enum {
   PQKV_ERR_ARG = 1,   /* null pointer, bad enum, unsupported size, small buffer */
   PQKV_ERR_OOM = 2,   /* block pool cannot satisfy an allocation (no change made) */
   PQKV_ERR_STATE = 3, /* refcount underflow / freeing or sharing a free block */
-  PQKV_ERR_CUDA = 4   /* a CUDA runtime call or launch failed */
+  PQKV_ERR_CUDA = 4,  /* a CUDA runtime call or launch failed */
+  PQKV_ERR_SCRATCH = 5 /* the request needs more than PQKV_NOALLOC_SCRATCH_BYTES of scratch */
 };
 
 /* ---- element types ---------------------------------------------------------- */
@@ -187,6 +188,34 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
                                 float scale, int split_blocks, void* out,
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err_flag, pqkv_stream_t stream);
+
+/*
+ * pqkv_paged_decode_attention without a workspace argument, for callers that
+ * cannot allocate device memory (for example a host whose device memory is
+ * fully reserved by its own pool, or a latency-critical path where cudaMalloc
+ * and its possible device synchronization are not acceptable). The pages
+ * describe no counterpart; this is a property of this library only.
+ * The scratch is one static device array of PQKV_NOALLOC_SCRATCH_BYTES that
+ * every GPU loading the library holds until exit. Requests needing more
+ * (pqkv_decode_workspace_bytes of the same sizes) return PQKV_ERR_SCRATCH and
+ * launch nothing; with split_blocks = 0, head_dim <= 128 and up to 8 query heads
+ * per KV head the need stays below 16 MiB on a 148-SM GPU. Nothing is
+ * allocated. The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and should come before any stream capture. All calls
+ * share the array: calls that overlap on the GPU (other streams, other host
+ * threads) race on it and must be ordered by the caller. No part of the array
+ * needs to start at zero; it keeps the last call's contents. Other arguments,
+ * results and errors as pqkv_paged_decode_attention.
+ */
+#define PQKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+int pqkv_paged_decode_attention_noalloc(const void* q, int q_dtype, int batch, int num_q_heads,
+                                        const void* cache, const void* scales,
+                                        const void* outliers_idx, const void* outliers_val,
+                                        int kv_dtype, int num_blocks, int num_kv_heads,
+                                        int head_dim, const int32_t* block_tables,
+                                        int max_blocks_per_seq, const int32_t* seq_lens,
+                                        float scale, int split_blocks, void* out,
+                                        int32_t* err_flag, pqkv_stream_t stream);
 
 /* Zero-fill a decode workspace on `stream` (optional; results never depend on
  * the workspace's prior contents). */

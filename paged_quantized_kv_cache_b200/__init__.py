@@ -23,7 +23,8 @@ LIB_PATH = os.path.join(_HERE, "libpqkv.so")
 
 FP16, BF16, FP8_E4M3, FP8_E5M2, FP4_E2M1 = 0, 1, 2, 3, 4
 DTYPE_NAMES = {FP16: "fp16", BF16: "bf16", FP8_E4M3: "fp8_e4m3", FP8_E5M2: "fp8_e5m2", FP4_E2M1: "fp4_e2m1"}
-OK, ERR_ARG, ERR_OOM, ERR_STATE, ERR_CUDA = 0, 1, 2, 3, 4
+OK, ERR_ARG, ERR_OOM, ERR_STATE, ERR_CUDA, ERR_SCRATCH = 0, 1, 2, 3, 4, 5
+NOALLOC_SCRATCH_BYTES = 16 << 20
 DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_RUN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 BLOCK_SIZE = 16
 MAX_BATCH = 4096
@@ -34,6 +35,7 @@ EXPORTS = (
     "pqkv_decode_workspace_bytes", "pqkv_paged_decode_attention", "pqkv_decode_workspace_init",
     "pqkv_encode", "pqkv_pool_create", "pqkv_pool_destroy", "pqkv_pool_alloc", "pqkv_pool_share",
     "pqkv_pool_free", "pqkv_pool_num_free", "pqkv_pool_refcount", "pqkv_build_slot_mapping",
+    "pqkv_paged_decode_attention_noalloc",
 )
 
 
@@ -66,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "pqkv_pool_num_free": (ctypes.c_int32, [P]),
         "pqkv_pool_refcount": (ctypes.c_int32, [P, ctypes.c_int32]),
         "pqkv_build_slot_mapping": (I, [P, I, I, P, P, P]),
+        "pqkv_paged_decode_attention_noalloc": (I, [P, I, I, I, P, P, P, P, I, I, I, I, P, I, P, ctypes.c_float,
+                                                    I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)

@@ -122,6 +122,7 @@ const char* pqkv_status_string(int status) {
     case PQKV_ERR_OOM: return "block pool exhausted";
     case PQKV_ERR_STATE: return "invalid block state";
     case PQKV_ERR_CUDA: return "CUDA error";
+    case PQKV_ERR_SCRATCH: return "request exceeds the static scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
