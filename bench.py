@@ -303,10 +303,12 @@ def dist_env():
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value of x over the ranks of the default process group."""
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
