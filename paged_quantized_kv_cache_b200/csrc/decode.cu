@@ -150,11 +150,19 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
     // d = 32c + 8qd .. +7 of token rows g and g + 8 and multiplies them by the
     // token's E4M3 scale of group 2c + qd/2 (the product is exact in f16).
     constexpr int SPR = D / 16;  // scale bytes per token row
-    uint32_t s_lo = 0, s_hi = 0;
+    // The scale of chunk c for this lane is byte 2c + qd/2 of the token's scale
+    // row: pick it from whole words and broadcast it to (s, s) in f16.
+    uint32_t sa2[D / 32], sb2[D / 32];
+    {
+      const int a = qd >> 1;
+      const uint32_t sel = (uint32_t)(a | (a << 4) | ((a + 2) << 8) | ((a + 2) << 12));
+      const uint32_t* ra = reinterpret_cast<const uint32_t*>(side + g * SPR);
+      const uint32_t* rb = reinterpret_cast<const uint32_t*>(side + (g + 8) * SPR);
 #pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      s_lo |= (uint32_t)side[g * SPR + 2 * c + (qd >> 1)] << (8 * c);
-      s_hi |= (uint32_t)side[(g + 8) * SPR + 2 * c + (qd >> 1)] << (8 * c);
+      for (int w = 0; w < SPR / 4; ++w) {  // word w = groups 4w..4w+3 = chunks 2w, 2w+1
+        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(ra[w], 0u, sel), sa2[2 * w], sa2[2 * w + 1]);
+        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(rb[w], 0u, sel), sb2[2 * w], sb2[2 * w + 1]);
+      }
     }
 #pragma unroll
     for (int cp = 0; cp < D / 64; ++cp) {
@@ -164,10 +172,8 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
       for (int e = 0; e < 2; ++e) {
         const int c = 2 * cp + e;
         const uint32_t ra = e ? r2 : r0, rb = e ? r3 : r1;
-        const uint32_t sca = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_lo >> (8 * c)) & 0xFFu);
-        const uint32_t scb = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>((s_hi >> (8 * c)) & 0xFFu);
-        const __half2 sa = __low2half2(*reinterpret_cast<const __half2*>(&sca));
-        const __half2 sb = __low2half2(*reinterpret_cast<const __half2*>(&scb));
+        const __half2 sa = *reinterpret_cast<const __half2*>(&sa2[c]);
+        const __half2 sb = *reinterpret_cast<const __half2*>(&sb2[c]);
         uint32_t ha[4], hb[4];
         dec_e2m1x8(ra, ha);
         dec_e2m1x8(rb, hb);
@@ -211,15 +217,17 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
 template <int KVF, int D>
 __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const LdsmOffsets<KVF, D>& lo, int lane,
                                          int valid, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
-                                         float (&acc)[D / 16][4]) {
+                                         float (&acc)[D / 16][4], float* oext) {
   using Gm = DecodeGeom<KVF, D>;
   constexpr int KT = D / 16;
   constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
   const int g = lane >> 2, qd = lane & 3;
   const int t0 = 2 * qd, t1 = 2 * qd + 8;
+  // FP4 keeps P in f16 only (its tolerance allows it); the others add P_lo.
+  constexpr bool kSplitP = !Gm::kFp4;
   auto mma_pv = [&](float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
     mma16816<kBf>(d, a0, a1, a2, a3, b0, b1);
-    mma16816<kBf>(d, a0, a1, a2, a3, c0, c1);
+    if constexpr (kSplitP) mma16816<kBf>(d, a0, a1, a2, a3, c0, c1);
   };
   if constexpr (Gm::k16) {
 #pragma unroll
@@ -264,15 +272,19 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
     constexpr int SPR = D / 16;
     const uint8_t* vs = side + 16 * SPR;  // V scales [16][D/16]
     const int gs = g >> 2;
+    // scale pairs (token t, t + 1) of chunk c: bytes 2c + g/4 of the two tokens'
+    // scale rows, picked from whole words
     uint32_t sp[2][D / 32];
+    {
+      const uint32_t sel = (uint32_t)(gs | ((4 + gs) << 4) | ((2 + gs) << 8) | ((6 + gs) << 12));
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int ta = 2 * qd + 8 * hh;
+      for (int hh = 0; hh < 2; ++hh) {
+        const int ta = 2 * qd + 8 * hh;
+        const uint32_t* w0 = reinterpret_cast<const uint32_t*>(vs + ta * SPR);
+        const uint32_t* w1 = reinterpret_cast<const uint32_t*>(vs + (ta + 1) * SPR);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        const uint32_t two =
-            (uint32_t)vs[ta * SPR + 2 * c + gs] | ((uint32_t)vs[(ta + 1) * SPR + 2 * c + gs] << 8);
-        sp[hh][c] = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(two);
+        for (int w = 0; w < SPR / 4; ++w)
+          dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], sel), sp[hh][2 * w], sp[hh][2 * w + 1]);
       }
     }
 #pragma unroll
@@ -311,8 +323,10 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
         mma_pv(acc[2 * c + 1], fa[2], fa[3], fb[2], fb[3]);
       }
     }
-    // outlier channels: O^T[idx_r] += Vout^T (4 slots x 16 tokens) P^T; the
-    // result of slot r sits in lanes 4r..4r+3 and moves to the lanes owning d = idx_r
+    // outlier channels: Oext[n][idx_r] += (Vout^T (4 slots x 16 tokens) P^T)[r][n].
+    // The result of slot r sits in lanes 4r..4r+3 (heads 2qd, 2qd+1); it is
+    // added to the warp's shared-memory accumulator of outlier channels, which
+    // follows O's rescaling and is folded into O when the piece ends.
     {
       const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes + 8;                         // V idx
       const uint16_t* vv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes + 128);    // V vals
@@ -327,26 +341,14 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
       }
       float ex[4] = {0.f, 0.f, 0.f, 0.f};
       mma_pv(ex, a0, 0u, a2, 0u);
-#pragma unroll
-      for (int r = 0; r < kOutSlots; ++r) {
-        const int dch = idx[r];
-        const float e0 = __shfl_sync(kFull, ex[0], r * 4 + qd);
-        const float e1 = __shfl_sync(kFull, ex[1], r * 4 + qd);
-        if (dch >= D) continue;  // warp-uniform
-        const int c = dch >> 5, rem = dch & 31;
-        const int tile = 2 * c + ((rem & 3) >> 1), half = rem & 1;
-        if (g == (rem >> 2)) {
-#pragma unroll
-          for (int mt = 0; mt < KT; ++mt) {
-            if (mt == tile) {
-              acc[mt][0] += half ? 0.f : e0;
-              acc[mt][1] += half ? 0.f : e1;
-              acc[mt][2] += half ? e0 : 0.f;
-              acc[mt][3] += half ? e1 : 0.f;
-            }
-          }
+      if (g < 4) {
+        const int dch = idx[g];
+        if (dch < D) {
+          oext[(2 * qd) * D + dch] += ex[0];
+          oext[(2 * qd + 1) * D + dch] += ex[1];
         }
       }
+      __syncwarp();
     }
   }
 }
@@ -433,7 +435,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   uint8_t* sides = tiles + Sm::kTilesBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(sides + Sm::kSideBytes);
   uint16_t* qcopy = reinterpret_cast<uint16_t*>(reinterpret_cast<uint8_t*>(bars) + Sm::kBarBytes);
-  int* P = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(qcopy) + Sm::kQBytes);
+  float* oext_all = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(qcopy) + Sm::kQBytes);
+  int* P = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(oext_all) + Sm::kOextBytes);
   __shared__ int warp_sums[NW];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -443,6 +446,9 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
   uint16_t* wq = qcopy + warp * 8 * D;
+  float* woext = oext_all + warp * 8 * D;  // FP4: O of outlier channels [8 heads][D]
+  if constexpr (Gm::kFp4)
+    for (int i = lane; i < 8 * D; i += 32) woext[i] = 0.f;
   const LdsmOffsets<KVF, D> lofs(lane);
 
   if (lane == 0) {
@@ -640,6 +646,18 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       }
       const float vs = Gm::kFp8 ? vref : 1.f;
       const int n0 = 2 * qd, n1 = 2 * qd + 1;
+      if constexpr (Gm::kFp4) {  // fold the outlier channels' O in and clear it
+        __syncwarp();
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            float* slot = woext + (2 * qd + (e & 1)) * D + dmap<KVF>(mt, g + 8 * (e >> 1));
+            acc[mt][e] += *slot;
+            *slot = 0.f;
+          }
+        __syncwarp();
+      }
       if (!started_before && !ends_after) {
         const float i0 = lt0 > 0.f ? vs / lt0 : 0.f;
         const float i1 = lt1 > 0.f ? vs / lt1 : 0.f;
@@ -770,6 +788,15 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
           acc[mt][2] *= f0c;
           acc[mt][3] *= f1c;
         }
+        if constexpr (Gm::kFp4) {  // the outlier channels' O follows the same rescale
+          __syncwarp();
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              woext[(2 * qd + (e & 1)) * D + dmap<KVF>(mt, g + 8 * (e >> 1))] *= (e & 1) ? f1c : f0c;
+          __syncwarp();
+        }
       }
       const bool live0 = m0 != kNegInf, live1 = m1 != kNegInf;
       const float pA0 = live0 ? ex2(xA0 - m0) : 0.f, pA2 = live0 ? ex2(xA2 - m0) : 0.f;
@@ -779,13 +806,17 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       l0 += (pA0 + pA2) + (pB0 + pB2);
       l1 += (pA1 + pA3) + (pB1 + pB3);
 
-      // ---- O^T += V^T P^T; P = P_hi + P_lo so ~16 significant bits survive ----
+      // ---- O^T += V^T P^T; P = P_hi + P_lo (except FP4) so ~16 significant bits survive ----
       auto pv = [&](uint32_t tb, const uint8_t* sd, int valid, float w0, float w1, float w2, float w3) {
         const uint32_t hA = pack_f32x2(w0, w1, kBf16Mma), hB = pack_f32x2(w2, w3, kBf16Mma);
-        const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
-        const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
-        block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), movmatrix_t(lA), movmatrix_t(lB),
-                         acc);
+        if constexpr (Gm::kFp4) {
+          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), 0u, 0u, acc, woext);
+        } else {
+          const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
+          const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
+          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), movmatrix_t(lA),
+                           movmatrix_t(lB), acc, woext);
+        }
       };
       if (useA && (!Gm::kFp8 || prA > 0.f))
         pv(tbA, sdA, validA, pA0 * prA, pA1 * prA, pA2 * prA, pA3 * prA);

@@ -98,9 +98,10 @@ struct DecodeSmem {
   static constexpr int kTilesBytes = Gm::kWarps * Gm::kStages * Gm::kTile;
   static constexpr int kSideBytes = Gm::kWarps * Gm::kStages * Gm::kSideStride;
   static constexpr int kBarBytes = Gm::kWarps * Gm::kStages * 8;
-  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 2 : 0;  // per-warp f16 q copy
+  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 2 : 0;     // per-warp f16 q copy
+  static constexpr int kOextBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 4 : 0;  // per-warp outlier-channel O
   static size_t bytes(int B) {
-    return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + (size_t)(B + 1) * 4;
+    return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + kOextBytes + (size_t)(B + 1) * 4;
   }
 };
 
