@@ -13,6 +13,7 @@ cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& t
                           int grid, cudaStream_t st);
 cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
 size_t decode_smem_bytes(int kv_dtype, int D, int B);
+int decode_warps(int kv_dtype, int D);
 }  // namespace pqkv
 
 using namespace pqkv;
@@ -104,10 +105,9 @@ bool cached_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb,
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace = plan header (chunk length + block prefix per sequence, written by
-// the decode kernel, read by the merge kernel) followed by two partial-result
-// slots per chunk. Nothing in it needs to be initialized by the caller.
-size_t plan_bytes(int batch) { return round_up((size_t)(batch + 2) * 4, 256); }
+// Workspace = two partial-result slots per chunk of the split, written by the
+// decode kernel before the merge kernel reads them; nothing in it needs to be
+// initialized by the caller.
 
 }  // namespace
 
@@ -185,7 +185,7 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
   const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
   const size_t chunks = split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks
                                          : (size_t)di.sms * kDecodeWarps;
-  return plan_bytes(batch) + 2 * chunks * slot;
+  return 2 * chunks * slot;
 }
 
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_stream_t stream) {
@@ -236,8 +236,7 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   p.block_tables = block_tables;
   p.seq_lens = seq_lens;
   p.err = err_flag;
-  p.plan = static_cast<int32_t*>(workspace);
-  p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + plan_bytes(batch));
+  p.partials = static_cast<float*>(workspace);
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
@@ -252,13 +251,16 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms, st);
   if (e != cudaSuccess) return PQKV_ERR_CUDA;
   MergeParams mp;
-  mp.plan = p.plan;
+  mp.seq_lens = seq_lens;
   mp.partials = p.partials;
   mp.out = out;
   mp.B = batch;
   mp.Hq = num_q_heads;
   mp.Hkv = num_kv_heads;
   mp.G = p.G;
+  mp.maxblk = max_blocks_per_seq;
+  mp.warps = di.sms * decode_warps(kv_dtype, head_dim);
+  mp.split_blocks = split_blocks;
   mp.slot_floats = p.slot_floats;
   e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;

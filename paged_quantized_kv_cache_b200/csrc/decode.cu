@@ -360,22 +360,52 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
 // the pieces are combined as M = max_j m_j, L = sum_j l_j 2^(m_j - M),
 // out = sum_j O_j 2^(m_j - M) / L, in fixed piece order). One warp per
 // (sequence b, KV head h, query head n of the group). Launched as a
-// programmatic dependent of the decode kernel: it waits for that grid before
-// reading the plan and the partials it wrote.
+// programmatic dependent of the decode kernel: it rebuilds the decode's split
+// plan from seq_lens while that grid is still running and waits for it only
+// before reading the partials.
 // ---------------------------------------------------------------------------
 template <int D, bool QBF16>
 __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  extern __shared__ int P[];  // [B + 1]: blocks of the sequences before b, as in the decode
+  __shared__ int wsum[4];
   constexpr int DPL = D / 32;
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  {
+    const int B = p.B, per = (B + 127) / 128;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    const int lim = kBlock * p.maxblk;
+    int local = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      local += (L < 0 || L > lim) ? 0 : (L + kBlock - 1) / kBlock;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < warp; ++w) run += wsum[w];
+    if (tid == 0) P[0] = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      run += (L < 0 || L > lim) ? 0 : (L + kBlock - 1) / kBlock;
+      P[i + 1] = run;
+    }
+    __syncthreads();
+  }
+  const int T = p.Hkv * P[p.B];
+  const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + p.warps - 1) / p.warps);
   const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (wid >= (long)p.B * p.Hq) return;
   const int b = (int)(wid / p.Hq), hq = (int)(wid % p.Hq);
   const int h = hq / p.G, n = hq % p.G;
-  const int Qc = p.plan[0];
-  const int Pb = p.plan[1 + b], nblk = p.plan[2 + b] - Pb;
+  const int nblk = P[b + 1] - P[b];
   if (nblk == 0) return;
-  const int s0 = p.Hkv * Pb + h * nblk;
+  const int s0 = p.Hkv * P[b] + h * nblk;
   const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
   if (k0 == k1) return;  // the pair was finished inside one chunk
   const int np = k1 - k0 + 1;
@@ -383,16 +413,23 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     const int kk = k0 + i;
     return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
   };
-  // weights: lanes over pieces
-  float M = kNegInf;
-  for (int i = lane; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // weights: lanes over pieces; lane i keeps piece i's (m, l) for the common np <= 32
+  float mi = kNegInf, li = 0.f;
+  if (lane < np) {
+    const float* bs = slot_base(lane);
+    mi = __ldcg(bs + p.G * D + n);
+    li = __ldcg(bs + p.G * D + p.G + n);
+  }
+  float M = mi;
+  for (int i = lane + 32; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-  float L = 0.f;
-  for (int i = lane; i < np; i += 32) {
+  const float wi = (M == kNegInf || lane >= np) ? 0.f : exp2f(mi - M);
+  float L = wi * li;
+  for (int i = lane + 32; i < np; i += 32) {
     const float* bs = slot_base(i);
-    const float m = __ldcg(bs + p.G * D + n);
-    L += (M == kNegInf) ? 0.f : exp2f(m - M) * __ldcg(bs + p.G * D + p.G + n);
+    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M) * __ldcg(bs + p.G * D + p.G + n);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
@@ -403,8 +440,8 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
 #pragma unroll 4
   for (int i = 0; i < np; ++i) {
     const float* bs = slot_base(i);
-    const float m = __ldcg(bs + p.G * D + n);
-    const float w = (M == kNegInf) ? 0.f : exp2f(m - M);
+    float w = __shfl_sync(kFull, wi, i & 31);
+    if (i >= 32) w = (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M);
     if constexpr (DPL == 4) {
       const float4 v = __ldcg(reinterpret_cast<const float4*>(bs + n * D + lane * 4));
       acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
@@ -425,6 +462,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   using Gm = DecodeGeom<KVF, D>;
   using Sm = DecodeSmem<KVF, D>;
   constexpr int NW = Gm::kWarps;
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // inputs may come from the previous kernel
   constexpr int NS = Gm::kStages;
   constexpr int KT = D / 16;  // k-steps of QK^T and m-tiles of PV
   constexpr bool kBf16Mma = (KVF == PQKV_DTYPE_BF16);
@@ -500,10 +538,6 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   const int W = gridDim.x * NW;
   const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + W - 1) / W);
   const int K = T > 0 ? (T + Qc - 1) / Qc : 0;
-  if (blockIdx.x == 0) {  // the plan the merge kernel reads
-    if (tid == 0) p.plan[0] = Qc;
-    for (int i = tid; i <= B; i += blockDim.x) p.plan[1 + i] = P[i];
-  }
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   uint32_t phase = 0;     // parity bit per stage
@@ -875,7 +909,21 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
-  kern<<<grid, DecodeGeom<KVF, D>::kWarps * 32, smem, st>>>(tmap, p);
+  // programmatic dependent of whatever precedes it on the stream (usually the
+  // cache write): the kernel waits for that grid before its first read, so
+  // only the launch overlaps
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(DecodeGeom<KVF, D>::kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -887,7 +935,7 @@ cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
   cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = (size_t)(p.B + 1) * 4;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -899,6 +947,19 @@ cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t 
                   : cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, false>, p);
   return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, true>, p)
                 : cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, false>, p);
+}
+
+int decode_warps(int kv_dtype, int D) {
+  switch (kv_dtype) {
+    case PQKV_DTYPE_FP16:
+    case PQKV_DTYPE_BF16:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_BF16, 128>::kWarps : DecodeGeom<PQKV_DTYPE_BF16, 64>::kWarps;
+    case PQKV_DTYPE_FP8_E4M3:
+    case PQKV_DTYPE_FP8_E5M2:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP8_E4M3, 128>::kWarps : DecodeGeom<PQKV_DTYPE_FP8_E4M3, 64>::kWarps;
+    default:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP4_E2M1, 128>::kWarps : DecodeGeom<PQKV_DTYPE_FP4_E2M1, 64>::kWarps;
+  }
 }
 
 size_t decode_smem_bytes(int kv_dtype, int D, int B) {

@@ -43,7 +43,6 @@ struct DecodeParams {
   const int32_t* block_tables;  // [B][maxblk]
   const int32_t* seq_lens;      // [B]
   int32_t* err;
-  int32_t* plan;                // workspace header: [0] = chunk length, [1..B+1] = block prefix P
   float* partials;              // [2 * chunks][slot_floats]
   int B, Hq, Hkv, G, nb, maxblk;
   int split_blocks;
@@ -53,10 +52,12 @@ struct DecodeParams {
 };
 
 struct MergeParams {
-  const int32_t* plan;
+  const int32_t* seq_lens;
   const float* partials;
   void* out;
-  int B, Hq, Hkv, G;
+  int B, Hq, Hkv, G, maxblk;
+  int warps;         // warps of the decode grid (its balanced chunk length depends on it)
+  int split_blocks;
   int slot_floats;
 };
 

@@ -73,6 +73,9 @@ __device__ __forceinline__ int run_length(const WriteParams& p, int ts, int s0, 
 // ---- 16-bit formats: one warp copies the K and V rows of one (token, head) ----
 template <int D>
 __global__ void __launch_bounds__(256) write16_kernel(const WriteParams p) {
+  // inputs may come from the previous kernel; let the next one start launching
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (wid >= (long)p.T * p.Hkv) return;
@@ -95,6 +98,9 @@ __global__ void __launch_bounds__(256) write16_kernel(const WriteParams p) {
 // ---- FP8: absmax scale per (block, head, K|V), grown on append ----
 template <int KVF, int D, bool INBF16>
 __global__ void __launch_bounds__(128) write_fp8_kernel(const WriteParams p) {
+  // inputs may come from the previous kernel; let the next one start launching
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int CPL = D / 32;  // channels per lane
   constexpr float kMax = (KVF == PQKV_DTYPE_FP8_E4M3) ? 448.0f : 57344.0f;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -173,6 +179,9 @@ __global__ void __launch_bounds__(128) write_fp8_kernel(const WriteParams p) {
 // ---- FP4 E2M1 + FP16 outlier channels ----
 template <int D, bool INBF16>
 __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
+  // inputs may come from the previous kernel; let the next one start launching
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   constexpr int CPL = D / 32;          // channels per lane
   constexpr int LPG = kGroup / CPL;    // lanes per 16-channel group
   __shared__ float s_norm[4][D];
@@ -346,22 +355,38 @@ __global__ void encode_kernel(const float* x, int64_t n, uint8_t* out) {
 
 // ---- launchers --------------------------------------------------------------
 
+// Launch as a programmatic dependent of the previous kernel on the stream (the
+// kernels wait for it at entry, so only the launch overlaps).
+template <typename... Args>
+static cudaError_t launch_pdl(void (*kern)(Args...), dim3 grid, unsigned block, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 cudaError_t launch_write(int kv_dtype, int in_dtype, int D, const WriteParams& p, cudaStream_t st) {
   if (p.T <= 0) return cudaSuccess;
   const bool bf = (in_dtype == PQKV_DTYPE_BF16);
   if (kv_dtype == PQKV_DTYPE_FP16 || kv_dtype == PQKV_DTYPE_BF16) {
     const long warps = (long)p.T * p.Hkv;
     const int grid = (int)((warps + 7) / 8);
-    if (D == 128) write16_kernel<128><<<grid, 256, 0, st>>>(p);
-    else write16_kernel<64><<<grid, 256, 0, st>>>(p);
-    return cudaGetLastError();
+    return D == 128 ? launch_pdl(write16_kernel<128>, dim3(grid), 256, st, p)
+                    : launch_pdl(write16_kernel<64>, dim3(grid), 256, st, p);
   }
   // a warp owns the runs starting in a window of tpw tokens of one (head, K|V)
   WriteParams q = p;
   q.tpw = (p.T <= 8192) ? 1 : 32;
   const dim3 grid((unsigned)((p.T + 4 * q.tpw - 1) / (4 * q.tpw)), (unsigned)p.Hkv, 2u);
 #define PQKV_W8(F, DD, B) \
-  if (kv_dtype == F && D == DD && bf == B) { write_fp8_kernel<F, DD, B><<<grid, 128, 0, st>>>(q); return cudaGetLastError(); }
+  if (kv_dtype == F && D == DD && bf == B) return launch_pdl(write_fp8_kernel<F, DD, B>, grid, 128, st, q);
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 128, true)
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 128, false)
   PQKV_W8(PQKV_DTYPE_FP8_E4M3, 64, true)
@@ -372,14 +397,11 @@ cudaError_t launch_write(int kv_dtype, int in_dtype, int D, const WriteParams& p
   PQKV_W8(PQKV_DTYPE_FP8_E5M2, 64, false)
 #undef PQKV_W8
   if (kv_dtype == PQKV_DTYPE_FP4_E2M1) {
-    if (D == 128) {
-      if (bf) write_fp4_kernel<128, true><<<grid, 128, 0, st>>>(q);
-      else write_fp4_kernel<128, false><<<grid, 128, 0, st>>>(q);
-    } else {
-      if (bf) write_fp4_kernel<64, true><<<grid, 128, 0, st>>>(q);
-      else write_fp4_kernel<64, false><<<grid, 128, 0, st>>>(q);
-    }
-    return cudaGetLastError();
+    if (D == 128)
+      return bf ? launch_pdl(write_fp4_kernel<128, true>, grid, 128, st, q)
+                : launch_pdl(write_fp4_kernel<128, false>, grid, 128, st, q);
+    return bf ? launch_pdl(write_fp4_kernel<64, true>, grid, 128, st, q)
+              : launch_pdl(write_fp4_kernel<64, false>, grid, 128, st, q);
   }
   return cudaErrorInvalidValue;
 }
