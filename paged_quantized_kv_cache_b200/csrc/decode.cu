@@ -433,21 +433,37 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
-  // outputs: lanes over head dims, pieces in order
+  // outputs: lanes over head dims, pieces in order; the loads of up to 16
+  // pieces are all issued before the first one is folded in
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-#pragma unroll 4
-  for (int i = 0; i < np; ++i) {
-    const float* bs = slot_base(i);
-    float w = __shfl_sync(kFull, wi, i & 31);
-    if (i >= 32) w = (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M);
-    if constexpr (DPL == 4) {
-      const float4 v = __ldcg(reinterpret_cast<const float4*>(bs + n * D + lane * 4));
-      acc[0] += w * v.x; acc[1] += w * v.y; acc[2] += w * v.z; acc[3] += w * v.w;
-    } else {
+  constexpr int kBatch = 16;
+  for (int i0 = 0; i0 < np; i0 += kBatch) {
+    float v[kBatch][DPL];
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] += w * __ldcg(bs + n * D + lane * DPL + e);
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u;
+      if (i < np) {
+        const float* bs = slot_base(i) + n * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(bs));
+          v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) v[u][e] = __ldcg(bs + e);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u;
+      float w = __shfl_sync(kFull, wi, i & 31);
+      if (i < np) {
+        if (i >= 32) w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + p.G * D + n) - M);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] += w * v[u][e];
+      }
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
