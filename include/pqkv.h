@@ -38,8 +38,14 @@
  *   FP8 E4M3/E5M2: cache [nb][H][2][16][D] one code per byte
  *                 scales [nb][H][4] float32 = {scale_K, scale_V, 0, 0}
  *                 (value = decode(code) * scale; 16-byte granule per pair)
- *   FP4 E2M1    : cache  [nb][H][2][16][D/2] bytes, channel 2i in the low nibble,
- *                 channel 2i+1 in the high nibble
+ *   FP4 E2M1    : cache  [nb][H][2][16][D/2] bytes of two E2M1 codes each
+ *                 K rows: row t = token t; byte i = channel 2i (low nibble)
+ *                 and channel 2i+1 (high nibble)
+ *                 V rows: one byte = one channel of a token pair. Pair p = 2k
+ *                 (k < 4) is tokens (2k, 2k+1), pair p = 2k+1 is tokens
+ *                 (2k+8, 2k+9); the even token takes the low nibble. Row p
+ *                 holds channels [0, D/2) of pair p, row 8+p channels
+ *                 [D/2, D); byte b of a row = channel b (+ D/2)
  *                 scales [nb][H][2][16][D/16] unsigned E4M3 codes, one per
  *                 16 consecutive channels of one token
  *                 outliers_idx [nb][H][2][8] uint8: slots 0..3 hold the outlier

@@ -194,17 +194,34 @@ static uint16_t* fp4_val_ptr(const cache_t* c, int blk, int h, int kv, int t) {
   return (uint16_t*)(c->oval + ((tile_index(c, blk, h, kv) * BS + t) * R_OUT) * 2);
 }
 
+/* Where the E2M1 code of (token t, channel ch) lives, and in which nibble.
+ * The storage order is this library's own (the pages fix none):
+ *  K tile: row t holds token t; byte i = channels 2i (low nibble), 2i + 1.
+ *  V tile: byte = one channel of two tokens. Tokens (t, t + 1), t even, form a
+ *    pair; pair p = 2k (k < 4) is tokens (2k, 2k + 1), pair 2k + 1 is tokens
+ *    (2k + 8, 2k + 9); the even token is the low nibble. Channels [0, D/2) of
+ *    pair p sit in row p, channels [D/2, D) in row 8 + p, byte = ch mod D/2. */
+static uint8_t* fp4_code_byte(const cache_t* c, int blk, int h, int kv, int t, int ch, int* shift) {
+  if (kv == 0) {
+    *shift = (ch & 1) ? 4 : 0;
+    return row_ptr(c, blk, h, kv, t) + ch / 2;
+  }
+  const int half = c->D / 2;
+  const int pair = (t < 8) ? (t & ~1) : (((t - 8) & ~1) + 1);
+  *shift = (t & 1) ? 4 : 0;
+  return row_ptr(c, blk, h, kv, (ch / half) * 8 + pair) + ch % half;
+}
+
 static int fp4_get_code(const cache_t* c, int blk, int h, int kv, int t, int ch) {
-  uint8_t byte = row_ptr(c, blk, h, kv, t)[ch / 2];
-  return (ch & 1) ? (byte >> 4) : (byte & 0xF);
+  int shift;
+  const uint8_t byte = *fp4_code_byte(c, blk, h, kv, t, ch, &shift);
+  return (byte >> shift) & 0xF;
 }
 
 static void fp4_set_code(const cache_t* c, int blk, int h, int kv, int t, int ch, int code) {
-  uint8_t* p = row_ptr(c, blk, h, kv, t) + ch / 2;
-  if (ch & 1)
-    *p = (uint8_t)((*p & 0x0F) | (code << 4));
-  else
-    *p = (uint8_t)((*p & 0xF0) | code);
+  int shift;
+  uint8_t* p = fp4_code_byte(c, blk, h, kv, t, ch, &shift);
+  *p = (uint8_t)((*p & ~(0xF << shift)) | (code << shift));
 }
 
 /* Dequantized value of channel ch of token offset t ([P1] step 4 for FP4: the

@@ -13,7 +13,9 @@ constexpr float kNegInf = -INFINITY;
 // The running max m is only moved (and O, l rescaled) when a block's max
 // exceeds it by more than this many log2 units, so most blocks skip the
 // rescale; probabilities then stay below 2^kLazy, well inside f16 / bf16.
-constexpr float kLazy = 8.f;
+// FP4 multiplies P by E4M3 group scales (<= 448) in f16, so it keeps P <= 16.
+template <int KVF>
+constexpr float lazy_of() { return KVF == PQKV_DTYPE_FP4_E2M1 ? 4.f : 8.f; }
 
 // Zero the low (token t0) / high (token t0 + 1) half of a packed pair when the
 // token lies past the end of the sequence (its bytes may hold anything).
@@ -83,9 +85,15 @@ struct LdsmOffsets {
       if constexpr (Gm::k16) {
         k[i] = Gm::off(((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
         v[i] = Gm::off(16 + ((mi >> 1) << 3) + ri, (2 * i + (mi & 1)) * 16);
-      } else {
+      } else if constexpr (Gm::kFp8) {
         k[i] = Gm::off(((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
         v[i] = Gm::off(16 + ((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
+      } else {
+        // V: matrix mi of load i is m-tile c = 4i + mi, the 8 pair rows of
+        // its half of the channels at the 16-byte column of its 16 channels
+        const int c = 4 * i + mi;
+        k[i] = Gm::off(((mi & 1) << 3) + ri, (2 * i + (mi >> 1)) * 16);
+        v[i] = Gm::off(16 + 8 * (c / (D / 32)) + ri, 16 * (c % (D / 32)));
       }
     }
   }
@@ -98,13 +106,8 @@ template <int KVF>
 __device__ __forceinline__ int dmap(int mt, int rr) {
   if constexpr (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16) {
     return 16 * mt + rr;
-  } else if constexpr (KVF == PQKV_DTYPE_FP4_E2M1) {
-    // tiles (2c, 2c+1) cover d in [32c, 32c + 32): tile 2c+e, row g -> 32c + 4g + 2e,
-    // row g + 8 -> 32c + 4g + 2e + 1
-    const int c = mt >> 1, e = mt & 1;
-    return 32 * c + 4 * (rr & 7) + 2 * e + (rr >> 3);
   } else {
-    // FP8: tile c covers [16c, 16c + 16): row g -> 16c + 2g, row g + 8 -> 16c + 2g + 1
+    // FP8, FP4: tile c covers [16c, 16c + 16): row g -> 16c + 2g, row g + 8 -> 16c + 2g + 1
     return 16 * mt + 2 * (rr & 7) + (rr >> 3);
   }
 }
@@ -197,8 +200,8 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
         const int r0i = idx[2 * qd], r1i = idx[2 * qd + 1];
         a0 = (uint32_t)kv[g * 4 + 2 * qd] | ((uint32_t)kv[g * 4 + 2 * qd + 1] << 16);
         a1 = (uint32_t)kv[(g + 8) * 4 + 2 * qd] | ((uint32_t)kv[(g + 8) * 4 + 2 * qd + 1] << 16);
-        const uint32_t q0 = (r0i < D) ? wq[g * D + r0i] : 0u;
-        const uint32_t q1 = (r1i < D) ? wq[g * D + r1i] : 0u;
+        const uint32_t q0 = (r0i < D) ? wq[g * Gm::kQStride + r0i] : 0u;
+        const uint32_t q1 = (r1i < D) ? wq[g * Gm::kQStride + r1i] : 0u;
         b0 = q0 | (q1 << 16);
         if (r0i >= D) { a0 &= 0xFFFF0000u; a1 &= 0xFFFF0000u; }
         if (r1i >= D) { a0 &= 0x0000FFFFu; a1 &= 0x0000FFFFu; }
@@ -266,61 +269,42 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
       }
     }
   } else {
-    // FP4: ldmatrix.trans gives lane (g, qd) the codes d0 = 32c + 4g .. +3 of
-    // tokens 2qd, 2qd + 1; a nibble transpose pairs the tokens per d, and each
-    // pair is multiplied by the two tokens' E4M3 scales of group 2c + g/4.
+    // FP4: a V byte holds one channel of a token pair, so ldmatrix.trans of 8
+    // pair rows hands lane (g, qd) the whole A fragment of m-tile c in one word:
+    // d = 16c + 2g, 16c + 2g + 1 of tokens (2qd, 2qd + 1) and (2qd + 8, 2qd + 9).
+    // m-tile c is scale group c, so the tokens' E4M3 group scales multiply P
+    // (in f16: P <= 16, scale <= 448) instead of the codes.
     constexpr int SPR = D / 16;
     const uint8_t* vs = side + 16 * SPR;  // V scales [16][D/16]
-    const int gs = g >> 2;
-    // scale pairs (token t, t + 1) of chunk c: bytes 2c + g/4 of the two tokens'
-    // scale rows, picked from whole words
-    uint32_t sp[2][D / 32];
-    {
-      const uint32_t sel = (uint32_t)(gs | ((4 + gs) << 4) | ((2 + gs) << 8) | ((6 + gs) << 12));
+    uint32_t sp[2][D / 16];               // (s(t, c), s(t + 1, c)), t = 2qd | 2qd + 8
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int ta = 2 * qd + 8 * hh;
-        const uint32_t* w0 = reinterpret_cast<const uint32_t*>(vs + ta * SPR);
-        const uint32_t* w1 = reinterpret_cast<const uint32_t*>(vs + (ta + 1) * SPR);
+    for (int hh = 0; hh < 2; ++hh) {
+      const int ta = 2 * qd + 8 * hh;
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(vs + ta * SPR);
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(vs + (ta + 1) * SPR);
 #pragma unroll
-        for (int w = 0; w < SPR / 4; ++w)
-          dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], sel), sp[hh][2 * w], sp[hh][2 * w + 1]);
+      for (int w = 0; w < SPR / 4; ++w) {
+        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], 0x5140u), sp[hh][4 * w], sp[hh][4 * w + 1]);
+        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], 0x7362u), sp[hh][4 * w + 2], sp[hh][4 * w + 3]);
+      }
+      if (valid < kBlock) {  // scales past the end may be NaN codes
+#pragma unroll
+        for (int c = 0; c < D / 16; ++c) sp[hh][c] = mask_pair(sp[hh][c], ta, valid);
       }
     }
 #pragma unroll
-    for (int cp = 0; cp < D / 64; ++cp) {
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4_t(tb + lo.v[cp], r0, r1, r2, r3);
+    for (int i = 0; i < D / 64; ++i) {
+      uint32_t r[4];
+      ldsm_x4_t(tb + lo.v[i], r[0], r[1], r[2], r[3]);
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int c = 2 * cp + e;
-        uint32_t fa[4], fb[4];
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const uint32_t x = hh ? (e ? r3 : r1) : (e ? r2 : r0);
-          const uint32_t lo = x & 0x0F0F0F0Fu, hi = (x >> 4) & 0x0F0F0F0Fu;
-          const uint32_t A = prmt(lo, hi, 0x5140u), Bv = prmt(lo, hi, 0x7362u);
-          const uint32_t nib = A | (Bv << 4);  // bytes: d0, d0+1, d0+2, d0+3 (token pair)
-          const __half2 scl = *reinterpret_cast<const __half2*>(&sp[hh][c]);
-          uint32_t dv[4];
-          dec_e2m1x8(nib, dv);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __half2 w = __hmul2(*reinterpret_cast<__half2*>(&dv[i]), scl);
-            if (hh) fb[i] = *reinterpret_cast<uint32_t*>(&w);
-            else fa[i] = *reinterpret_cast<uint32_t*>(&w);
-          }
-        }
-        if (valid < kBlock) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            fa[i] = mask_pair(fa[i], t0, valid);
-            fb[i] = mask_pair(fb[i], t1, valid);
-          }
-        }
-        // tile 2c: rows g -> d0, g+8 -> d0+1; tile 2c+1: rows g -> d0+2, g+8 -> d0+3
-        mma_pv(acc[2 * c], fa[0], fa[1], fb[0], fb[1]);
-        mma_pv(acc[2 * c + 1], fa[2], fa[3], fb[2], fb[3]);
+      for (int e = 0; e < 4; ++e) {
+        const int c = 4 * i + e;
+        uint32_t a[4];
+        dec_e2m1x8(r[e], a);
+        const __half2 p0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), *reinterpret_cast<const __half2*>(&sp[0][c]));
+        const __half2 p1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), *reinterpret_cast<const __half2*>(&sp[1][c]));
+        mma16816<false>(acc[c], a[0], a[1], a[2], a[3], *reinterpret_cast<const uint32_t*>(&p0),
+                        *reinterpret_cast<const uint32_t*>(&p1));
       }
     }
     // outlier channels: Oext[n][idx_r] += (Vout^T (4 slots x 16 tokens) P^T)[r][n].
@@ -344,8 +328,8 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
       if (g < 4) {
         const int dch = idx[g];
         if (dch < D) {
-          oext[(2 * qd) * D + dch] += ex[0];
-          oext[(2 * qd + 1) * D + dch] += ex[1];
+          oext[(2 * qd) * Gm::kOStride + dch] += ex[0];
+          oext[(2 * qd + 1) * Gm::kOStride + dch] += ex[1];
         }
       }
       __syncwarp();
@@ -499,10 +483,10 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   uint64_t* wbar = bars + warp * NS;
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
-  uint16_t* wq = qcopy + warp * 8 * D;
-  float* woext = oext_all + warp * 8 * D;  // FP4: O of outlier channels [8 heads][D]
+  uint16_t* wq = qcopy + warp * 8 * Gm::kQStride;
+  float* woext = oext_all + warp * 8 * Gm::kOStride;  // FP4: O of outlier channels [8 heads][D (+pad)]
   if constexpr (Gm::kFp4)
-    for (int i = lane; i < 8 * D; i += 32) woext[i] = 0.f;
+    for (int i = lane; i < 8 * Gm::kOStride; i += 32) woext[i] = 0.f;
   const LdsmOffsets<KVF, D> lofs(lane);
 
   if (lane == 0) {
@@ -681,7 +665,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         for (int i = lane; i < 8 * D; i += 32) {
           const int n = i / D;
           const float v = (n < G) ? q_at<QBF16>(p.q, ((size_t)b * Hq + (size_t)h * G + n) * D + (i % D)) : 0.f;
-          wq[i] = __half_as_ushort(__float2half_rn(v));
+          wq[n * Gm::kQStride + i % D] = __half_as_ushort(__float2half_rn(v));
         }
         __syncwarp();
       }
@@ -702,7 +686,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         for (int mt = 0; mt < KT; ++mt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            float* slot = woext + (2 * qd + (e & 1)) * D + dmap<KVF>(mt, g + 8 * (e >> 1));
+            float* slot = woext + (2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1));
             acc[mt][e] += *slot;
             *slot = 0.f;
           }
@@ -806,6 +790,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
         bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
       }
+      constexpr float kLazy = lazy_of<KVF>();
       const bool need0 = bm0 > m0 + kLazy, need1 = bm1 > m1 + kLazy;
       float f0c = 1.f, f1c = 1.f;
       bool rescale = __any_sync(kFull, need0 || need1);
@@ -844,7 +829,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
           for (int mt = 0; mt < KT; ++mt)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
-              woext[(2 * qd + (e & 1)) * D + dmap<KVF>(mt, g + 8 * (e >> 1))] *= (e & 1) ? f1c : f0c;
+              woext[(2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1))] *= (e & 1) ? f1c : f0c;
           __syncwarp();
         }
       }

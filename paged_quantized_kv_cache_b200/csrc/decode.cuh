@@ -81,6 +81,9 @@ struct DecodeGeom {
   static constexpr int kWarps = k16 ? (D == 128 ? 6 : 8) : 12;
   static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 4 : 6) : (D == 128 ? 4 : 6));
   static constexpr uint32_t kTx = kTile + kSide;
+  // FP4 per-warp shared rows, padded so that the 8 rows fall in different banks
+  static constexpr int kQStride = D + 2;  // f16 query copy, halves per row
+  static constexpr int kOStride = D + 1;  // outlier-channel O, floats per row
   // byte offset in a tile of (row r, byte b of that row); rows 0-15 K, 16-31 V.
   __device__ static __forceinline__ uint32_t off(int r, int b) {
     const int box = b / kBoxRow;
@@ -99,8 +102,8 @@ struct DecodeSmem {
   static constexpr int kTilesBytes = Gm::kWarps * Gm::kStages * Gm::kTile;
   static constexpr int kSideBytes = Gm::kWarps * Gm::kStages * Gm::kSideStride;
   static constexpr int kBarBytes = Gm::kWarps * Gm::kStages * 8;
-  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 2 : 0;     // per-warp f16 q copy
-  static constexpr int kOextBytes = Gm::kFp4 ? Gm::kWarps * 8 * D * 4 : 0;  // per-warp outlier-channel O
+  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * Gm::kQStride * 2 : 0;     // per-warp f16 q copy
+  static constexpr int kOextBytes = Gm::kFp4 ? Gm::kWarps * 8 * Gm::kOStride * 4 : 0;  // per-warp outlier-channel O
   static size_t bytes(int B) {
     return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + kOextBytes + (size_t)(B + 1) * 4;
   }

@@ -288,6 +288,7 @@ __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
         is_out[e] = (c == oc[0]) || (c == oc[1]) || (c == oc[2]) || (c == oc[3]);
       }
       // step 3: per token, fp16 outlier values, E4M3 group scales, E2M1 codes
+      uint32_t vpend = 0;  // V codes of the even token of a pair, stored with its partner
 #pragma unroll
       for (int j = 0; j < kBlock; ++j) {
         if (j >= n) break;
@@ -325,12 +326,38 @@ __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
         float y[CPL];
 #pragma unroll
         for (int e = 0; e < CPL; ++e) y[e] = (is_out[e] || sd == 0.f) ? 0.f : __fdiv_rn(xs[j][e], sd);
-        uint8_t* crow = p.cache + (tile * kBlock + row) * (D / 2) + lane * (CPL / 2);
-        if constexpr (CPL == 4) {
-          const uint32_t c = enc_e2m1x2(y[0], y[1]) | (enc_e2m1x2(y[2], y[3]) << 8);
-          *reinterpret_cast<uint16_t*>(crow) = (uint16_t)c;
+        const uint32_t c01 = enc_e2m1x2(y[0], y[1]);
+        const uint32_t c23 = (CPL == 4) ? enc_e2m1x2(y[2], y[3]) : 0u;
+        if (kv == 0) {
+          // K: one row per token, channel 2i in the low nibble of byte i
+          uint8_t* crow = p.cache + (tile * kBlock + row) * (D / 2) + lane * (CPL / 2);
+          if constexpr (CPL == 4)
+            *reinterpret_cast<uint16_t*>(crow) = (uint16_t)(c01 | (c23 << 8));
+          else
+            *crow = (uint8_t)c01;
         } else {
-          *crow = (uint8_t)enc_e2m1x2(y[0], y[1]);
+          // V: a byte holds one channel of a token pair (even token in the low
+          // nibble). Pairs inside the run are stored whole; a pair split by the
+          // run's ends keeps the other token's nibbles.
+          const uint32_t cw = (c01 & 0xFu) | ((c01 >> 4) << 8) | ((c23 & 0xFu) << 16) | ((c23 >> 4) << 24);
+          const int pr = (row < 8) ? (row & ~1) : (((row - 8) & ~1) + 1);
+          const int cb = lane * CPL;
+          uint8_t* vb = p.cache + (tile * kBlock + 8 * (cb / (D / 2)) + pr) * (D / 2) + cb % (D / 2);
+          const bool odd = row & 1;
+          if (!odd && j + 1 < n) {
+            vpend = cw;
+          } else {
+            const int sh = odd ? 4 : 0;
+            uint32_t keep = odd ? 0x0F0F0F0Fu : 0xF0F0F0F0u, put = cw << sh;
+            if (odd && j > 0) { keep = 0u; put |= vpend; }
+            if constexpr (CPL == 4) {
+              uint32_t* w = reinterpret_cast<uint32_t*>(vb);
+              *w = (keep ? (*w & keep) : 0u) | put;
+            } else {
+              uint16_t* w = reinterpret_cast<uint16_t*>(vb);
+              *w = (uint16_t)((keep ? (*w & keep) : 0u) | put);
+            }
+          }
         }
         if ((lane % LPG) == 0)
           p.scales[(tile * kBlock + row) * (D / kGroup) + (lane * CPL) / kGroup] = (uint8_t)sc;

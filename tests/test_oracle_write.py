@@ -89,13 +89,54 @@ def test_fp4_hand_example():
     idx = c.oidx.reshape(nb, H, 2, 8)
     val = c.oval.view(np.uint16).reshape(nb, H, 2, 16, 4)
     hexs = lambda xs: np.array([int(x, 16) for x in xs])
+    for t in range(16):
+        np.testing.assert_array_equal(rows[0, 0, 0, t], hexs(g["k_row_bytes"]))
+        want_v = g["v_rows_0_to_7"] if t < 8 else g["v_rows_8_to_15"]
+        np.testing.assert_array_equal(rows[0, 0, 1, t], hexs(want_v))
     for kv, name in ((0, "k"), (1, "v")):
         for t in range(16):
-            np.testing.assert_array_equal(rows[0, 0, kv, t], hexs(g[name + "_row_bytes"]))
             np.testing.assert_array_equal(scl[0, 0, kv, t], hexs(g[name + "_scales"]))
             np.testing.assert_array_equal(val[0, 0, kv, t], hexs(g[name + "_vals"]))
         np.testing.assert_array_equal(idx[0, 0, kv], hexs(g[name + "_idx"]))
     assert (rows[1] == 0xFF).all()
+
+
+# E2M1 magnitudes in code order (OCP Microscaling Formats, E2M1).
+_E2M1_MAGS = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_fp4_v_tile_pair_order(D):
+    """The V tile's storage order as include/pqkv.h states it: one byte holds one
+    channel of a token pair, pair p = 2k is tokens (2k, 2k+1), pair 2k+1 is tokens
+    (2k+8, 2k+9), even token in the low nibble, channels [0, D/2) in row p and
+    [D/2, D) in row 8+p. Each token gets codes known by construction: channel c of
+    token t is the E2M1 value of magnitude code (t + 3c) % 8 with sign (-1)^(c // 2)
+    (zero kept positive),
+    so every 16-channel group reaches 6 (scale 6/6 = 1, exact) and every channel
+    reaches norm 6 (variance 0: channels 0-3 are the outliers, their codes 0)."""
+    t = np.arange(16)[:, None]
+    c = np.arange(D)[None, :]
+    mag = (t + 3 * c) % 8
+    sign = np.where((c // 2) % 2 == 0, 1.0, -1.0)
+    x = np.where(mag == 0, 0.0, np.array(_E2M1_MAGS)[mag] * sign).astype(np.float32)[:, None, :]
+    code = mag | np.where((sign < 0) & (mag > 0), 8, 0)
+    code[:, :4] = 0
+    cache = oracle.Cache(oracle.DT_E2M1, 1, 1, D)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    assert oracle.kv_cache_write(cache, xt, xt, np.arange(16, dtype=np.int32)) == 0
+    rows, scl, idx, _ = _fp4_views(cache)
+    assert list(idx[0, 0, 1][:4]) == [0, 1, 2, 3]
+    assert (scl[0, 0, 1] == 0x38).all()  # E4M3 1.0
+    half = D // 2
+    for p in range(8):
+        ta = p if p % 2 == 0 else p + 7
+        for part in range(2):
+            chans = np.arange(half) + part * half
+            want = code[ta, chans] | (code[ta + 1, chans] << 4)
+            np.testing.assert_array_equal(rows[0, 0, 1, 8 * part + p], want)
+    # K keeps one row per token, channel 2i in the low nibble
+    np.testing.assert_array_equal(_fp4_codes(rows[0, 0, 0]), code)
 
 
 @pytest.mark.parametrize("dt", [oracle.DT_FP16, oracle.DT_BF16])
