@@ -16,6 +16,10 @@ bracketed by barriers and the time taken is the maximum over ranks.
 
 --impl reference times the CPU oracle (the fp64 restatement used by the tests)
 on a bounded sample of the same workload on the host cores.
+
+--op copy_blocks | swap measures the whole-block moves instead (copy-on-write
+copies inside the cache; swap of blocks to pinned host memory and back) on the
+workload's cache format; one JSON line of the same shape.
 """
 from __future__ import annotations
 
@@ -562,6 +566,145 @@ def run_e2e(st: Setup, args, world: int) -> dict:
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
+def run_block_op(args) -> None:
+    """copy_blocks: n random (src, dst) pairs of the workload's pool per step.
+    swap: n blocks out to pinned host records, then back in, per step; the host
+    link's reference is a plain cudaMemcpyAsync of the same bytes each way."""
+    import oracle
+    import paged_quantized_kv_cache_b200 as pq
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    s = bench_spec(args.workload, args.kv_dtype, None, args.pool_blocks)
+    nb = s.pool_blocks
+    g = pq.allocate_cache(s.kv_dtype, nb, s.num_kv_heads, s.head_dim, device=dev)
+    for a in g.arrays():
+        if a is not None:
+            a.copy_(torch.randint(0, 256, a.shape, dtype=torch.uint8, device=dev))
+    rec = pq.block_record_bytes(s.kv_dtype, s.num_kv_heads, s.head_dim)
+    rng = np.random.default_rng(100 + rank)
+    n = args.op_blocks
+    ids = rng.choice(nb, size=2 * n, replace=False).astype(np.int32)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    if args.op == "copy_blocks":
+        pairs_h = torch.from_numpy(ids.reshape(2, n).T.copy()).pin_memory()
+        pairs = pairs_h.to(dev)
+        step = lambda: pq.copy_blocks(g, pairs, err)  # noqa: E731
+        bytes_step = 2 * n * rec
+        metric = "copy_blocks GB/s (bytes read + written; copy-on-write block copies)"
+    else:
+        host = torch.empty(n * rec, dtype=torch.uint8).pin_memory()
+        blk = torch.from_numpy(ids[:n].copy()).to(dev)
+        blk_in = torch.from_numpy(ids[n:].copy()).to(dev)
+
+        def step():
+            pq.swap_out(g, blk, host, err)
+            pq.swap_in(g, blk_in, host, err)
+        bytes_step = 2 * n * rec
+        metric = "swap GB/s over the host link (blocks out to pinned host records and back in)"
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError("device error bits %d" % int(err.item()))
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+    value = bytes_step * world / (ms * 1e-3) / 1e9
+    peaks = measured_peaks()
+    if args.op == "copy_blocks":
+        roofline = {"bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": value / world / peaks["hbm_gbs"], "traffic": None, "kernel": "block_move_kernel<copy>",
+                    "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, a read+write copy)"}
+        # e2e: the pairs come from pinned host memory every step, the error flag goes back
+        h_err = torch.empty(1, dtype=torch.int32).pin_memory()
+
+        def e2e_step():
+            pairs.copy_(pairs_h, non_blocking=True)
+            step()
+            h_err.copy_(err, non_blocking=True)
+        h2d, d2h = pairs_h.numel() * 4, 4
+    else:
+        # reference for the host link: cudaMemcpyAsync of the same bytes each way
+        dbuf = torch.empty(n * rec, dtype=torch.uint8, device=dev)
+        for _ in range(3):
+            host.copy_(dbuf, non_blocking=True)
+            dbuf.copy_(host, non_blocking=True)
+        torch.cuda.synchronize(dev)
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        m0.record(stream)
+        for _ in range(K):
+            host.copy_(dbuf, non_blocking=True)
+            dbuf.copy_(host, non_blocking=True)
+        m1.record(stream)
+        torch.cuda.synchronize(dev)
+        memcpy_gbs = bytes_step / (m0.elapsed_time(m1) / K * 1e-3) / 1e9
+        roofline = {"bound": "host link", "achieved": value / world, "peak": memcpy_gbs, "unit": "GB/s",
+                    "frac": value / world / memcpy_gbs, "traffic": None, "kernel": "block_move_kernel<to/from host>",
+                    "peak_source": "cudaMemcpyAsync of the same bytes D2H + H2D (pinned), measured in this run"}
+        e2e_step, h2d, d2h = step, n * rec, n * rec
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(K):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / K
+    e2e = {"value": bytes_step * world / (ms_e2e * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_e2e,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            # the oracle's block copy (numpy slices) on a bounded host-memory sample
+            nsm = min(n, 256)
+            oc = oracle.Cache(s.kv_dtype, 2 * nsm, s.num_kv_heads, s.head_dim, poison=False)
+            pr = np.stack([np.arange(nsm), np.arange(nsm) + nsm], axis=1)
+            reps, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < min(args.cpu_budget, 5.0):
+                oracle.copy_blocks(oc, pr)
+                reps += 1
+            dt = time.perf_counter() - t0
+            cpu = {"value": 2 * nsm * rec * reps / dt / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                   "sample": "%d block copies of %d bytes, repeated for %.1f s" % (nsm, rec, dt)}
+        line = {
+            "metric": metric, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": "%s cache (%s, %d KV heads, head_dim %d, pool %d blocks): %d blocks of %d "
+                                   "bytes per step" % (args.workload, DT_LABEL[s.kv_dtype], s.num_kv_heads,
+                                                       s.head_dim, nb, n, rec),
+                       "op": args.op, "blocks_per_step": n, "record_bytes": rec,
+                       "l2": "%.0f MB moved per step vs 126 MB L2" % (bytes_step / 1e6)},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": (1 if args.op == "copy_blocks" else 2) * K, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -577,6 +720,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle timing")
     ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample")
+    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap"], default="decode")
+    ap.add_argument("--op-blocks", type=int, default=4096, help="blocks moved per step (--op copy_blocks|swap)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -584,6 +729,8 @@ def main():
         args.ref_seqs = {"tiny": 4, "llama8b": 64, "fp8": 32, "llama70b": 4, "fp4": 16}[args.workload]
     if args.impl == "reference":
         run_reference(args)
+    elif args.op != "decode":
+        run_block_op(args)
     else:
         run_ours(args)
 

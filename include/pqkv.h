@@ -12,9 +12,12 @@
  *        16-token blocks, page tables) and "Field Observations & Production
  *        Failure Modes" (block pool exhaustion).
  *   [P3] "vLLM" glossary (inferensys.com), entries "PagedAttention" (fixed-size
- *        blocks, logical-to-physical mapping, sharing across sequences),
- *        "Continuous batching" (blocks returned to the pool), "KV cache
- *        quantization" (FP8 just-in-time quantization).
+ *        blocks, logical-to-physical mapping, sharing across sequences for beam
+ *        search and parallel sampling), "Continuous batching" (blocks returned
+ *        to the pool), "KV cache quantization" (FP8 just-in-time quantization),
+ *        "Prefix caching" and "Automatic prefix caching" (requests with a
+ *        common prompt prefix reuse its KV blocks), "Preemption support"
+ *        (swapping KV cache blocks out to CPU RAM) and "CPU offloading".
  * Number formats follow the public OCP 8-bit Floating Point Specification
  * (OFP8: E4M3 "fn" with max 448 and no infinities, E5M2 with max 57344) and the
  * OCP Microscaling Formats specification (E2M1: values 0, .5, 1, 1.5, 2, 3, 4, 6).
@@ -223,6 +226,47 @@ int pqkv_paged_decode_attention_noalloc(const void* q, int q_dtype, int batch, i
                                         float scale, int split_blocks, void* out,
                                         int32_t* err_flag, pqkv_stream_t stream);
 
+/*
+ * Whole-block copy for copy-on-write ([P3] PagedAttention: blocks shared across
+ * sequences for beam search and parallel sampling; a sequence that forks off a
+ * shared partial block writes into its own copy). pairs: device int32
+ * [num_pairs][2] = (src, dst) block ids. Each pair copies everything the
+ * block holds for all KV heads: its K/V codes and, per format, its scales and
+ * outlier buffers (for the cache arrays of the formats above; unused arrays
+ * may be NULL). Destinations must be distinct and not among the sources of the
+ * same call. An id outside [0, num_blocks) skips the pair and sets
+ * PQKV_DEVERR_BLOCK_ID in *err_flag. One kernel on `stream`.
+ */
+int pqkv_copy_blocks(void* cache, void* scales, void* outliers_idx, void* outliers_val,
+                     int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                     const int32_t* pairs, int num_pairs, int32_t* err_flag,
+                     pqkv_stream_t stream);
+
+/*
+ * Block swap to host memory ([P3] "Preemption support": KV cache blocks are
+ * swapped out to CPU RAM under memory pressure and back in later; "CPU
+ * offloading"). A swapped block is one record of
+ * pqkv_block_record_bytes(kv_dtype, num_kv_heads, head_dim) bytes: the block's
+ * cache bytes (all heads, K and V), then its scales, outlier indices and
+ * outlier values as far as the format has them, each in the cache's own layout.
+ * host_records: page-locked host memory (cudaHostAlloc / cudaHostRegister) of
+ * num records (record i for block_ids[i]); the GPU reads or writes it
+ * directly, so no device staging buffer is needed. block_ids: device int32
+ * [num]. pqkv_swap_out copies blocks into records, pqkv_swap_in records into
+ * blocks (ids distinct). An id outside [0, num_blocks) skips its record and
+ * sets PQKV_DEVERR_BLOCK_ID. host_records not accessible from the device ->
+ * PQKV_ERR_ARG. One kernel on `stream`.
+ */
+size_t pqkv_block_record_bytes(int kv_dtype, int num_kv_heads, int head_dim);
+int pqkv_swap_out(const void* cache, const void* scales, const void* outliers_idx,
+                  const void* outliers_val, int kv_dtype, int num_blocks, int num_kv_heads,
+                  int head_dim, const int32_t* block_ids, int num, void* host_records,
+                  int32_t* err_flag, pqkv_stream_t stream);
+int pqkv_swap_in(void* cache, void* scales, void* outliers_idx, void* outliers_val,
+                 int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                 const int32_t* block_ids, int num, const void* host_records,
+                 int32_t* err_flag, pqkv_stream_t stream);
+
 /* Zero-fill a decode workspace on `stream` (optional; results never depend on
  * the workspace's prior contents). */
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
@@ -258,9 +302,50 @@ int pqkv_pool_share(pqkv_pool* pool, const int32_t* ids, int n);
  * the pool. Dropping more references than an id holds (counting repeats in
  * ids) gives PQKV_ERR_STATE and no change. */
 int pqkv_pool_free(pqkv_pool* pool, const int32_t* ids, int n);
+/* Blocks neither referenced nor cached. */
 int32_t pqkv_pool_num_free(const pqkv_pool* pool);
 /* Reference count of `id`, or -1 if out of range. */
 int32_t pqkv_pool_refcount(const pqkv_pool* pool, int32_t id);
+
+/*
+ * Prefix cache ([P3] "Prefix caching", "Automatic prefix caching"). Only full
+ * 16-token blocks are cached. A cached block is identified by its 16 token ids
+ * and by the cache entry of the block before it in the prompt, so a hit always
+ * means the same whole prefix (no hashing shortcut can return another
+ * prefix's block). A cached block that no sequence references stays cached and
+ * is "evictable": pqkv_pool_alloc / pqkv_pool_cow take free blocks first, then
+ * evict the least recently released evictable block (dropping its entry; the
+ * entries that continued its prefix can then never be found again and are
+ * evicted in their turn). Cached blocks must not be written: a sequence that
+ * appends into a block it shares, or into a cached block, calls pqkv_pool_cow
+ * first.
+ */
+int32_t pqkv_pool_num_evictable(const pqkv_pool* pool);
+/* Number of cache entries (referenced or evictable). */
+int32_t pqkv_pool_num_cached(const pqkv_pool* pool);
+/* Longest cached prefix of token_ids[0..num_tokens) (host), in whole blocks:
+ * writes the ids of the hit blocks to ids_out (host, room for num_tokens/16)
+ * and their count to *num_hit; each hit block gains one reference (an evictable
+ * one stops being evictable). A caller that must compute at least one token
+ * passes num_tokens = prompt length - 1. */
+int pqkv_pool_prefix_lookup(pqkv_pool* pool, const int32_t* token_ids, int num_tokens,
+                            int32_t* ids_out, int* num_hit);
+/* Register the full blocks of a prompt whose KV has been written: block b of
+ * token_ids[0..num_tokens) lives in ids[b] (host, b < min(num_tokens/16,
+ * num_ids); every id referenced). Blocks whose prefix is cached already (in
+ * that block, as returned by a lookup, or in another one) are skipped. From the
+ * first prefix not cached on, each block becomes a new entry; such a block
+ * already cached under another prefix, or repeated, gives PQKV_ERR_STATE and no
+ * change. References are not changed. */
+int pqkv_pool_prefix_insert(pqkv_pool* pool, const int32_t* token_ids, int num_tokens,
+                            const int32_t* ids, int num_ids);
+/* Copy-on-write before writing into block `id` (referenced by the caller).
+ * If the caller holds the only reference and the block is not cached, *new_id
+ * = id and *copy_needed = 0. Otherwise a block is allocated (as
+ * pqkv_pool_alloc), the caller's reference moves from `id` to it, *new_id is
+ * that block and *copy_needed = 1: the caller then copies `id` into it with
+ * pqkv_copy_blocks before writing. PQKV_ERR_OOM / ERR_STATE: no change. */
+int pqkv_pool_cow(pqkv_pool* pool, int32_t id, int32_t* new_id, int* copy_needed);
 
 /*
  * Host helper: slot mapping for appending tokens. For each sequence b, tokens

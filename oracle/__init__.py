@@ -178,3 +178,56 @@ def paged_decode(c: Cache, q: torch.Tensor, block_tables: np.ndarray, seq_lens: 
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments")
     return out, int(err[0])
+
+
+# ---- whole-block moves ------------------------------------------------------
+# "vLLM" glossary, "PagedAttention": blocks shared across sequences (beam search,
+# parallel sampling), so a sequence writing into a shared block takes its own
+# copy first; "Preemption support": KV cache blocks swapped out to CPU RAM and
+# back. A block is the same slice of each cache array (all arrays are
+# [num_blocks][...]); its record is those slices in array order: codes, scales,
+# outlier indices, outlier values.
+
+def _block_views(c: Cache):
+    return [a.reshape(c.nb, -1) for a in c.arrays() if a is not None]
+
+
+def block_record_bytes(dt: int, H: int, D: int) -> int:
+    return sum(cache_sizes(dt, 1, H, D))
+
+
+def copy_blocks(c: Cache, pairs) -> int:
+    """Copy block src into block dst for each (src, dst), in order. Returns error bits."""
+    err = 0
+    for s, d in np.asarray(pairs, dtype=np.int64).reshape(-1, 2):
+        if not (0 <= s < c.nb and 0 <= d < c.nb):
+            err |= ERR_BLOCK_ID
+            continue
+        for v in _block_views(c):
+            v[d] = v[s]
+    return err
+
+
+def swap_out(c: Cache, ids, records: np.ndarray) -> int:
+    """Record i = block ids[i]'s slices, concatenated. records: uint8 [n][record bytes]."""
+    err = 0
+    for i, b in enumerate(np.asarray(ids, dtype=np.int64).ravel()):
+        if not (0 <= b < c.nb):
+            err |= ERR_BLOCK_ID
+            continue
+        records[i] = np.concatenate([v[b] for v in _block_views(c)])
+    return err
+
+
+def swap_in(c: Cache, ids, records: np.ndarray) -> int:
+    """Inverse of swap_out: record i back into block ids[i]."""
+    err = 0
+    for i, b in enumerate(np.asarray(ids, dtype=np.int64).ravel()):
+        if not (0 <= b < c.nb):
+            err |= ERR_BLOCK_ID
+            continue
+        off = 0
+        for v in _block_views(c):
+            v[b] = records[i, off:off + v.shape[1]]
+            off += v.shape[1]
+    return err

@@ -35,7 +35,9 @@ EXPORTS = (
     "pqkv_decode_workspace_bytes", "pqkv_paged_decode_attention", "pqkv_decode_workspace_init",
     "pqkv_encode", "pqkv_pool_create", "pqkv_pool_destroy", "pqkv_pool_alloc", "pqkv_pool_share",
     "pqkv_pool_free", "pqkv_pool_num_free", "pqkv_pool_refcount", "pqkv_build_slot_mapping",
-    "pqkv_paged_decode_attention_noalloc",
+    "pqkv_paged_decode_attention_noalloc", "pqkv_pool_num_evictable", "pqkv_pool_num_cached",
+    "pqkv_pool_prefix_lookup", "pqkv_pool_prefix_insert", "pqkv_pool_cow", "pqkv_copy_blocks",
+    "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in",
 )
 
 
@@ -70,6 +72,15 @@ def _load() -> ctypes.CDLL:
         "pqkv_build_slot_mapping": (I, [P, I, I, P, P, P]),
         "pqkv_paged_decode_attention_noalloc": (I, [P, I, I, I, P, P, P, P, I, I, I, I, P, I, P, ctypes.c_float,
                                                     I, P, P, P]),
+        "pqkv_pool_num_evictable": (ctypes.c_int32, [P]),
+        "pqkv_pool_num_cached": (ctypes.c_int32, [P]),
+        "pqkv_pool_prefix_lookup": (I, [P, P, I, P, ctypes.POINTER(I)]),
+        "pqkv_pool_prefix_insert": (I, [P, P, I, P, I]),
+        "pqkv_pool_cow": (I, [P, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(I)]),
+        "pqkv_copy_blocks": (I, [P, P, P, P, I, I, I, I, P, I, P, P]),
+        "pqkv_block_record_bytes": (Z, [I, I, I]),
+        "pqkv_swap_out": (I, [P, P, P, P, I, I, I, I, P, I, P, P, P]),
+        "pqkv_swap_in": (I, [P, P, P, P, I, I, I, I, P, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -235,6 +246,63 @@ def encode(x: torch.Tensor, code_dtype: int, out: torch.Tensor, stream=None) -> 
                                            _stream_handle(stream, x.device)))
 
 
+def copy_blocks(cache: KVCache, pairs: torch.Tensor, err_flag: torch.Tensor, stream=None) -> None:
+    """pqkv_copy_blocks: pairs int32 [n][2] (src, dst) on the device."""
+    if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2:
+        raise ValueError("pairs must be int32 [n][2]")
+    _check("pqkv_copy_blocks", _lib.pqkv_copy_blocks(
+        _dev_ptr(cache.cache, "cache"), _dev_ptr(cache.scales, "scales"),
+        _dev_ptr(cache.outliers_idx, "outliers_idx"), _dev_ptr(cache.outliers_val, "outliers_val"),
+        cache.kv_dtype, cache.num_blocks, cache.num_kv_heads, cache.head_dim,
+        _dev_ptr(pairs, "pairs"), pairs.shape[0], _dev_ptr(err_flag, "err_flag"),
+        _stream_handle(stream, cache.cache.device)))
+
+
+def block_record_bytes(kv_dtype: int, num_kv_heads: int, head_dim: int) -> int:
+    n = int(_lib.pqkv_block_record_bytes(kv_dtype, num_kv_heads, head_dim))
+    if n == 0:
+        raise PqkvError("pqkv_block_record_bytes", ERR_ARG)
+    return n
+
+
+def _host_records(records: torch.Tensor, n: int, rec: int) -> int:
+    if not isinstance(records, torch.Tensor) or records.is_cuda or not records.is_pinned():
+        raise ValueError("records must be a pinned host tensor")
+    if not records.is_contiguous() or records.numel() * records.element_size() < n * rec:
+        raise ValueError("records must be contiguous with room for %d records of %d bytes" % (n, rec))
+    return records.data_ptr()
+
+
+def swap_out(cache: KVCache, block_ids: torch.Tensor, records: torch.Tensor, err_flag: torch.Tensor,
+             stream=None) -> None:
+    """pqkv_swap_out: block_ids int32 [n] (device) -> records (pinned host, n records)."""
+    if block_ids.dtype != torch.int32 or block_ids.dim() != 1:
+        raise ValueError("block_ids must be int32 [n]")
+    n = block_ids.numel()
+    rec = block_record_bytes(cache.kv_dtype, cache.num_kv_heads, cache.head_dim)
+    _check("pqkv_swap_out", _lib.pqkv_swap_out(
+        _dev_ptr(cache.cache, "cache"), _dev_ptr(cache.scales, "scales"),
+        _dev_ptr(cache.outliers_idx, "outliers_idx"), _dev_ptr(cache.outliers_val, "outliers_val"),
+        cache.kv_dtype, cache.num_blocks, cache.num_kv_heads, cache.head_dim,
+        _dev_ptr(block_ids, "block_ids"), n, _host_records(records, n, rec), _dev_ptr(err_flag, "err_flag"),
+        _stream_handle(stream, cache.cache.device)))
+
+
+def swap_in(cache: KVCache, block_ids: torch.Tensor, records: torch.Tensor, err_flag: torch.Tensor,
+            stream=None) -> None:
+    """pqkv_swap_in: records (pinned host, n records) -> blocks block_ids int32 [n] (device)."""
+    if block_ids.dtype != torch.int32 or block_ids.dim() != 1:
+        raise ValueError("block_ids must be int32 [n]")
+    n = block_ids.numel()
+    rec = block_record_bytes(cache.kv_dtype, cache.num_kv_heads, cache.head_dim)
+    _check("pqkv_swap_in", _lib.pqkv_swap_in(
+        _dev_ptr(cache.cache, "cache"), _dev_ptr(cache.scales, "scales"),
+        _dev_ptr(cache.outliers_idx, "outliers_idx"), _dev_ptr(cache.outliers_val, "outliers_val"),
+        cache.kv_dtype, cache.num_blocks, cache.num_kv_heads, cache.head_dim,
+        _dev_ptr(block_ids, "block_ids"), n, _host_records(records, n, rec), _dev_ptr(err_flag, "err_flag"),
+        _stream_handle(stream, cache.cache.device)))
+
+
 class BlockPool:
     """Host block-pool allocator (pqkv_pool_*): physical ids with reference counts."""
 
@@ -278,6 +346,36 @@ class BlockPool:
 
     def refcount(self, block_id: int) -> int:
         return int(_lib.pqkv_pool_refcount(self._h, block_id))
+
+    @property
+    def num_evictable(self) -> int:
+        return int(_lib.pqkv_pool_num_evictable(self._h))
+
+    @property
+    def num_cached(self) -> int:
+        return int(_lib.pqkv_pool_num_cached(self._h))
+
+    def prefix_lookup(self, token_ids) -> np.ndarray:
+        """Ids of the longest cached prefix of token_ids (whole blocks); each gains a reference."""
+        t = self._ids(token_ids)
+        out = np.empty(max(1, t.size // 16), dtype=np.int32)
+        hit = ctypes.c_int(0)
+        _check("pqkv_pool_prefix_lookup", _lib.pqkv_pool_prefix_lookup(
+            self._h, t.ctypes.data, t.size, out.ctypes.data, ctypes.byref(hit)))
+        return out[:hit.value].copy()
+
+    def prefix_insert(self, token_ids, ids) -> None:
+        t = self._ids(token_ids)
+        a = self._ids(ids)
+        _check("pqkv_pool_prefix_insert", _lib.pqkv_pool_prefix_insert(
+            self._h, t.ctypes.data, t.size, a.ctypes.data, a.size))
+
+    def cow(self, block_id: int) -> Tuple[int, bool]:
+        """(block to write into, whether block_id must be copied into it first)."""
+        new = ctypes.c_int32(-1)
+        need = ctypes.c_int(0)
+        _check("pqkv_pool_cow", _lib.pqkv_pool_cow(self._h, block_id, ctypes.byref(new), ctypes.byref(need)))
+        return int(new.value), bool(need.value)
 
 
 def build_slot_mapping(block_tables: np.ndarray, start_pos: Sequence[int], num_new: Sequence[int]) -> np.ndarray:

@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "blocks.cuh"
 #include "decode.cuh"
 #include "write.cuh"
 
@@ -264,6 +265,61 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   mp.slot_floats = p.slot_floats;
   e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+size_t pqkv_block_record_bytes(int kv_dtype, int num_kv_heads, int head_dim) {
+  if (!is_kv_dtype(kv_dtype) || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128)) return 0;
+  size_t b[4];
+  if (pqkv_cache_layout(kv_dtype, 1, num_kv_heads, head_dim, b) != PQKV_OK) return 0;
+  return b[0] + b[1] + b[2] + b[3];
+}
+
+static int block_move(int mode, void* cache, void* scales, void* outliers_idx, void* outliers_val, int kv_dtype,
+                      int num_blocks, int num_kv_heads, int head_dim, const int32_t* ids, int num, void* host,
+                      int32_t* err_flag, pqkv_stream_t stream) {
+  if (!is_kv_dtype(kv_dtype) || num_blocks < 1 || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128) ||
+      num < 0)
+    return PQKV_ERR_ARG;
+  if (num == 0) return PQKV_OK;
+  if (!ids || !err_flag || !cache) return PQKV_ERR_ARG;
+  BlockArrays a;
+  if (!block_arrays(kv_dtype, num_kv_heads, head_dim, cache, scales, outliers_idx, outliers_val, a))
+    return PQKV_ERR_ARG;
+  void* dev_host = nullptr;
+  if (mode != kMoveCopy) {
+    if (!host || !aligned16(host)) return PQKV_ERR_ARG;
+    if (cudaHostGetDevicePointer(&dev_host, host, 0) != cudaSuccess || !aligned16(dev_host)) {
+      (void)cudaGetLastError();  // clear the error this query left behind
+      return PQKV_ERR_ARG;
+    }
+  }
+  DeviceInfo di;
+  if (!device_info(di)) return PQKV_ERR_CUDA;
+  const cudaError_t e = launch_block_move(mode, a, ids, num, num_blocks, dev_host, err_flag, di.sms,
+                                          reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+int pqkv_copy_blocks(void* cache, void* scales, void* outliers_idx, void* outliers_val, int kv_dtype,
+                     int num_blocks, int num_kv_heads, int head_dim, const int32_t* pairs, int num_pairs,
+                     int32_t* err_flag, pqkv_stream_t stream) {
+  return block_move(kMoveCopy, cache, scales, outliers_idx, outliers_val, kv_dtype, num_blocks, num_kv_heads,
+                    head_dim, pairs, num_pairs, nullptr, err_flag, stream);
+}
+
+int pqkv_swap_out(const void* cache, const void* scales, const void* outliers_idx, const void* outliers_val,
+                  int kv_dtype, int num_blocks, int num_kv_heads, int head_dim, const int32_t* block_ids, int num,
+                  void* host_records, int32_t* err_flag, pqkv_stream_t stream) {
+  return block_move(kMoveToHost, const_cast<void*>(cache), const_cast<void*>(scales),
+                    const_cast<void*>(outliers_idx), const_cast<void*>(outliers_val), kv_dtype, num_blocks,
+                    num_kv_heads, head_dim, block_ids, num, host_records, err_flag, stream);
+}
+
+int pqkv_swap_in(void* cache, void* scales, void* outliers_idx, void* outliers_val, int kv_dtype, int num_blocks,
+                 int num_kv_heads, int head_dim, const int32_t* block_ids, int num, const void* host_records,
+                 int32_t* err_flag, pqkv_stream_t stream) {
+  return block_move(kMoveFromHost, cache, scales, outliers_idx, outliers_val, kv_dtype, num_blocks, num_kv_heads,
+                    head_dim, block_ids, num, const_cast<void*>(host_records), err_flag, stream);
 }
 
 int pqkv_encode(const float* x, int64_t n, int code_dtype, uint8_t* codes, pqkv_stream_t stream) {
