@@ -20,6 +20,11 @@ on a bounded sample of the same workload on the host cores.
 --op copy_blocks | swap measures the whole-block moves instead (copy-on-write
 copies inside the cache; swap of blocks to pinned host memory and back) on the
 workload's cache format; one JSON line of the same shape.
+
+--op prefill measures chunked-prefill attention: 16 sequences (Llama-3-8B
+shaped, 32 q / 8 KV heads, head_dim 128), each with a prefix of U[0, 7680]
+cached tokens and a 512-token chunk; a step writes the chunk's K/V into the
+cache and runs the causal attention of its queries over the whole context.
 """
 from __future__ import annotations
 
@@ -268,8 +273,8 @@ def measured_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 def decode_source_hash() -> str:
@@ -705,6 +710,177 @@ def run_block_op(args) -> None:
         dist.destroy_process_group()
 
 
+PREFILL_DESCR = ("chunked prefill, Llama-3-8B-shaped layer: 16 seqs, prefix U[0,7680] cached tokens + a 512-token "
+                 "chunk each (written, then causal attention over prefix + chunk), 32 q / 8 kv heads, head_dim 128, "
+                 "block 16")
+
+
+def run_prefill(args) -> None:
+    import oracle
+    import paged_quantized_kv_cache_b200 as pq
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    kv = KV_NAMES[args.kv_dtype or "bf16"]
+    B, Hq, Hkv, D, C = args.batch or 16, 32, 8, 128, 512
+    rng = np.random.default_rng(7 + rank)
+    prefix = rng.integers(0, 7681, size=B)
+    lens = (prefix + C).astype(np.int32)
+    nblk = (lens + 15) // 16
+    maxblk = int(nblk.max())
+    nb = int(nblk.sum()) + 64
+    perm = rng.permutation(nb).astype(np.int32)
+    tables = np.full((B, maxblk), -1, dtype=np.int32)
+    o = 0
+    for b in range(B):
+        tables[b, :nblk[b]] = perm[o:o + nblk[b]]
+        o += nblk[b]
+    in_dt = torch.float16 if kv == W.DT_FP16 else torch.bfloat16
+    g = pq.allocate_cache(kv, nb, Hkv, D, device=dev, fill=0)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11 + rank)
+    # prefixes: written once, untimed
+    for b in range(B):
+        if prefix[b]:
+            k = torch.randn((int(prefix[b]), Hkv, D), generator=gen, device=dev).to(in_dt)
+            v = torch.randn((int(prefix[b]), Hkv, D), generator=gen, device=dev).to(in_dt)
+            sl = pq.build_slot_mapping(tables[b:b + 1], [0], [int(prefix[b])])
+            pq.kv_cache_write(k, v, torch.from_numpy(sl).to(dev), g, err)
+    # the step's inputs: chunk K/V, slots, queries, metadata (packed pinned host copy for e2e)
+    ck = torch.randn((B * C, Hkv, D), generator=gen, device=dev).to(in_dt)
+    cv = torch.randn((B * C, Hkv, D), generator=gen, device=dev).to(in_dt)
+    q = torch.randn((B * C, Hq, D), generator=gen, device=dev).to(in_dt)
+    slots = torch.from_numpy(pq.build_slot_mapping(tables, prefix, [C] * B)).to(dev)
+    cu = torch.from_numpy(np.arange(0, (B + 1) * C, C, dtype=np.int32)).to(dev)
+    bt = torch.from_numpy(tables).to(dev)
+    sl = torch.from_numpy(lens).to(dev)
+    out = torch.empty_like(q)
+    scale = 1.0 / math.sqrt(D)
+    stream = torch.cuda.current_stream(dev)
+
+    def write():
+        pq.kv_cache_write(ck, cv, slots, g, err)
+
+    def attend():
+        pq.paged_prefill_attention(q, cu, C, g, bt, sl, scale, out, err)
+
+    for _ in range(max(args.warmup, 3)):
+        write()
+        attend()
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    e0.record(stream)
+    for i in range(K):
+        ev[i][0].record(stream)
+        write()
+        ev[i][1].record(stream)
+        attend()
+        ev[i][2].record(stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks.stop()
+    barrier(world)
+    if int(err.item()) != 0:
+        raise RuntimeError("device error bits %d" % int(err.item()))
+    ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+    att_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
+    wr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+    # causal attention flops: 4 * Hq * D per (query token, visible position)
+    flops = 4.0 * Hq * D * float(sum(C * int(prefix[b]) + C * (C + 1) // 2 for b in range(B)))
+    value = flops * world / (ms * 1e-3) / 1e12
+    peaks = measured_peaks()
+    peak = peaks["bf16_tflops"]
+    achieved = flops / (att_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": None, "kernel": "paged_prefill_kernel",
+                "peak_source": peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, cuBLAS bf16 burst; the f16 "
+                "operands of quantized caches run at the same dense rate)",
+                "flops_per_launch": flops, "avg_launch_ms": att_ms}
+    # e2e: the step's inputs from pinned host memory, the output back, every step
+    h_q, h_k, h_v = q.cpu().pin_memory(), ck.cpu().pin_memory(), cv.cpu().pin_memory()
+    h_slots = slots.cpu().pin_memory()
+    h_meta = torch.cat([cu.cpu(), sl.cpu(), bt.cpu().ravel()]).pin_memory()
+    d_meta = torch.empty_like(h_meta, device=dev)
+    h_out = torch.empty_like(out, device="cpu").pin_memory()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        ck.copy_(h_k, non_blocking=True)
+        cv.copy_(h_v, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        d_meta.copy_(h_meta, non_blocking=True)
+        write()
+        attend()
+        h_out.copy_(out, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    Ke = max(1, min(K, 50))
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / Ke
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_meta))
+    e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * h_out.element_size()}
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            # the oracle's prefill of one sequence: a 64-token chunk after 1024 cached tokens
+            r2 = np.random.default_rng(3)
+            L, qn = 1088, 64
+            oc = oracle.Cache(kv, (L + 15) // 16, Hkv, D, poison=False)
+            tab = np.arange((L + 15) // 16, dtype=np.int32)[None]
+            kk = torch.from_numpy(r2.standard_normal((L, Hkv, D)).astype(np.float32)).to(in_dt)
+            vv = torch.from_numpy(r2.standard_normal((L, Hkv, D)).astype(np.float32)).to(in_dt)
+            oracle.kv_cache_write(oc, kk, vv, np.arange(L, dtype=np.int32))
+            qq = torch.from_numpy(r2.standard_normal((qn, Hq, D)).astype(np.float32)).to(in_dt)
+            cuq = np.array([0, qn], np.int32)
+            f1 = 4.0 * Hq * D * (qn * (L - qn) + qn * (qn + 1) // 2)
+            reps, t0 = 0, time.perf_counter()
+            while time.perf_counter() - t0 < min(args.cpu_budget, 10.0):
+                oracle.paged_prefill(oc, qq, cuq, tab, np.array([L], np.int32), scale)
+                reps += 1
+            dt = time.perf_counter() - t0
+            cpu = {"value": f1 * reps / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                   "sample": "%d runs of one sequence: a %d-token chunk after %d cached tokens, %s cache, %.1f s"
+                             % (reps, qn, L - qn, DT_LABEL[kv], dt)}
+        line = {
+            "metric": "chunked-prefill attention TFLOP/s (causal, paged cache)", "value": value, "unit": "TFLOP/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if kv == W.DT_BF16 else ("fp16" if kv == W.DT_FP16 else DT_LABEL[kv] + "->f16"),
+            "data": "synthetic",
+            "config": {"workload": PREFILL_DESCR + "; KV " + DT_LABEL[kv], "batch": B, "chunk": C,
+                       "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "context_tokens": int(lens.sum()),
+                       "l2": "KV read per step %.0f MB (prefix + chunk, once per query tile) vs 126 MB L2; no flush"
+                             % (float(lens.sum()) * Hkv * 2 * D * (2 if kv <= 1 else 1) / 1e6)},
+            "attention_kernel_ms": att_ms, "write_kernel_ms": wr_ms,
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": 2 * K, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -720,7 +896,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=10.0, help="seconds of oracle timing")
     ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample")
-    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap"], default="decode")
+    ap.add_argument("--op", choices=["decode", "copy_blocks", "swap", "prefill"], default="decode")
     ap.add_argument("--op-blocks", type=int, default=4096, help="blocks moved per step (--op copy_blocks|swap)")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -729,6 +905,8 @@ def main():
         args.ref_seqs = {"tiny": 4, "llama8b": 64, "fp8": 32, "llama70b": 4, "fp4": 16}[args.workload]
     if args.impl == "reference":
         run_reference(args)
+    elif args.op == "prefill":
+        run_prefill(args)
     elif args.op != "decode":
         run_block_op(args)
     else:

@@ -17,7 +17,8 @@
  *        to the pool), "KV cache quantization" (FP8 just-in-time quantization),
  *        "Prefix caching" and "Automatic prefix caching" (requests with a
  *        common prompt prefix reuse its KV blocks), "Preemption support"
- *        (swapping KV cache blocks out to CPU RAM) and "CPU offloading".
+ *        (swapping KV cache blocks out to CPU RAM), "CPU offloading" and
+ *        "Chunked prefill" (long prompts processed in chunks).
  * Number formats follow the public OCP 8-bit Floating Point Specification
  * (OFP8: E4M3 "fn" with max 448 and no infinities, E5M2 with max 57344) and the
  * OCP Microscaling Formats specification (E2M1: values 0, .5, 1, 1.5, 2, 3, 4, 6).
@@ -225,6 +226,35 @@ int pqkv_paged_decode_attention_noalloc(const void* q, int q_dtype, int batch, i
                                         int max_blocks_per_seq, const int32_t* seq_lens,
                                         float scale, int split_blocks, void* out,
                                         int32_t* err_flag, pqkv_stream_t stream);
+
+/*
+ * Chunked-prefill attention over the paged cache ([P3] "Chunked prefill": a
+ * long prompt is processed in chunks; [P1] architecture diagram: 512-token
+ * chunks, and step 4: the attention kernel reads the compressed codes and the
+ * fp16 outlier channels together; [P3] "PagedAttention": K/V through the
+ * block table). Sequence b's query tokens are rows cu_q_lens[b] ..
+ * cu_q_lens[b+1]-1 of q ([cu_q_lens[batch]][num_q_heads][head_dim], device,
+ * q_dtype FP16 or BF16; 16-bit caches need q_dtype == kv_dtype); they are its
+ * last qn_b = cu_q_lens[b+1] - cu_q_lens[b] positions, i.e. the chunk's K/V are
+ * written into the cache first (pqkv_kv_cache_write) and seq_lens[b] counts
+ * them. Query token i sits at position p = seq_lens[b] - qn_b + i and attends
+ * to positions 0..p (causal): out_row = softmax(scale * q K[0..p]^T) V[0..p],
+ * written to the same row of out (same shape and dtype as q). Query head hq
+ * reads KV head hq / (num_q_heads / num_kv_heads); that ratio must divide 128.
+ * cu_q_lens: device int32 [batch + 1], non-decreasing. max_q_len (host) bounds
+ * every qn_b: rows past it are not computed and PQKV_DEVERR_SEQ_LEN is set. A
+ * sequence with qn_b > seq_lens[b] or seq_lens[b] > 16 * max_blocks_per_seq
+ * gets zero rows and PQKV_DEVERR_SEQ_LEN; tokens of a block id outside
+ * [0, num_blocks) are skipped (PQKV_DEVERR_BLOCK_ID). One kernel on `stream`,
+ * on the tensor cores (tcgen05); no workspace.
+ */
+int pqkv_paged_prefill_attention(const void* q, int q_dtype, int batch, int max_q_len,
+                                 int num_q_heads, const int32_t* cu_q_lens, const void* cache,
+                                 const void* scales, const void* outliers_idx,
+                                 const void* outliers_val, int kv_dtype, int num_blocks,
+                                 int num_kv_heads, int head_dim, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* seq_lens, float scale,
+                                 void* out, int32_t* err_flag, pqkv_stream_t stream);
 
 /*
  * Whole-block copy for copy-on-write ([P3] PagedAttention: blocks shared across

@@ -52,6 +52,9 @@ def lib() -> ctypes.CDLL:
         _lib.oracle_paged_decode.argtypes = [P, I, ctypes.c_int, I, P, P, P, P, I, I, I, I, P, I, P,
                                              ctypes.c_float, P, P]
         _lib.oracle_paged_decode.restype = I
+        _lib.oracle_paged_prefill.argtypes = [P, I, P, I, I, P, P, P, P, I, I, I, I, P, I, P,
+                                              ctypes.c_float, P, P]
+        _lib.oracle_paged_prefill.restype = I
         _lib.oracle_num_threads.restype = I
     return _lib
 
@@ -177,6 +180,29 @@ def paged_decode(c: Cache, q: torch.Tensor, block_tables: np.ndarray, seq_lens: 
                                    _ptr(err))
     if rc != 0:
         raise ValueError("oracle decode rejected its arguments")
+    return out, int(err[0])
+
+
+def paged_prefill(c: Cache, q: torch.Tensor, cu_q: np.ndarray, block_tables: np.ndarray,
+                  seq_lens: np.ndarray, scale: float) -> Tuple[np.ndarray, int]:
+    """Causal chunked-prefill attention: q [cu_q[-1]][Hq][D]; sequence b's query
+    tokens are its last cu_q[b+1] - cu_q[b] positions. fp64 output, error bits."""
+    T, Hq, D = q.shape
+    assert D == c.D
+    q_dt = DT_BF16 if q.dtype == torch.bfloat16 else DT_FP16
+    cu = np.ascontiguousarray(cu_q, dtype=np.int32)
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    B = sl.size
+    assert cu.size == B + 1 and cu[-1] == T
+    out = np.zeros((T, Hq, D), dtype=np.float64)
+    err = np.zeros(1, dtype=np.int32)
+    qu = _u16(q)
+    rc = lib().oracle_paged_prefill(_ptr(qu), q_dt, _ptr(cu), B, Hq, _ptr(c.cache), _ptr(c.scales),
+                                    _ptr(c.oidx), _ptr(c.oval), c.dt, c.nb, c.H, c.D, _ptr(bt),
+                                    bt.shape[1], _ptr(sl), ctypes.c_float(scale), _ptr(out), _ptr(err))
+    if rc != 0:
+        raise ValueError("oracle prefill rejected its arguments")
     return out, int(err[0])
 
 

@@ -13,7 +13,8 @@
  *  [P2] "vLLM v0.7.2" field report -- "Deconstructing the v0.7.2 Architecture"
  *       (FP8 E4M3/E5M2 KV cache, 16-token blocks, page tables).
  *  [P3] "vLLM" glossary -- "PagedAttention" (logical-to-physical block mapping,
- *       blocks shared across sequences), "KV cache quantization".
+ *       blocks shared across sequences), "KV cache quantization", "Chunked
+ *       prefill" (long prompts processed in chunks).
  *  [OFP8] OCP 8-bit Floating Point Specification: E4M3 (bias 7, max 448, no
  *       infinities, S.1111.111 = NaN) and E5M2 (bias 15, max 57344, IEEE-like).
  *  [MX] OCP Microscaling Formats specification: E2M1 (bias 1, values
@@ -533,6 +534,59 @@ int oracle_paged_decode(const uint16_t* q, int q_dt, int B, int Hq, const uint8_
       const size_t qoff = ((size_t)b * Hq + (size_t)h * G + g) * D;
       for (int ch = 0; ch < D; ++ch) qd[ch] = (double)in_value(q, q_dt, qoff + ch);
       attend(qd, kd, vd, valid, L, D, (double)scale, ob + (size_t)g * D, sb);
+    }
+    free(kd);
+    free(vd);
+    free(sb);
+    free(valid);
+  }
+  *err |= flags;
+  return 0;
+}
+
+/* Chunked-prefill attention ([P1] architecture diagram: prompts processed in
+ * 512-token chunks; [P3] "Chunked prefill"). The qn = cu_q[b+1] - cu_q[b] query
+ * tokens of sequence b are its last qn positions: query token i sits at
+ * position p = seq_lens[b] - qn + i and attends to positions 0..p (causal), read
+ * through the block table like decode. q and out: [cu_q[B]][Hq][D]. A sequence
+ * with qn > seq_lens[b] or seq_lens[b] beyond its table is skipped (SEQ_LEN,
+ * zero output rows). */
+int oracle_paged_prefill(const uint16_t* q, int q_dt, const int32_t* cu_q, int B, int Hq,
+                         const uint8_t* cache, const uint8_t* scales, const uint8_t* oidx,
+                         const uint8_t* oval, int kv_dt, int nb, int H, int D, const int32_t* tables,
+                         int maxblk, const int32_t* seq_lens, float scale, double* out, int32_t* err) {
+  if (Hq % H != 0) return 1;
+  const int G = Hq / H;
+  int32_t flags = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : flags)
+  for (int bh = 0; bh < B * H; ++bh) {
+    const int b = bh / H, h = bh % H;
+    const int L = seq_lens[b];
+    const int qn = cu_q[b + 1] - cu_q[b];
+    if (qn <= 0) continue;
+    if (L < 0 || (int64_t)L > (int64_t)BS * maxblk || qn > L) {
+      flags |= ERR_SEQ_LEN;
+      for (int i = 0; i < qn; ++i)
+        for (size_t e = 0; e < (size_t)G * D; ++e)
+          out[((size_t)(cu_q[b] + i) * Hq + (size_t)h * G) * D + e] = 0.0;
+      continue;
+    }
+    double* kd = (double*)malloc(sizeof(double) * (size_t)L * D);
+    double* vd = (double*)malloc(sizeof(double) * (size_t)L * D);
+    double* sb = (double*)malloc(sizeof(double) * (size_t)L);
+    uint8_t* valid = (uint8_t*)malloc((size_t)L);
+    double qd[128];
+    oracle_gather(cache, scales, oidx, oval, kv_dt, nb, H, D, tables + (size_t)b * maxblk, L, h, kd, vd,
+                  valid);
+    for (int t = 0; t < L; ++t)
+      if (!valid[t]) flags |= ERR_BLOCK_ID;
+    for (int i = 0; i < qn; ++i) {
+      const int pos = L - qn + i;
+      for (int g = 0; g < G; ++g) {
+        const size_t row = ((size_t)(cu_q[b] + i) * Hq + (size_t)h * G + g) * D;
+        for (int ch = 0; ch < D; ++ch) qd[ch] = (double)in_value(q, q_dt, row + ch);
+        attend(qd, kd, vd, valid, pos + 1, D, (double)scale, out + row, sb);
+      }
     }
     free(kd);
     free(vd);

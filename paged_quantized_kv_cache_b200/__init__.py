@@ -37,7 +37,7 @@ EXPORTS = (
     "pqkv_pool_free", "pqkv_pool_num_free", "pqkv_pool_refcount", "pqkv_build_slot_mapping",
     "pqkv_paged_decode_attention_noalloc", "pqkv_pool_num_evictable", "pqkv_pool_num_cached",
     "pqkv_pool_prefix_lookup", "pqkv_pool_prefix_insert", "pqkv_pool_cow", "pqkv_copy_blocks",
-    "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in",
+    "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in", "pqkv_paged_prefill_attention",
 )
 
 
@@ -81,6 +81,8 @@ def _load() -> ctypes.CDLL:
         "pqkv_block_record_bytes": (Z, [I, I, I]),
         "pqkv_swap_out": (I, [P, P, P, P, I, I, I, I, P, I, P, P, P]),
         "pqkv_swap_in": (I, [P, P, P, P, I, I, I, I, P, I, P, P, P]),
+        "pqkv_paged_prefill_attention": (I, [P, I, I, I, I, P, P, P, P, P, I, I, I, I, P, I, P, ctypes.c_float,
+                                             P, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -236,6 +238,32 @@ def paged_decode_attention(q: torch.Tensor, cache: KVCache, block_tables: torch.
         _dev_ptr(out, "out"), _dev_ptr(workspace, "workspace"), workspace.numel(),
         _dev_ptr(err_flag, "err_flag"), _stream_handle(stream, q.device))
     _check("pqkv_paged_decode_attention", st)
+
+
+def paged_prefill_attention(q: torch.Tensor, cu_q_lens: torch.Tensor, max_q_len: int, cache: KVCache,
+                            block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float, out: torch.Tensor,
+                            err_flag: torch.Tensor, stream=None) -> None:
+    """pqkv_paged_prefill_attention: q, out [T][Hq][D]; cu_q_lens int32 [B + 1]; block_tables int32
+    [B][max_blocks]; seq_lens int32 [B] (each sequence's query tokens are its last positions)."""
+    T, Hq, D = q.shape
+    B = seq_lens.numel()
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    if cu_q_lens.dtype != torch.int32 or cu_q_lens.numel() != B + 1:
+        raise ValueError("cu_q_lens must be int32 [B + 1]")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B][max_blocks_per_seq]")
+    if seq_lens.dtype != torch.int32:
+        raise ValueError("seq_lens must be int32 [B]")
+    st = _lib.pqkv_paged_prefill_attention(
+        _dev_ptr(q, "q"), _dt_of(q, "q"), B, max_q_len, Hq, _dev_ptr(cu_q_lens, "cu_q_lens"),
+        _dev_ptr(cache.cache, "cache"), _dev_ptr(cache.scales, "scales"),
+        _dev_ptr(cache.outliers_idx, "outliers_idx"), _dev_ptr(cache.outliers_val, "outliers_val"),
+        cache.kv_dtype, cache.num_blocks, cache.num_kv_heads, cache.head_dim,
+        _dev_ptr(block_tables, "block_tables"), block_tables.shape[1], _dev_ptr(seq_lens, "seq_lens"),
+        ctypes.c_float(scale), _dev_ptr(out, "out"), _dev_ptr(err_flag, "err_flag"),
+        _stream_handle(stream, q.device))
+    _check("pqkv_paged_prefill_attention", st)
 
 
 def encode(x: torch.Tensor, code_dtype: int, out: torch.Tensor, stream=None) -> None:

@@ -7,6 +7,7 @@
 
 #include "blocks.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 #include "write.cuh"
 
 namespace pqkv {
@@ -81,6 +82,22 @@ bool make_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb, i
                                                 : CU_TENSOR_MAP_SWIZZLE_32B;
   const CUresult r = fn(map, dt, 2, const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// TMA descriptor for the prefill's 16-bit operand tiles: the same rows, one box
+// = 16 rows (the K or the V of one (block, head) pair) x 64 elements, 128-byte
+// swizzle (the tensor cores' operand layout).
+bool make_prefill_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb, int H, int D) {
+  auto fn = encode_fn();
+  if (!fn || !is_16(kv_dtype)) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)nb * H * 2 * 16};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(cache), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -320,6 +337,62 @@ int pqkv_swap_in(void* cache, void* scales, void* outliers_idx, void* outliers_v
                  int32_t* err_flag, pqkv_stream_t stream) {
   return block_move(kMoveFromHost, cache, scales, outliers_idx, outliers_val, kv_dtype, num_blocks, num_kv_heads,
                     head_dim, block_ids, num, const_cast<void*>(host_records), err_flag, stream);
+}
+
+int pqkv_paged_prefill_attention(const void* q, int q_dtype, int batch, int max_q_len, int num_q_heads,
+                                 const int32_t* cu_q_lens, const void* cache, const void* scales,
+                                 const void* outliers_idx, const void* outliers_val, int kv_dtype, int num_blocks,
+                                 int num_kv_heads, int head_dim, const int32_t* block_tables,
+                                 int max_blocks_per_seq, const int32_t* seq_lens, float scale, void* out,
+                                 int32_t* err_flag, pqkv_stream_t stream) {
+  if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
+  if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
+  if (batch < 0 || max_q_len < 1 || num_q_heads < 1 || num_kv_heads < 1 || num_blocks < 1 ||
+      max_blocks_per_seq < 1 || (head_dim != 64 && head_dim != 128))
+    return PQKV_ERR_ARG;
+  if (num_q_heads % num_kv_heads != 0) return PQKV_ERR_ARG;
+  const int G = num_q_heads / num_kv_heads;
+  if (128 % G != 0) return PQKV_ERR_ARG;
+  if (num_kv_heads > 65535 || !(scale == scale)) return PQKV_ERR_ARG;
+  if (batch == 0) return PQKV_OK;
+  const int64_t tiles = ((int64_t)max_q_len * G + 127) / 128;
+  if (tiles * batch > INT32_MAX) return PQKV_ERR_ARG;
+  if (!q || !cu_q_lens || !cache || !block_tables || !seq_lens || !out || !err_flag) return PQKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(out) || !aligned16(cache)) return PQKV_ERR_ARG;
+  if (!is_16(kv_dtype) && (!scales || !aligned16(scales))) return PQKV_ERR_ARG;
+  if (kv_dtype == PQKV_DTYPE_FP4_E2M1 &&
+      (!outliers_idx || !outliers_val || !aligned16(outliers_idx) || !aligned16(outliers_val)))
+    return PQKV_ERR_ARG;
+  DeviceInfo di;
+  if (!device_info(di)) return PQKV_ERR_CUDA;
+  if ((size_t)di.max_smem < prefill_smem_bytes(kv_dtype, head_dim)) return PQKV_ERR_CUDA;
+  CUtensorMap tmap;
+  std::memset(&tmap, 0, sizeof(tmap));
+  if (is_16(kv_dtype) && !make_prefill_map(&tmap, cache, kv_dtype, num_blocks, num_kv_heads, head_dim))
+    return PQKV_ERR_CUDA;
+  PrefillParams p;
+  p.q = q;
+  p.out = out;
+  p.cache = static_cast<const uint8_t*>(cache);
+  p.scales = static_cast<const uint8_t*>(scales);
+  p.oidx = static_cast<const uint8_t*>(outliers_idx);
+  p.oval = static_cast<const uint8_t*>(outliers_val);
+  p.cu_q = cu_q_lens;
+  p.seq_lens = seq_lens;
+  p.block_tables = block_tables;
+  p.err = err_flag;
+  p.B = batch;
+  p.Hq = num_q_heads;
+  p.Hkv = num_kv_heads;
+  p.G = G;
+  p.nb = num_blocks;
+  p.maxblk = max_blocks_per_seq;
+  p.tiles_per_seq = (int)tiles;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.timeout_ns = kWaitLimitNs;
+  const cudaError_t e = launch_prefill(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p,
+                                       reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
 }
 
 int pqkv_encode(const float* x, int64_t n, int code_dtype, uint8_t* codes, pqkv_stream_t stream) {

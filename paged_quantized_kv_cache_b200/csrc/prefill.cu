@@ -1,0 +1,622 @@
+// prefill.cu -- chunked-prefill attention over the paged, quantized KV cache,
+// on the sm_100a tensor cores (tcgen05, accumulators in tensor memory).
+//
+// Method: "vLLM" glossary, "Chunked prefill" (a long prompt is processed in
+// chunks) and "PagedAttention" (K/V read through the block table); "vLLM 0.7
+// Ships Unified KV Cache Compression", architecture diagram (512-token chunks)
+// and step 4 (the attention kernel reads the compressed codes and the fp16
+// outlier channels together). The q_len query tokens of a sequence are its last
+// q_len cached positions (the chunk is written to the cache first); query token
+// i at position p attends to positions 0..p.
+//
+// Work decomposition. One CTA (4 warps, 128 threads) per (sequence, KV head,
+// tile of 128 rows); a row is (query token, query head of the GQA group), so a
+// tile holds 128 / G query tokens, and thread r owns row r: its S and O rows
+// live in tensor-memory lane r. The CTA walks the KV positions the tile needs
+// in tiles of 64 tokens (4 cache blocks):
+//   S(t) = Q K(t)^T            tcgen05.mma M=128 N=64, two S buffers in TMEM
+//   online softmax of S(t)     one row per thread, no shuffles, lazy rescale
+//   O += P(t) V(t)             tcgen05.mma M=128 N=D, P from shared memory
+//                              (P = P_hi + P_lo in two products, except FP4)
+// S(t+1) is issued before the softmax of tile t, so the tensor cores compute
+// while the threads exponentiate. Operands are 128-byte-swizzled shared-memory
+// tiles: 16-bit K/V land there directly by TMA; FP8 / FP4 tiles are fetched raw
+// (one bulk copy per block plus its scales and outlier buffers) and the threads
+// dequantize them into f16 operands. FP8 scales stay out of the operands: the
+// K scale multiplies S, the V scale multiplies P relative to the largest V
+// scale seen so far (O is kept in units of it). FP4 operands are exact in f16
+// (E2M1 x E4M3 and the fp16 outlier values).
+#include <atomic>
+
+#include "prefill.cuh"
+#include "tcgen05.cuh"
+
+namespace pqkv {
+
+namespace {
+
+constexpr int kM = 128;        // rows (query token, head) per CTA
+constexpr int kN = 64;         // KV tokens per tile (4 blocks)
+constexpr int kThreads = 128;
+constexpr int kStages = 3;     // KV tiles in flight
+constexpr float kLazy = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+template <int KVF, int D>
+struct PrefillGeom {
+  static constexpr bool k16 = (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16);
+  static constexpr bool kFp8 = (KVF == PQKV_DTYPE_FP8_E4M3 || KVF == PQKV_DTYPE_FP8_E5M2);
+  static constexpr bool kFp4 = (KVF == PQKV_DTYPE_FP4_E2M1);
+  static constexpr int NB = D / 64;                // 128-byte boxes per operand row
+  static constexpr int kQBytes = NB * kM * 128;    // Q operand [box][128 rows][128 B]
+  static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
+  static constexpr int kPBytes = kM * 128;         // P operand: 64 tokens (2 B) per row
+  // P = P_hi + P_lo, both rounded to the operand type, keeps ~16 significant
+  // bits of the probabilities (a bf16 P alone errs by up to |v| 2^-9); FP4's
+  // tolerance allows a single f16 P
+  static constexpr bool kSplitP = !kFp4;
+  static constexpr int kRawTile = 32 * row_bytes(KVF, D);  // one block's K|V codes
+  static constexpr int kScaleBytes = kFp8 ? 16 : (kFp4 ? 2 * 16 * (D / 16) : 0);
+  static constexpr int kValBytes = kFp4 ? 2 * 16 * 4 * 2 : 0;
+  static constexpr int kIdxBytes = kFp4 ? 16 : 0;
+  static constexpr int kSide = kScaleBytes + kValBytes + kIdxBytes;
+  static constexpr int kRawStage = k16 ? 2 * kOpBytes : 4 * (kRawTile + kSide);
+  static constexpr int kStageBytes = (kRawStage + 1023) / 1024 * 1024;
+  static constexpr int kKops = k16 ? 0 : 2;        // dequantized K tiles (S of tile t-1 may still read one)
+  static constexpr int kVops = k16 ? 0 : 3;        // dequantized V tiles (PV of tile t-2 may still read one)
+  static constexpr int oQ = 0;
+  static constexpr int oStage = oQ + kQBytes;
+  static constexpr int oKop = oStage + kStages * kStageBytes;
+  static constexpr int oVop = oKop + kKops * kOpBytes;
+  static constexpr int oP = oVop + kVops * kOpBytes;
+  static constexpr int oMisc = oP + (kSplitP ? 2 : 1) * kPBytes;
+  static constexpr int kMiscBytes = 256;
+  static constexpr int kSmem = oMisc + kMiscBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kTmemCols = 256;      // O: columns [0, D); S buffers at D and D + 64
+};
+
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Bounded wait on an mbarrier phase, agreed by the whole CTA.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+  return __syncthreads_and(mbar_wait_bounded(bar, parity, limit_ns) ? 1 : 0) != 0;
+}
+
+// Replace element e (0..7) of eight f16 values held as four f16x2 words.
+__device__ __forceinline__ void put_half(uint32_t (&f)[4], int e, uint16_t v) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if ((e >> 1) == i) f[i] = (e & 1) ? ((f[i] & 0x0000FFFFu) | ((uint32_t)v << 16)) : ((f[i] & 0xFFFF0000u) | v);
+  }
+}
+
+// E4M3 scale byte -> f16x2 (s, s).
+__device__ __forceinline__ __half2 scale2(uint32_t byte) {
+  const uint32_t r = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(byte | (byte << 8));
+  return *reinterpret_cast<const __half2*>(&r);
+}
+
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, __half2 s) {
+  __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&a), s);
+  return *reinterpret_cast<uint32_t*>(&x);
+}
+
+}  // namespace
+
+template <int KVF, int D, bool QBF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap, const PrefillParams p) {
+  using Gm = PrefillGeom<KVF, D>;
+  constexpr bool kBfMma = (KVF == PQKV_DTYPE_BF16);  // operand type: bf16 for a bf16 cache, else f16
+  constexpr uint32_t kIdescS = tc::f16_idesc(kBfMma, kM, kN, false);
+  constexpr uint32_t kIdescPV = tc::f16_idesc(kBfMma, kM, D, true);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* sQ = smem + Gm::oQ;
+  uint8_t* sStage = smem + Gm::oStage;
+  uint8_t* sKop = smem + Gm::oKop;
+  uint8_t* sVop = smem + Gm::oVop;
+  uint8_t* sP = smem + Gm::oP;
+  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + Gm::oMisc);  // [kStages]
+  uint64_t* bar_s = bar_tma + kStages;                                // [2]
+  uint64_t* bar_pv = bar_s + 2;                                       // [1]
+  int* stage_mask = reinterpret_cast<int*>(bar_pv + 1);               // [kStages]: blocks loaded
+  int* tile_mask = stage_mask + kStages;                              // [2]: blocks holding valid tokens
+  float* tile_sk = reinterpret_cast<float*>(tile_mask + 2);           // [2][4] FP8 K scales
+  float* tile_sv = tile_sk + 8;                                       // [2][4] FP8 V scales
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
+
+  asm volatile("griddepcontrol.wait;" ::: "memory");  // the chunk's K/V may come from the previous kernel
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int h = blockIdx.y;
+  const int b = blockIdx.x / p.tiles_per_seq;
+  const int mt = p.tiles_per_seq - 1 - (int)(blockIdx.x % p.tiles_per_seq);  // long tiles first
+  const int G = p.G, TOK = kM / G;
+  const int q0 = p.cu_q[b], qn = p.cu_q[b + 1] - q0;
+  const int L = p.seq_lens[b];
+  const int i0 = mt * TOK;
+  if (i0 == 0 && h == 0 && threadIdx.x == 0 && qn > p.tiles_per_seq * TOK)
+    raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
+  if (qn <= 0 || i0 >= qn) return;
+  const int my_i = i0 + tid / G, my_n = tid % G;
+  const bool row_ok = my_i < qn;
+  const size_t orow = ((size_t)(q0 + (row_ok ? my_i : 0)) * p.Hq + (size_t)h * G + my_n) * D;
+  if (L < 0 || L > kBlock * p.maxblk || qn > L) {
+    if (i0 == 0 && h == 0 && tid == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
+    if (row_ok) {
+      uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) + orow * 2);
+      for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
+    }
+    return;
+  }
+  const int pos0 = L - qn;                          // position of query token 0
+  const int my_pos = pos0 + my_i;                   // this row attends to [0, my_pos]
+  const int n_kv = pos0 + min(i0 + TOK, qn);        // positions the tile reads
+  const int T = (n_kv + kN - 1) / kN;
+  const int32_t* table = p.block_tables + (size_t)b * p.maxblk;
+
+  // ---- setup: tensor memory, barriers, Q tile ----
+  if (warp == 0) tc::tmem_alloc(tmem_slot, Gm::kTmemCols);
+  if (tid == 32) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bar_tma[s], 1);
+    mbar_init(&bar_s[0], 1);
+    mbar_init(&bar_s[1], 1);
+    mbar_init(bar_pv, 1);
+    fence_mbar_init();
+  }
+  if constexpr (Gm::k16)
+    if (tid == 64) prefetch_tensormap(&tmap);
+  {
+    // row tid of Q, converted to the operand type, 16-byte chunks swizzled
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.q) + orow * 2);
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (row_ok) v = __ldg(src + c);
+      if constexpr (!Gm::k16 && QBF16) {  // bf16 query -> f16 operand
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = to_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        v = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      const int bx = c >> 3, ch = c & 7;
+      *reinterpret_cast<uint4*>(sQ + bx * (kM * 128) + tid * 128 + ((ch ^ (tid & 7)) << 4)) = v;
+    }
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+
+  uint32_t ph_tma = 0, ph_s = 0, ph_pv = 0;  // parity bits per barrier
+  bool aborted = false;
+  // operations issued and waited for (the same on every thread), so that a
+  // timeout can let the ones still in flight finish before the CTA exits
+  int n_issued = 0, n_prepared = 0, n_s = 0, n_s_waited = 0, n_pv_waited = 0;
+
+  // ---- producer: fetch the blocks of KV tile t into stage t % kStages (thread 0) ----
+  auto issue = [&](int t) {
+    const int s = t % kStages;
+    uint8_t* st = sStage + s * Gm::kStageBytes;
+    int ids[4];
+    int mask = 0;
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      ids[j] = -1;
+      const int blk = 4 * t + j;
+      if (blk * kBlock < n_kv) {
+        const int id = __ldg(table + blk);
+        if (id >= 0 && id < p.nb) {
+          ids[j] = id;
+          mask |= 1 << j;
+          bytes += Gm::k16 ? 2u * Gm::NB * kBlock * 128u : (uint32_t)(Gm::kRawTile + Gm::kSide);
+        } else {
+          raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
+        }
+      }
+    }
+    stage_mask[s] = mask;
+    mbar_arrive_expect_tx(&bar_tma[s], bytes);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (ids[j] < 0) continue;
+      const size_t pair = (size_t)ids[j] * p.Hkv + h;
+      if constexpr (Gm::k16) {
+        const int y = (int)pair * 32;
+#pragma unroll
+        for (int bx = 0; bx < Gm::NB; ++bx) {
+          tma_load_2d(st + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y, &bar_tma[s]);
+          tma_load_2d(st + Gm::kOpBytes + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y + 16, &bar_tma[s]);
+        }
+      } else {
+        bulk_load(st + j * Gm::kRawTile, p.cache + pair * Gm::kRawTile, Gm::kRawTile, &bar_tma[s]);
+        uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+        if constexpr (Gm::kFp8) {
+          bulk_load(side, p.scales + pair * 16, 16, &bar_tma[s]);
+        } else {
+          bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, &bar_tma[s]);
+          bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, &bar_tma[s]);
+          bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, &bar_tma[s]);
+        }
+      }
+    }
+  };
+
+  // ---- make KV tile t's operands ready (all threads); false on a timeout ----
+  auto prepare = [&](int t) -> bool {
+    const int s = t % kStages;
+    if (!cta_wait(&bar_tma[s], (ph_tma >> s) & 1u, p.timeout_ns)) return false;
+    ph_tma ^= 1u << s;
+    ++n_prepared;
+    const int mask = stage_mask[s];
+    const int base = t * kN;
+    uint8_t* st = sStage + s * Gm::kStageBytes;
+    if constexpr (Gm::k16) {
+      // V rows without valid data (past the sequence, or a block not loaded)
+      // are zeroed: P is 0 there, and 0 x NaN would poison O
+      if (mask != 0xF || base + kN > L) {
+        for (int u = tid; u < kN * Gm::NB * 8; u += kThreads) {
+          const int r = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
+          if (((mask >> (r >> 4)) & 1) && base + r < L) continue;
+          *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + r * 128 + ((k & 7) << 4)) =
+              make_uint4(0, 0, 0, 0);
+        }
+      }
+    } else {
+      uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
+      uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
+      constexpr int CPR = D / 8;  // 16-byte operand chunks per row
+      for (int u = tid; u < kN * CPR; u += kThreads) {
+        const int r = u / CPR, c = u % CPR, j = r >> 4, tr = r & 15;
+        const bool ok = ((mask >> j) & 1) && base + r < L;
+        uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
+        if (ok) {
+          const uint8_t* tile = st + j * Gm::kRawTile;
+          if constexpr (Gm::kFp8) {
+            const uint2 kc = *reinterpret_cast<const uint2*>(tile + tr * D + 8 * c);
+            const uint2 vc = *reinterpret_cast<const uint2*>(tile + (16 + tr) * D + 8 * c);
+            kf[0] = dec_fp8x2<KVF>(kc.x);
+            kf[1] = dec_fp8x2<KVF>(kc.x >> 16);
+            kf[2] = dec_fp8x2<KVF>(kc.y);
+            kf[3] = dec_fp8x2<KVF>(kc.y >> 16);
+            vf[0] = dec_fp8x2<KVF>(vc.x);
+            vf[1] = dec_fp8x2<KVF>(vc.x >> 16);
+            vf[2] = dec_fp8x2<KVF>(vc.y);
+            vf[3] = dec_fp8x2<KVF>(vc.y >> 16);
+          } else {
+            const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+            constexpr int SPR = D / 16;  // scale bytes per token row
+            // K: row tr, channels 8c..8c+7 = 4 bytes, channel 2i in the low nibble
+            dec_e2m1x8(*reinterpret_cast<const uint32_t*>(tile + tr * (D / 2) + 4 * c), kf);
+            // V: token-pair rows; this token's nibble of channels 8c..8c+7
+            const int hh = (8 * c) / (D / 2);
+            const int pr = tr < 8 ? (tr & ~1) : (((tr - 8) & ~1) + 1);
+            const uint2 wv = *reinterpret_cast<const uint2*>(tile + (16 + 8 * hh + pr) * (D / 2) + (8 * c) % (D / 2));
+            const uint32_t x0 = ((tr & 1) ? (wv.x >> 4) : wv.x) & 0x0F0F0F0Fu;
+            const uint32_t x1 = ((tr & 1) ? (wv.y >> 4) : wv.y) & 0x0F0F0F0Fu;
+            dec_e2m1x8(prmt(x0 | (x0 >> 4), x1 | (x1 >> 4), 0x6420u), vf);
+            const __half2 sk = scale2(side[tr * SPR + (c >> 1)]);
+            const __half2 sv = scale2(side[16 * SPR + tr * SPR + (c >> 1)]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              kf[i] = hmul2u(kf[i], sk);
+              vf[i] = hmul2u(vf[i], sv);
+            }
+            // outlier channels (their codes are 0): the fp16 values themselves
+            const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;
+            const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+              const int kc = idx[rr], vc = idx[8 + rr];
+              if (kc < D && (kc >> 3) == c) put_half(kf, kc & 7, val[tr * 4 + rr]);
+              if (vc < D && (vc >> 3) == c) put_half(vf, vc & 7, val[64 + tr * 4 + rr]);
+            }
+          }
+        }
+        const uint32_t off = (c >> 3) * (kN * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(kop + off) = make_uint4(kf[0], kf[1], kf[2], kf[3]);
+        *reinterpret_cast<uint4*>(vop + off) = make_uint4(vf[0], vf[1], vf[2], vf[3]);
+      }
+      if constexpr (Gm::kFp8) {
+        if (tid < 4) {
+          const bool ok = (mask >> tid) & 1;
+          const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + tid * Gm::kSide);
+          tile_sk[(t & 1) * 4 + tid] = ok ? sc[0] : 0.f;
+          tile_sv[(t & 1) * 4 + tid] = ok ? sc[1] : 0.f;
+        }
+      }
+    }
+    if (tid == 0) tile_mask[t & 1] = mask;
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    return true;
+  };
+
+  // ---- MMA issue (thread 0) ----
+  auto issue_s = [&](int t) {
+    tc::fence_after_sync();
+    const uint32_t d = tmem + D + 64 * (t & 1);
+    const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
+    const uint32_t qa = smem_u32(sQ), ka = smem_u32(kop);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+      const uint64_t bd = tc::sw128_desc(ka + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+      tc::mma_ss(d, a, bd, kIdescS, kk > 0);
+    }
+    tc::commit(&bar_s[t & 1]);
+  };
+  auto issue_pv = [&](int t, bool first) {
+    tc::fence_after_sync();
+    const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
+                                 : sVop + (t % 3) * Gm::kOpBytes;
+    const uint32_t pa = smem_u32(sP), va = smem_u32(vop);
+#pragma unroll
+    for (int kk = 0; kk < kN / 16; ++kk) {
+      const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
+      tc::mma_ss(tmem, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
+      if constexpr (Gm::kSplitP)
+        tc::mma_ss(tmem, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
+    }
+    tc::commit(bar_pv);
+  };
+
+  // ---- main loop ----
+  float m = -INFINITY, l = 0.f, vref = 0.f;
+  int pv_done = 0;  // PV products issued so far
+  if (tid == 0) {
+    issue(0);
+    if (T > 1) issue(1);
+  }
+  n_issued = T > 1 ? 2 : 1;
+  if (!prepare(0)) aborted = true;
+  else {
+    if (tid == 0) issue_s(0);
+    n_s = 1;
+  }
+
+  for (int t = 0; t < T && !aborted; ++t) {
+    if (t + 1 < T) {
+      if (!prepare(t + 1)) { aborted = true; break; }
+      if (tid == 0) issue_s(t + 1);
+      ++n_s;
+    }
+    if (!cta_wait(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns)) { aborted = true; break; }
+    ph_s ^= 1u << (t & 1);
+    ++n_s_waited;
+    tc::fence_after_sync();
+
+    // scores of this row
+    uint32_t sv[64];
+    {
+      uint32_t a[32], c2[32];
+      tc::tmem_ld32(t_row + D + 64 * (t & 1), a);
+      tc::tmem_ld32(t_row + D + 64 * (t & 1) + 32, c2);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        sv[i] = a[i];
+        sv[32 + i] = c2[i];
+      }
+    }
+    const int mask = tile_mask[t & 1];
+    float ks[4] = {1.f, 1.f, 1.f, 1.f};
+    float vs[4] = {1.f, 1.f, 1.f, 1.f};
+    if constexpr (Gm::kFp8) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ks[j] = tile_sk[(t & 1) * 4 + j];
+        vs[j] = tile_sv[(t & 1) * 4 + j];
+      }
+    }
+    float x[64];
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 64; ++c) {
+      const int j = c >> 4;
+      float v = __uint_as_float(sv[c]) * (p.scale_log2 * ks[j]);
+      if (t * kN + c > my_pos || !((mask >> j) & 1) || !row_ok) v = -INFINITY;
+      x[c] = v;
+      mx = fmaxf(mx, v);
+    }
+    float fm = 1.f;  // rescale of l and O for a larger row max
+    if (mx > m + kLazy) {
+      fm = ex2(m - mx);  // 0 when m was -inf
+      m = mx;
+    }
+    float fv = 1.f;  // FP8: O moves to units of a larger V scale (same on every thread)
+    if constexpr (Gm::kFp8) {
+      float svm = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if ((mask >> j) & 1) svm = fmaxf(svm, vs[j]);
+      if (svm > vref) {
+        fv = vref / svm;
+        vref = svm;
+      }
+    }
+    l *= fm;
+    const float fo = fm * fv;
+    uint32_t pk[32], pl[32];
+    {
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 64; c += 2) {
+        const float pa = (m == -INFINITY) ? 0.f : ex2(x[c] - m);
+        const float pb = (m == -INFINITY) ? 0.f : ex2(x[c + 1] - m);
+        rs += pa + pb;
+        float wa = pa, wb = pb;
+        if constexpr (Gm::kFp8) {
+          const float r = vref > 0.f ? vs[c >> 4] / vref : 0.f;
+          wa *= r;
+          wb *= r;
+        }
+        pk[c >> 1] = pack_f32x2(wa, wb, kBfMma);
+        if constexpr (Gm::kSplitP)
+          pl[c >> 1] = pack_f32x2(wa - unpack_lo(pk[c >> 1], kBfMma), wb - unpack_hi(pk[c >> 1], kBfMma), kBfMma);
+      }
+      l += rs;
+    }
+
+    // PV(t-1) must be done before O is rescaled or P is overwritten
+    if (t > 0) {
+      if (!cta_wait(bar_pv, ph_pv, p.timeout_ns)) { aborted = true; break; }
+      ph_pv ^= 1u;
+      ++n_pv_waited;
+      tc::fence_after_sync();
+    }
+    if (pv_done > 0 && __any_sync(kFull, fo != 1.f)) {
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tc::tmem_ld32(t_row + c0, o);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
+        tc::tmem_st32(t_row + c0, o);
+      }
+    }
+    // P row -> shared memory (K-major operand, 128-byte swizzle)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      *reinterpret_cast<uint4*>(sP + tid * 128 + ((c ^ (tid & 7)) << 4)) =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      if constexpr (Gm::kSplitP)
+        *reinterpret_cast<uint4*>(sP + Gm::kPBytes + tid * 128 + ((c ^ (tid & 7)) << 4)) =
+            make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+    }
+    tc::fence_smem_to_async();
+    tc::fence_before_sync();
+    __syncthreads();
+    if (tid == 0) {
+      issue_pv(t, pv_done == 0);
+      if (t + 2 < T) issue(t + 2);
+    }
+    ++pv_done;
+    if (t + 2 < T) ++n_issued;
+  }
+
+  if (!aborted && pv_done > 0) {
+    if (!cta_wait(bar_pv, ph_pv, p.timeout_ns)) aborted = true;
+    else {
+      ph_pv ^= 1u;
+      ++n_pv_waited;
+    }
+  }
+  if (aborted) {
+    if (tid == 0) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+    // let copies and products still in flight land (each wait bounded)
+    for (int k = n_prepared; k < n_issued; ++k)
+      (void)mbar_wait_bounded(&bar_tma[k % kStages], (uint32_t)(k / kStages) & 1u, p.timeout_ns);
+    for (int k = n_s_waited; k < n_s; ++k)
+      (void)mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.timeout_ns);
+    for (int k = n_pv_waited; k < pv_done; ++k)
+      (void)mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.timeout_ns);
+  } else {
+    tc::fence_after_sync();
+    const float inv = l > 0.f ? (Gm::kFp8 ? vref : 1.f) / l : 0.f;
+    uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + orow * 2;
+#pragma unroll 1
+    for (int c0 = 0; c0 < D; c0 += 32) {
+      uint32_t o[32];
+      tc::tmem_ld32(t_row + c0, o);
+      if (row_ok) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t w[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            w[i] = pack_f32x2(__uint_as_float(o[8 * k + 2 * i]) * inv, __uint_as_float(o[8 * k + 2 * i + 1]) * inv,
+                              QBF16);
+          *reinterpret_cast<uint4*>(dst + (c0 + 8 * k) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+      }
+    }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, Gm::kTmemCols);
+  }
+}
+
+// ---- launch ------------------------------------------------------------------
+
+template <int KVF, int D, bool QBF16>
+static cudaError_t launch_prefill_t(const CUtensorMap& tmap, const PrefillParams& p, cudaStream_t st) {
+  auto kern = paged_prefill_kernel<KVF, D, QBF16>;
+  constexpr int smem = PrefillGeom<KVF, D>::kSmem;
+  static std::atomic<uint64_t> configured{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (!(configured.load() & bit)) {
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(bit);
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.B * p.tiles_per_seq), (unsigned)p.Hkv);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tmap, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+size_t prefill_smem_bytes(int kv_dtype, int D) {
+#define PQKV_PS(F)                                                                               \
+  if (kv_dtype == F) return D == 128 ? PrefillGeom<F, 128>::kSmem : PrefillGeom<F, 64>::kSmem;
+  PQKV_PS(PQKV_DTYPE_FP16)
+  PQKV_PS(PQKV_DTYPE_BF16)
+  PQKV_PS(PQKV_DTYPE_FP8_E4M3)
+  PQKV_PS(PQKV_DTYPE_FP8_E5M2)
+  PQKV_PS(PQKV_DTYPE_FP4_E2M1)
+#undef PQKV_PS
+  return 0;
+}
+
+cudaError_t launch_prefill(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap16, const PrefillParams& p,
+                           cudaStream_t st) {
+#define PQKV_PF(KVF, DD, QB) \
+  if (kv_dtype == KVF && D == DD && q_bf16 == QB) return launch_prefill_t<KVF, DD, QB>(tmap16, p, st);
+  PQKV_PF(PQKV_DTYPE_FP16, 128, false)
+  PQKV_PF(PQKV_DTYPE_FP16, 64, false)
+  PQKV_PF(PQKV_DTYPE_BF16, 128, true)
+  PQKV_PF(PQKV_DTYPE_BF16, 64, true)
+  PQKV_PF(PQKV_DTYPE_FP8_E4M3, 128, true)
+  PQKV_PF(PQKV_DTYPE_FP8_E4M3, 128, false)
+  PQKV_PF(PQKV_DTYPE_FP8_E4M3, 64, true)
+  PQKV_PF(PQKV_DTYPE_FP8_E4M3, 64, false)
+  PQKV_PF(PQKV_DTYPE_FP8_E5M2, 128, true)
+  PQKV_PF(PQKV_DTYPE_FP8_E5M2, 128, false)
+  PQKV_PF(PQKV_DTYPE_FP8_E5M2, 64, true)
+  PQKV_PF(PQKV_DTYPE_FP8_E5M2, 64, false)
+  PQKV_PF(PQKV_DTYPE_FP4_E2M1, 128, true)
+  PQKV_PF(PQKV_DTYPE_FP4_E2M1, 128, false)
+  PQKV_PF(PQKV_DTYPE_FP4_E2M1, 64, true)
+  PQKV_PF(PQKV_DTYPE_FP4_E2M1, 64, false)
+#undef PQKV_PF
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace pqkv
