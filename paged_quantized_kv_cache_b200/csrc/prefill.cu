@@ -9,11 +9,14 @@
 // q_len cached positions (the chunk is written to the cache first); query token
 // i at position p attends to positions 0..p.
 //
-// Work decomposition. One CTA (4 warps, 128 threads) per (sequence, KV head,
-// tile of 128 rows); a row is (query token, query head of the GQA group), so a
-// tile holds 128 / G query tokens, and thread r owns row r: its S and O rows
-// live in tensor-memory lane r. The CTA walks the KV positions the tile needs
-// in tiles of 64 tokens (4 cache blocks):
+// Work decomposition. One CTA per (sequence, KV head, tile of 128 rows); a row
+// is (query token, query head of the GQA group), so a tile holds 128 / G query
+// tokens. Four compute warps own one row each per thread (its S and O rows live
+// in tensor-memory lane r); a fifth warp only fetches: it refills each stage of
+// a 4-deep ring as soon as the stage is released (by a tcgen05 commit after
+// the last product reading it, or once its raw codes are dequantized). The
+// compute warps walk the KV positions the tile needs in tiles of 64 tokens (4
+// cache blocks):
 //   S(t) = Q K(t)^T            tcgen05.mma M=128 N=64, two S buffers in TMEM
 //   online softmax of S(t)     one row per thread, no shuffles, lazy rescale
 //   O += P(t) V(t)             tcgen05.mma M=128 N=D, P from shared memory
@@ -37,8 +40,9 @@ namespace {
 
 constexpr int kM = 128;        // rows (query token, head) per CTA
 constexpr int kN = 64;         // KV tokens per tile (4 blocks)
-constexpr int kThreads = 128;
-constexpr int kStages = 3;     // KV tiles in flight
+constexpr int kComputeThreads = 128;              // 4 warps: one row (TMEM lane) per thread
+constexpr int kThreads = kComputeThreads + 32;     // + one producer warp
+constexpr int kStages = 4;     // KV tiles in flight
 constexpr float kLazy = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -86,17 +90,19 @@ __device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Bounded wait on an mbarrier phase, agreed by the whole CTA.
-__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
-  return __syncthreads_and(mbar_wait_bounded(bar, parity, limit_ns) ? 1 : 0) != 0;
-}
-
-// Replace element e (0..7) of eight f16 values held as four f16x2 words.
-__device__ __forceinline__ void put_half(uint32_t (&f)[4], int e, uint16_t v) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if ((e >> 1) == i) f[i] = (e & 1) ? ((f[i] & 0x0000FFFFu) | ((uint32_t)v << 16)) : ((f[i] & 0xFFFF0000u) | v);
-  }
+// Barrier of the 128 compute threads only (named barrier 1; the producer warp
+// runs on its own).
+__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// The same barrier, returning whether v held on every compute thread.
+__device__ __forceinline__ bool compute_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v)
+      : "memory");
+  return r != 0;
 }
 
 // E4M3 scale byte -> f16x2 (s, s).
@@ -127,17 +133,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sKop = smem + Gm::oKop;
   uint8_t* sVop = smem + Gm::oVop;
   uint8_t* sP = smem + Gm::oP;
-  uint64_t* bar_tma = reinterpret_cast<uint64_t*>(smem + Gm::oMisc);  // [kStages]
-  uint64_t* bar_s = bar_tma + kStages;                                // [2]
-  uint64_t* bar_pv = bar_s + 2;                                       // [1]
-  int* stage_mask = reinterpret_cast<int*>(bar_pv + 1);               // [kStages]: blocks loaded
-  int* tile_mask = stage_mask + kStages;                              // [2]: blocks holding valid tokens
-  float* tile_sk = reinterpret_cast<float*>(tile_mask + 2);           // [2][4] FP8 K scales
-  float* tile_sv = tile_sk + 8;                                       // [2][4] FP8 V scales
+  uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Gm::oMisc);  // [kStages] tile landed
+  uint64_t* bar_empty = bar_full + kStages;                             // [kStages] stage free again
+  uint64_t* bar_s = bar_empty + kStages;                                // [2] S(t) computed
+  uint64_t* bar_pv = bar_s + 2;                                         // [1] PV(t) computed
+  int* stage_mask = reinterpret_cast<int*>(bar_pv + 1);                 // [kStages] blocks loaded
+  int* tile_mask = stage_mask + kStages;                                // [2] blocks holding valid tokens
+  float* tile_sk = reinterpret_cast<float*>(tile_mask + 2);             // [2][4] FP8 K scales
+  float* tile_sv = tile_sk + 8;                                         // [2][4] FP8 V scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* n_issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
 
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the chunk's K/V may come from the previous kernel
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
   const int b = blockIdx.x / p.tiles_per_seq;
   const int mt = p.tiles_per_seq - 1 - (int)(blockIdx.x % p.tiles_per_seq);  // long tiles first
@@ -145,11 +154,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int q0 = p.cu_q[b], qn = p.cu_q[b + 1] - q0;
   const int L = p.seq_lens[b];
   const int i0 = mt * TOK;
-  if (i0 == 0 && h == 0 && threadIdx.x == 0 && qn > p.tiles_per_seq * TOK)
+  if (i0 == 0 && h == 0 && tid == 0 && qn > p.tiles_per_seq * TOK)
     raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
   if (qn <= 0 || i0 >= qn) return;
-  const int my_i = i0 + tid / G, my_n = tid % G;
-  const bool row_ok = my_i < qn;
+  const int r = tid & (kM - 1);  // compute thread tid = row r (the producer warp has no row)
+  const int my_i = i0 + r / G, my_n = r % G;
+  const bool row_ok = tid < kComputeThreads && my_i < qn;
   const size_t orow = ((size_t)(q0 + (row_ok ? my_i : 0)) * p.Hq + (size_t)h * G + my_n) * D;
   if (L < 0 || L > kBlock * p.maxblk || qn > L) {
     if (i0 == 0 && h == 0 && tid == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
@@ -168,16 +178,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   // ---- setup: tensor memory, barriers, Q tile ----
   if (warp == 0) tc::tmem_alloc(tmem_slot, Gm::kTmemCols);
   if (tid == 32) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bar_tma[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bar_full[s], 1);
+      mbar_init(&bar_empty[s], 1);
+    }
     mbar_init(&bar_s[0], 1);
     mbar_init(&bar_s[1], 1);
     mbar_init(bar_pv, 1);
+    *abort_flag = 0;
+    *n_issued_slot = 0;
     fence_mbar_init();
   }
   if constexpr (Gm::k16)
-    if (tid == 64) prefetch_tensormap(&tmap);
-  {
-    // row tid of Q, converted to the operand type, 16-byte chunks swizzled
+    if (tid == kComputeThreads) prefetch_tensormap(&tmap);
+  if (tid < kComputeThreads) {
+    // row r of Q, converted to the operand type, 16-byte chunks swizzled
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.q) + orow * 2);
 #pragma unroll 4
     for (int c = 0; c < D / 8; ++c) {
@@ -190,7 +205,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         v = make_uint4(w[0], w[1], w[2], w[3]);
       }
       const int bx = c >> 3, ch = c & 7;
-      *reinterpret_cast<uint4*>(sQ + bx * (kM * 128) + tid * 128 + ((ch ^ (tid & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(sQ + bx * (kM * 128) + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
     }
   }
   tc::fence_smem_to_async();
@@ -198,355 +213,418 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+  int n_prepared = 0;  // KV tiles consumed by the compute warps
 
-  uint32_t ph_tma = 0, ph_s = 0, ph_pv = 0;  // parity bits per barrier
-  bool aborted = false;
-  // operations issued and waited for (the same on every thread), so that a
-  // timeout can let the ones still in flight finish before the CTA exits
-  int n_issued = 0, n_prepared = 0, n_s = 0, n_s_waited = 0, n_pv_waited = 0;
-
-  // ---- producer: fetch the blocks of KV tile t into stage t % kStages (thread 0) ----
-  auto issue = [&](int t) {
-    const int s = t % kStages;
-    uint8_t* st = sStage + s * Gm::kStageBytes;
-    int ids[4];
-    int mask = 0;
-    uint32_t bytes = 0;
+  if (warp == kComputeThreads / 32) {
+    // ================= producer warp: KV tiles into the stage ring =================
+    if (lane == 0) {
+      int t = 0;
+      for (; t < T; ++t) {
+        const int s = t % kStages;
+        if (t >= kStages &&
+            !mbar_wait_bounded(&bar_empty[s], (uint32_t)((t / kStages) - 1) & 1u, p.timeout_ns))
+          break;
+        if (*abort_flag) break;
+        uint8_t* st = sStage + s * Gm::kStageBytes;
+        int ids[4];
+        int mask = 0;
+        uint32_t bytes = 0;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      ids[j] = -1;
-      const int blk = 4 * t + j;
-      if (blk * kBlock < n_kv) {
-        const int id = __ldg(table + blk);
-        if (id >= 0 && id < p.nb) {
-          ids[j] = id;
-          mask |= 1 << j;
-          bytes += Gm::k16 ? 2u * Gm::NB * kBlock * 128u : (uint32_t)(Gm::kRawTile + Gm::kSide);
-        } else {
-          raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
-        }
-      }
-    }
-    stage_mask[s] = mask;
-    mbar_arrive_expect_tx(&bar_tma[s], bytes);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      if (ids[j] < 0) continue;
-      const size_t pair = (size_t)ids[j] * p.Hkv + h;
-      if constexpr (Gm::k16) {
-        const int y = (int)pair * 32;
-#pragma unroll
-        for (int bx = 0; bx < Gm::NB; ++bx) {
-          tma_load_2d(st + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y, &bar_tma[s]);
-          tma_load_2d(st + Gm::kOpBytes + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y + 16, &bar_tma[s]);
-        }
-      } else {
-        bulk_load(st + j * Gm::kRawTile, p.cache + pair * Gm::kRawTile, Gm::kRawTile, &bar_tma[s]);
-        uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
-        if constexpr (Gm::kFp8) {
-          bulk_load(side, p.scales + pair * 16, 16, &bar_tma[s]);
-        } else {
-          bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, &bar_tma[s]);
-          bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, &bar_tma[s]);
-          bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, &bar_tma[s]);
-        }
-      }
-    }
-  };
-
-  // ---- make KV tile t's operands ready (all threads); false on a timeout ----
-  auto prepare = [&](int t) -> bool {
-    const int s = t % kStages;
-    if (!cta_wait(&bar_tma[s], (ph_tma >> s) & 1u, p.timeout_ns)) return false;
-    ph_tma ^= 1u << s;
-    ++n_prepared;
-    const int mask = stage_mask[s];
-    const int base = t * kN;
-    uint8_t* st = sStage + s * Gm::kStageBytes;
-    if constexpr (Gm::k16) {
-      // V rows without valid data (past the sequence, or a block not loaded)
-      // are zeroed: P is 0 there, and 0 x NaN would poison O
-      if (mask != 0xF || base + kN > L) {
-        for (int u = tid; u < kN * Gm::NB * 8; u += kThreads) {
-          const int r = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
-          if (((mask >> (r >> 4)) & 1) && base + r < L) continue;
-          *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + r * 128 + ((k & 7) << 4)) =
-              make_uint4(0, 0, 0, 0);
-        }
-      }
-    } else {
-      uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
-      uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
-      constexpr int CPR = D / 8;  // 16-byte operand chunks per row
-      for (int u = tid; u < kN * CPR; u += kThreads) {
-        const int r = u / CPR, c = u % CPR, j = r >> 4, tr = r & 15;
-        const bool ok = ((mask >> j) & 1) && base + r < L;
-        uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
-        if (ok) {
-          const uint8_t* tile = st + j * Gm::kRawTile;
-          if constexpr (Gm::kFp8) {
-            const uint2 kc = *reinterpret_cast<const uint2*>(tile + tr * D + 8 * c);
-            const uint2 vc = *reinterpret_cast<const uint2*>(tile + (16 + tr) * D + 8 * c);
-            kf[0] = dec_fp8x2<KVF>(kc.x);
-            kf[1] = dec_fp8x2<KVF>(kc.x >> 16);
-            kf[2] = dec_fp8x2<KVF>(kc.y);
-            kf[3] = dec_fp8x2<KVF>(kc.y >> 16);
-            vf[0] = dec_fp8x2<KVF>(vc.x);
-            vf[1] = dec_fp8x2<KVF>(vc.x >> 16);
-            vf[2] = dec_fp8x2<KVF>(vc.y);
-            vf[3] = dec_fp8x2<KVF>(vc.y >> 16);
-          } else {
-            const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
-            constexpr int SPR = D / 16;  // scale bytes per token row
-            // K: row tr, channels 8c..8c+7 = 4 bytes, channel 2i in the low nibble
-            dec_e2m1x8(*reinterpret_cast<const uint32_t*>(tile + tr * (D / 2) + 4 * c), kf);
-            // V: token-pair rows; this token's nibble of channels 8c..8c+7
-            const int hh = (8 * c) / (D / 2);
-            const int pr = tr < 8 ? (tr & ~1) : (((tr - 8) & ~1) + 1);
-            const uint2 wv = *reinterpret_cast<const uint2*>(tile + (16 + 8 * hh + pr) * (D / 2) + (8 * c) % (D / 2));
-            const uint32_t x0 = ((tr & 1) ? (wv.x >> 4) : wv.x) & 0x0F0F0F0Fu;
-            const uint32_t x1 = ((tr & 1) ? (wv.y >> 4) : wv.y) & 0x0F0F0F0Fu;
-            dec_e2m1x8(prmt(x0 | (x0 >> 4), x1 | (x1 >> 4), 0x6420u), vf);
-            const __half2 sk = scale2(side[tr * SPR + (c >> 1)]);
-            const __half2 sv = scale2(side[16 * SPR + tr * SPR + (c >> 1)]);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              kf[i] = hmul2u(kf[i], sk);
-              vf[i] = hmul2u(vf[i], sv);
-            }
-            // outlier channels (their codes are 0): the fp16 values themselves
-            const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;
-            const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);
-#pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
-              const int kc = idx[rr], vc = idx[8 + rr];
-              if (kc < D && (kc >> 3) == c) put_half(kf, kc & 7, val[tr * 4 + rr]);
-              if (vc < D && (vc >> 3) == c) put_half(vf, vc & 7, val[64 + tr * 4 + rr]);
+        for (int j = 0; j < 4; ++j) {
+          ids[j] = -1;
+          const int blk = 4 * t + j;
+          if (blk * kBlock < n_kv) {
+            const int id = __ldg(table + blk);
+            if (id >= 0 && id < p.nb) {
+              ids[j] = id;
+              mask |= 1 << j;
+              bytes += Gm::k16 ? 2u * Gm::NB * kBlock * 128u : (uint32_t)(Gm::kRawTile + Gm::kSide);
+            } else {
+              raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
             }
           }
         }
-        const uint32_t off = (c >> 3) * (kN * 128) + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(kop + off) = make_uint4(kf[0], kf[1], kf[2], kf[3]);
-        *reinterpret_cast<uint4*>(vop + off) = make_uint4(vf[0], vf[1], vf[2], vf[3]);
-      }
-      if constexpr (Gm::kFp8) {
-        if (tid < 4) {
-          const bool ok = (mask >> tid) & 1;
-          const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + tid * Gm::kSide);
-          tile_sk[(t & 1) * 4 + tid] = ok ? sc[0] : 0.f;
-          tile_sv[(t & 1) * 4 + tid] = ok ? sc[1] : 0.f;
+        stage_mask[s] = mask;
+        mbar_arrive_expect_tx(&bar_full[s], bytes);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (ids[j] < 0) continue;
+          const size_t pair = (size_t)ids[j] * p.Hkv + h;
+          if constexpr (Gm::k16) {
+            const int y = (int)pair * 32;
+#pragma unroll
+            for (int bx = 0; bx < Gm::NB; ++bx) {
+              tma_load_2d(st + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y, &bar_full[s]);
+              tma_load_2d(st + Gm::kOpBytes + bx * kN * 128 + j * kBlock * 128, &tmap, bx * 64, y + 16,
+                          &bar_full[s]);
+            }
+          } else {
+            bulk_load(st + j * Gm::kRawTile, p.cache + pair * Gm::kRawTile, Gm::kRawTile, &bar_full[s]);
+            uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+            if constexpr (Gm::kFp8) {
+              bulk_load(side, p.scales + pair * 16, 16, &bar_full[s]);
+            } else {
+              bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, &bar_full[s]);
+              bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, &bar_full[s]);
+              bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, &bar_full[s]);
+            }
+          }
         }
       }
+      *n_issued_slot = t;
     }
-    if (tid == 0) tile_mask[t & 1] = mask;
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    return true;
-  };
+  } else {
+    // ================= compute warpgroup: one row per thread =================
+    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+    uint32_t ph_full = 0, ph_s = 0, ph_pv = 0;  // parity bits per barrier
+    bool aborted = false;
+    // operations issued and waited for (the same on every thread), so that a
+    // timeout can let the ones still in flight finish before the CTA exits
+    int n_s = 0, n_s_waited = 0, n_pv_waited = 0;
 
-  // ---- MMA issue (thread 0) ----
-  auto issue_s = [&](int t) {
-    tc::fence_after_sync();
-    const uint32_t d = tmem + D + 64 * (t & 1);
-    const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
-    const uint32_t qa = smem_u32(sQ), ka = smem_u32(kop);
+    // ---- make KV tile t's operands ready; false on a timeout ----
+    auto prepare = [&](int t) -> bool {
+      const int s = t % kStages;
+      if (!compute_all(mbar_wait_bounded(&bar_full[s], (ph_full >> s) & 1u, p.timeout_ns))) return false;
+      ph_full ^= 1u << s;
+      ++n_prepared;
+      const int mask = stage_mask[s];
+      const int base = t * kN;
+      uint8_t* st = sStage + s * Gm::kStageBytes;
+      if constexpr (Gm::k16) {
+        // V rows without valid data (past the sequence, or a block not loaded)
+        // are zeroed: P is 0 there, and 0 x NaN would poison O
+        if (mask != 0xF || base + kN > L) {
+          for (int u = r; u < kN * Gm::NB * 8; u += kComputeThreads) {
+            const int rr = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
+            if (((mask >> (rr >> 4)) & 1) && base + rr < L) continue;
+            *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + rr * 128 + ((k & 7) << 4)) =
+                make_uint4(0, 0, 0, 0);
+          }
+        }
+      } else {
+        uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
+        uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
+        constexpr int CPR = D / 8;  // 16-byte operand chunks per row
+        for (int u = r; u < kN * CPR; u += kComputeThreads) {
+          const int rr = u / CPR, c = u % CPR, j = rr >> 4, tr = rr & 15;
+          const bool ok = ((mask >> j) & 1) && base + rr < L;
+          uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
+          if (ok) {
+            const uint8_t* tile = st + j * Gm::kRawTile;
+            if constexpr (Gm::kFp8) {
+              const uint2 kc = *reinterpret_cast<const uint2*>(tile + tr * D + 8 * c);
+              const uint2 vc = *reinterpret_cast<const uint2*>(tile + (16 + tr) * D + 8 * c);
+              kf[0] = dec_fp8x2<KVF>(kc.x);
+              kf[1] = dec_fp8x2<KVF>(kc.x >> 16);
+              kf[2] = dec_fp8x2<KVF>(kc.y);
+              kf[3] = dec_fp8x2<KVF>(kc.y >> 16);
+              vf[0] = dec_fp8x2<KVF>(vc.x);
+              vf[1] = dec_fp8x2<KVF>(vc.x >> 16);
+              vf[2] = dec_fp8x2<KVF>(vc.y);
+              vf[3] = dec_fp8x2<KVF>(vc.y >> 16);
+            } else {
+              const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+              constexpr int SPR = D / 16;  // scale bytes per token row
+              // K: row tr, channels 8c..8c+7 = 4 bytes, channel 2i in the low nibble
+              dec_e2m1x8(*reinterpret_cast<const uint32_t*>(tile + tr * (D / 2) + 4 * c), kf);
+              // V: token-pair rows; this token's nibble of channels 8c..8c+7
+              const int hh = (8 * c) / (D / 2);
+              const int pr = tr < 8 ? (tr & ~1) : (((tr - 8) & ~1) + 1);
+              const uint2 wv =
+                  *reinterpret_cast<const uint2*>(tile + (16 + 8 * hh + pr) * (D / 2) + (8 * c) % (D / 2));
+              const uint32_t x0 = ((tr & 1) ? (wv.x >> 4) : wv.x) & 0x0F0F0F0Fu;
+              const uint32_t x1 = ((tr & 1) ? (wv.y >> 4) : wv.y) & 0x0F0F0F0Fu;
+              dec_e2m1x8(prmt(x0 | (x0 >> 4), x1 | (x1 >> 4), 0x6420u), vf);
+              const __half2 sk = scale2(side[tr * SPR + (c >> 1)]);
+              const __half2 sv = scale2(side[16 * SPR + tr * SPR + (c >> 1)]);
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-      const uint64_t bd = tc::sw128_desc(ka + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-      tc::mma_ss(d, a, bd, kIdescS, kk > 0);
-    }
-    tc::commit(&bar_s[t & 1]);
-  };
-  auto issue_pv = [&](int t, bool first) {
-    tc::fence_after_sync();
-    const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
-                                 : sVop + (t % 3) * Gm::kOpBytes;
-    const uint32_t pa = smem_u32(sP), va = smem_u32(vop);
+              for (int i = 0; i < 4; ++i) {
+                kf[i] = hmul2u(kf[i], sk);
+                vf[i] = hmul2u(vf[i], sv);
+              }
+            }
+          }
+          const uint32_t off = (c >> 3) * (kN * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4);
+          *reinterpret_cast<uint4*>(kop + off) = make_uint4(kf[0], kf[1], kf[2], kf[3]);
+          *reinterpret_cast<uint4*>(vop + off) = make_uint4(vf[0], vf[1], vf[2], vf[3]);
+        }
+        if constexpr (Gm::kFp4) {
+          // outlier channels (their codes are 0): write the fp16 values over them;
+          // thread = (block j, K|V, slot, half of the tokens)
+          compute_sync();
+          {
+            const int j = r >> 5, kv = (r >> 4) & 1, slot = (r >> 2) & 3, part = r & 3;
+            if ((mask >> j) & 1) {
+              const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+              const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
+              if (ch < D) {
+                const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes) + kv * 64;
+                uint8_t* op = kv ? vop : kop;
+                const int c = ch >> 3;
 #pragma unroll
-    for (int kk = 0; kk < kN / 16; ++kk) {
-      const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
-      tc::mma_ss(tmem, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
-      if constexpr (Gm::kSplitP)
-        tc::mma_ss(tmem, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
-    }
-    tc::commit(bar_pv);
-  };
-
-  // ---- main loop ----
-  float m = -INFINITY, l = 0.f, vref = 0.f;
-  int pv_done = 0;  // PV products issued so far
-  if (tid == 0) {
-    issue(0);
-    if (T > 1) issue(1);
-  }
-  n_issued = T > 1 ? 2 : 1;
-  if (!prepare(0)) aborted = true;
-  else {
-    if (tid == 0) issue_s(0);
-    n_s = 1;
-  }
-
-  for (int t = 0; t < T && !aborted; ++t) {
-    if (t + 1 < T) {
-      if (!prepare(t + 1)) { aborted = true; break; }
-      if (tid == 0) issue_s(t + 1);
-      ++n_s;
-    }
-    if (!cta_wait(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns)) { aborted = true; break; }
-    ph_s ^= 1u << (t & 1);
-    ++n_s_waited;
-    tc::fence_after_sync();
-
-    // scores of this row
-    uint32_t sv[64];
-    {
-      uint32_t a[32], c2[32];
-      tc::tmem_ld32(t_row + D + 64 * (t & 1), a);
-      tc::tmem_ld32(t_row + D + 64 * (t & 1) + 32, c2);
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        sv[i] = a[i];
-        sv[32 + i] = c2[i];
-      }
-    }
-    const int mask = tile_mask[t & 1];
-    float ks[4] = {1.f, 1.f, 1.f, 1.f};
-    float vs[4] = {1.f, 1.f, 1.f, 1.f};
-    if constexpr (Gm::kFp8) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        ks[j] = tile_sk[(t & 1) * 4 + j];
-        vs[j] = tile_sv[(t & 1) * 4 + j];
-      }
-    }
-    float x[64];
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const int j = c >> 4;
-      float v = __uint_as_float(sv[c]) * (p.scale_log2 * ks[j]);
-      if (t * kN + c > my_pos || !((mask >> j) & 1) || !row_ok) v = -INFINITY;
-      x[c] = v;
-      mx = fmaxf(mx, v);
-    }
-    float fm = 1.f;  // rescale of l and O for a larger row max
-    if (mx > m + kLazy) {
-      fm = ex2(m - mx);  // 0 when m was -inf
-      m = mx;
-    }
-    float fv = 1.f;  // FP8: O moves to units of a larger V scale (same on every thread)
-    if constexpr (Gm::kFp8) {
-      float svm = 0.f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        if ((mask >> j) & 1) svm = fmaxf(svm, vs[j]);
-      if (svm > vref) {
-        fv = vref / svm;
-        vref = svm;
-      }
-    }
-    l *= fm;
-    const float fo = fm * fv;
-    uint32_t pk[32], pl[32];
-    {
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float pa = (m == -INFINITY) ? 0.f : ex2(x[c] - m);
-        const float pb = (m == -INFINITY) ? 0.f : ex2(x[c + 1] - m);
-        rs += pa + pb;
-        float wa = pa, wb = pb;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                  const int tr = 4 * part + q4, rr = 16 * j + tr;
+                  if (base + rr < L)
+                    *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 +
+                                                 (((c & 7) ^ (rr & 7)) << 4) + (ch & 7) * 2) = val[tr * 4 + slot];
+                }
+              }
+            }
+          }
+        }
         if constexpr (Gm::kFp8) {
-          const float r = vref > 0.f ? vs[c >> 4] / vref : 0.f;
-          wa *= r;
-          wb *= r;
+          if (r < 4) {
+            const bool ok = (mask >> r) & 1;
+            const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + r * Gm::kSide);
+            tile_sk[(t & 1) * 4 + r] = ok ? sc[0] : 0.f;
+            tile_sv[(t & 1) * 4 + r] = ok ? sc[1] : 0.f;
+          }
         }
-        pk[c >> 1] = pack_f32x2(wa, wb, kBfMma);
-        if constexpr (Gm::kSplitP)
-          pl[c >> 1] = pack_f32x2(wa - unpack_lo(pk[c >> 1], kBfMma), wb - unpack_hi(pk[c >> 1], kBfMma), kBfMma);
       }
-      l += rs;
+      if (r == 0) tile_mask[t & 1] = mask;
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+      compute_sync();
+      // a raw stage is free as soon as it is dequantized
+      if constexpr (!Gm::k16)
+        if (r == 0) mbar_arrive(&bar_empty[s]);
+      return true;
+    };
+
+    // ---- MMA issue (thread 0) ----
+    auto issue_s = [&](int t) {
+      tc::fence_after_sync();
+      const uint32_t d = tmem + D + 64 * (t & 1);
+      const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
+      const uint32_t qa = smem_u32(sQ), ka = smem_u32(kop);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+        const uint64_t bd = tc::sw128_desc(ka + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+        tc::mma_ss(d, a, bd, kIdescS, kk > 0);
+      }
+      tc::commit(&bar_s[t & 1]);
+    };
+    auto issue_pv = [&](int t, bool first) {
+      tc::fence_after_sync();
+      const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
+                                   : sVop + (t % 3) * Gm::kOpBytes;
+      const uint32_t pa = smem_u32(sP), va = smem_u32(vop);
+#pragma unroll
+      for (int kk = 0; kk < kN / 16; ++kk) {
+        const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
+        tc::mma_ss(tmem, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
+        if constexpr (Gm::kSplitP)
+          tc::mma_ss(tmem, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
+      }
+      tc::commit(bar_pv);
+      // a 16-bit stage holds the operands themselves: free once S(t) and PV(t) are done
+      if constexpr (Gm::k16) tc::commit(&bar_empty[t % kStages]);
+    };
+
+    // ---- main loop ----
+    float m = -INFINITY, l = 0.f, vref = 0.f;
+    int pv_done = 0;  // PV products issued so far
+    if (!prepare(0)) aborted = true;
+    else {
+      if (r == 0) issue_s(0);
+      n_s = 1;
     }
 
-    // PV(t-1) must be done before O is rescaled or P is overwritten
-    if (t > 0) {
-      if (!cta_wait(bar_pv, ph_pv, p.timeout_ns)) { aborted = true; break; }
-      ph_pv ^= 1u;
-      ++n_pv_waited;
+    for (int t = 0; t < T && !aborted; ++t) {
+      if (t + 1 < T) {
+        if (!prepare(t + 1)) { aborted = true; break; }
+        if (r == 0) issue_s(t + 1);
+        ++n_s;
+      }
+      if (!compute_all(mbar_wait_bounded(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns))) {
+        aborted = true;
+        break;
+      }
+      ph_s ^= 1u << (t & 1);
+      ++n_s_waited;
       tc::fence_after_sync();
+
+      // scores of this row
+      uint32_t sv[64];
+      {
+        uint32_t a[32], c2[32];
+        tc::tmem_ld32(t_row + D + 64 * (t & 1), a);
+        tc::tmem_ld32(t_row + D + 64 * (t & 1) + 32, c2);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          sv[i] = a[i];
+          sv[32 + i] = c2[i];
+        }
+      }
+      const int mask = tile_mask[t & 1];
+      // no column of this tile is masked for any row: all 4 blocks valid and the
+      // tile ends at or before the first row's position (rows past the chunk
+      // keep a zero query and are never stored)
+      const bool full = mask == 0xF && t * kN + kN - 1 <= pos0 + i0;
+      float vs[4] = {1.f, 1.f, 1.f, 1.f};
+      float xs[64];  // FP8: scores in log2 units; otherwise raw scores (scale applied in the exponent)
+      if constexpr (Gm::kFp8) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float cj = p.scale_log2 * tile_sk[(t & 1) * 4 + j];
+          vs[j] = tile_sv[(t & 1) * 4 + j];
+#pragma unroll
+          for (int c = 16 * j; c < 16 * j + 16; ++c) xs[c] = __uint_as_float(sv[c]) * cj;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) xs[c] = __uint_as_float(sv[c]);
+      }
+      if (!full) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (t * kN + c > my_pos || !((mask >> (c >> 4)) & 1) || !row_ok) xs[c] = -INFINITY;
+      }
+      float mx;
+      {
+        float mp[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mp[i] = xs[i];
+#pragma unroll
+        for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], xs[c]);
+        mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        if constexpr (!Gm::kFp8) mx *= p.scale_log2;  // -inf stays -inf (the scale is positive)
+      }
+      float fm = 1.f;  // rescale of l and O for a larger row max
+      if (mx > m + kLazy) {
+        fm = ex2(m - mx);  // 0 when m was -inf
+        m = mx;
+      }
+      float fv = 1.f;  // FP8: O moves to units of a larger V scale (same on every thread)
+      if constexpr (Gm::kFp8) {
+        float svm = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if ((mask >> j) & 1) svm = fmaxf(svm, vs[j]);
+        if (svm > vref) {
+          fv = vref / svm;
+          vref = svm;
+        }
+      }
+      l *= fm;
+      const float fo = fm * fv;
+      const float mu = (m == -INFINITY) ? 0.f : m;  // masked entries are -inf and give 0
+      uint32_t pk[32], pl[32];
+      {
+        float rp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        float vr[4] = {1.f, 1.f, 1.f, 1.f};
+        if constexpr (Gm::kFp8) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) vr[j] = vref > 0.f ? vs[j] / vref : 0.f;
+        }
+#pragma unroll
+        for (int c = 0; c < 64; c += 2) {
+          float pa, pb;
+          if constexpr (Gm::kFp8) {
+            pa = ex2(xs[c] - mu);
+            pb = ex2(xs[c + 1] - mu);
+          } else {
+            pa = ex2(fmaf(xs[c], p.scale_log2, -mu));
+            pb = ex2(fmaf(xs[c + 1], p.scale_log2, -mu));
+          }
+          rp[(c >> 1) & 7] += pa + pb;
+          float wa = pa, wb = pb;
+          if constexpr (Gm::kFp8) {
+            wa *= vr[c >> 4];
+            wb *= vr[c >> 4];
+          }
+          pk[c >> 1] = pack_f32x2(wa, wb, kBfMma);
+          if constexpr (Gm::kSplitP)
+            pl[c >> 1] = pack_f32x2(wa - unpack_lo(pk[c >> 1], kBfMma), wb - unpack_hi(pk[c >> 1], kBfMma), kBfMma);
+        }
+        l += ((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7]));
+      }
+
+      // PV(t-1) must be done before O is rescaled or P is overwritten
+      if (t > 0) {
+        if (!compute_all(mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns))) {
+          aborted = true;
+          break;
+        }
+        ph_pv ^= 1u;
+        ++n_pv_waited;
+        tc::fence_after_sync();
+      }
+      if (pv_done > 0 && __any_sync(kFull, fo != 1.f)) {
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tc::tmem_ld32(t_row + c0, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
+          tc::tmem_st32(t_row + c0, o);
+        }
+      }
+      // P row -> shared memory (K-major operand, 128-byte swizzle)
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        *reinterpret_cast<uint4*>(sP + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        if constexpr (Gm::kSplitP)
+          *reinterpret_cast<uint4*>(sP + Gm::kPBytes + r * 128 + ((c ^ (r & 7)) << 4)) =
+              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+      }
+      tc::fence_smem_to_async();
+      tc::fence_before_sync();
+      compute_sync();
+      if (r == 0) issue_pv(t, pv_done == 0);
+      ++pv_done;
     }
-    if (pv_done > 0 && __any_sync(kFull, fo != 1.f)) {
+
+    if (!aborted && pv_done > 0) {
+      if (!compute_all(mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns))) aborted = true;
+      else {
+        ph_pv ^= 1u;
+        ++n_pv_waited;
+      }
+    }
+    if (aborted) {
+      if (r == 0) {
+        *abort_flag = 1;
+        raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+      }
+      // let products still in flight finish (each wait bounded)
+      for (int k = n_s_waited; k < n_s; ++k)
+        (void)mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.timeout_ns);
+      for (int k = n_pv_waited; k < pv_done; ++k)
+        (void)mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.timeout_ns);
+    } else {
+      tc::fence_after_sync();
+      const float inv = l > 0.f ? (Gm::kFp8 ? vref : 1.f) / l : 0.f;
+      uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + orow * 2;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
         tc::tmem_ld32(t_row + c0, o);
+        if (row_ok) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fo);
-        tc::tmem_st32(t_row + c0, o);
-      }
-    }
-    // P row -> shared memory (K-major operand, 128-byte swizzle)
+          for (int k = 0; k < 4; ++k) {
+            uint32_t w[4];
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      *reinterpret_cast<uint4*>(sP + tid * 128 + ((c ^ (tid & 7)) << 4)) =
-          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      if constexpr (Gm::kSplitP)
-        *reinterpret_cast<uint4*>(sP + Gm::kPBytes + tid * 128 + ((c ^ (tid & 7)) << 4)) =
-            make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-    }
-    tc::fence_smem_to_async();
-    tc::fence_before_sync();
-    __syncthreads();
-    if (tid == 0) {
-      issue_pv(t, pv_done == 0);
-      if (t + 2 < T) issue(t + 2);
-    }
-    ++pv_done;
-    if (t + 2 < T) ++n_issued;
-  }
-
-  if (!aborted && pv_done > 0) {
-    if (!cta_wait(bar_pv, ph_pv, p.timeout_ns)) aborted = true;
-    else {
-      ph_pv ^= 1u;
-      ++n_pv_waited;
-    }
-  }
-  if (aborted) {
-    if (tid == 0) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
-    // let copies and products still in flight land (each wait bounded)
-    for (int k = n_prepared; k < n_issued; ++k)
-      (void)mbar_wait_bounded(&bar_tma[k % kStages], (uint32_t)(k / kStages) & 1u, p.timeout_ns);
-    for (int k = n_s_waited; k < n_s; ++k)
-      (void)mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.timeout_ns);
-    for (int k = n_pv_waited; k < pv_done; ++k)
-      (void)mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.timeout_ns);
-  } else {
-    tc::fence_after_sync();
-    const float inv = l > 0.f ? (Gm::kFp8 ? vref : 1.f) / l : 0.f;
-    uint8_t* dst = reinterpret_cast<uint8_t*>(p.out) + orow * 2;
-#pragma unroll 1
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      tc::tmem_ld32(t_row + c0, o);
-      if (row_ok) {
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint32_t w[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            w[i] = pack_f32x2(__uint_as_float(o[8 * k + 2 * i]) * inv, __uint_as_float(o[8 * k + 2 * i + 1]) * inv,
-                              QBF16);
-          *reinterpret_cast<uint4*>(dst + (c0 + 8 * k) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int i = 0; i < 4; ++i)
+              w[i] = pack_f32x2(__uint_as_float(o[8 * k + 2 * i]) * inv,
+                                __uint_as_float(o[8 * k + 2 * i + 1]) * inv, QBF16);
+            *reinterpret_cast<uint4*>(dst + (c0 + 8 * k) * 2) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
     }
   }
   tc::fence_before_sync();
   __syncthreads();
+  if (tid == 0) {
+    // tiles issued but never consumed (only after a timeout) land before the CTA exits
+    const int issued = *n_issued_slot;
+    for (int k = n_prepared; k < issued; ++k)
+      (void)mbar_wait_bounded(&bar_full[k % kStages], (uint32_t)(k / kStages) & 1u, p.timeout_ns);
+  }
   if (warp == 0) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, Gm::kTmemCols);
