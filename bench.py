@@ -72,12 +72,13 @@ L2_BYTES = 126 * 1024 * 1024
 # workload on the device
 # ---------------------------------------------------------------------------
 
-def bench_spec(name: str, kv_name: str | None, batch: int | None = None, pool: int | None = None) -> W.Spec:
+def bench_spec(name: str, kv_name: str | None, batch: int | None = None, pool: int | None = None,
+               q_len: int = 1) -> W.Spec:
     """The workload as bench.py runs it; batch / pool cut it down for profiling."""
     s = W.spec(name, kv_dtype=KV_NAMES[kv_name] if kv_name else None, batch=batch)
     if pool:
         s.pool_blocks = pool
-    s.append_tokens = 1  # every step appends one token per sequence
+    s.append_tokens = q_len  # every step appends q_len tokens per sequence
     if s.kv_dtype in (W.DT_FP16, W.DT_BF16):
         s.q_dtype = s.kv_dtype  # 16-bit caches take queries of their own type
     return s
@@ -111,7 +112,7 @@ def generate_kv(s: W.Spec, seqs, threads: int = 0, ahead: int = 8):
 class Setup:
     """Cache prefilled with the workload, plus one decode step's inputs, on `device`."""
 
-    def __init__(self, s: W.Spec, device, split_blocks: int):
+    def __init__(self, s: W.Spec, device, split_blocks: int, q_len: int = 1):
         import paged_quantized_kv_cache_b200 as pq
         self.pq = pq
         self.s = s
@@ -120,6 +121,7 @@ class Setup:
         self.tab = tab
         self.lens0 = W.seq_lens(s)
         self.lens = W.decode_lens(s)
+        self.q_len = q_len
         self.cache = pq.allocate_cache(s.kv_dtype, tab.num_blocks, s.num_kv_heads, s.head_dim, device=device,
                                        fill=0xFF)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
@@ -138,16 +140,16 @@ class Setup:
                 c1 = min(L0, c0 + step)
                 sl = torch.from_numpy(W.slots_for(tab.block_tables[b], c0, c1 - c0)).to(device)
                 pq.kv_cache_write(kd[c0:c1].contiguous(), vd[c0:c1].contiguous(), sl, self.cache, self.err)
-            newk.append(k[L0:L0 + 1])
-            newv.append(v[L0:L0 + 1])
+            newk.append(k[L0:L0 + q_len])
+            newv.append(v[L0:L0 + q_len])
         torch.cuda.synchronize(device)
         if int(self.err.item()) != 0:
             raise RuntimeError("prefill raised device error bits %d" % int(self.err.item()))
         self.k_new = torch.cat(newk).contiguous()
         self.v_new = torch.cat(newv).contiguous()
-        self.slots_new = np.array([W.slots_for(tab.block_tables[b], int(self.lens0[b]), 1)[0]
-                                   for b in range(s.batch)], np.int32)
-        self.q = W.query(s)
+        self.slots_new = np.concatenate([W.slots_for(tab.block_tables[b], int(self.lens0[b]), q_len)
+                                         for b in range(s.batch)]).astype(np.int32)
+        self.q = W.query(s) if q_len == 1 else W.multi_query(s, q_len)
         self.split_blocks = split_blocks
         self.scale = W.softmax_scale(s)
         # The step's inputs (q, new k / v, slots, block tables, lengths) live in
@@ -171,15 +173,20 @@ class Setup:
         self.d_slots, self.d_bt, self.d_lens = views["slots"], views["bt"], views["lens"]
         self.h2d_bytes = sum(t.numel() * t.element_size() for _, t in parts)
         self.d_out = torch.empty_like(self.d_q)
-        self.ws = pq.decode_workspace(s.batch, s.num_q_heads, s.num_kv_heads, s.head_dim, tab.max_blocks,
-                                      split_blocks, device=device)
+        self.ws = pq.decode_workspace(s.batch, s.num_q_heads * q_len, s.num_kv_heads, s.head_dim,
+                                      tab.max_blocks, split_blocks, device=device)
 
     def write(self):
         self.pq.kv_cache_write(self.d_k, self.d_v, self.d_slots, self.cache, self.err)
 
     def decode(self):
-        self.pq.paged_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale, self.d_out,
-                                       self.ws, self.err, split_blocks=self.split_blocks)
+        if self.q_len == 1:
+            self.pq.paged_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale, self.d_out,
+                                           self.ws, self.err, split_blocks=self.split_blocks)
+        else:
+            self.pq.paged_multi_query_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale,
+                                                       self.d_out, self.ws, self.err,
+                                                       split_blocks=self.split_blocks)
 
     def unique_tokens(self) -> int:
         s = self.s
@@ -191,7 +198,7 @@ class Setup:
     def step_bytes(self) -> dict:
         s = self.s
         kv = self.unique_tokens() * per_token_bytes(s)
-        qo = 2 * s.batch * s.num_q_heads * s.head_dim * 2
+        qo = 2 * s.batch * self.q_len * s.num_q_heads * s.head_dim * 2
         tables = int(sum(W.nblocks(int(L)) for L in self.lens)) * 4 + s.batch * 4
         return {"kv": kv, "q_out": qo, "tables": tables, "decode_total": kv + qo + tables}
 
@@ -434,7 +441,9 @@ def run_reference(args) -> None:
 
 def config_dict(args, s: W.Spec, st: Setup | None) -> dict:
     d = {"workload": args.workload + ": " + DESCR[args.workload] + "; KV " + DT_LABEL[s.kv_dtype] +
-         "; step = append 1 token per sequence + paged decode", "batch": s.batch,
+         ("; step = append 1 token per sequence + paged decode" if args.q_len == 1 else
+          "; step = append %d tokens per sequence + multi-query decode verifying them (speculative decoding)"
+          % args.q_len), "batch": s.batch, "q_len": args.q_len,
          "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
          "block_size": 16, "kv_dtype": DT_LABEL[s.kv_dtype], "split_blocks": args.split_blocks,
          "parallelism": "replicas (one independent batch per GPU)"}
@@ -462,8 +471,8 @@ def run_ours(args) -> None:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    s = bench_spec(args.workload, args.kv_dtype, args.batch, args.pool_blocks)
-    st = Setup(s, device, args.split_blocks)
+    s = bench_spec(args.workload, args.kv_dtype, args.batch, args.pool_blocks, args.q_len)
+    st = Setup(s, device, args.split_blocks, args.q_len)
     stream = torch.cuda.current_stream(device)
 
     for _ in range(max(args.warmup, 3)):
@@ -499,7 +508,7 @@ def run_ours(args) -> None:
 
     b = st.step_bytes()
     value = b["kv"] * world / (ms_step * 1e-3) / 1e9
-    tok_s = s.batch * world / (ms_step * 1e-3)
+    tok_s = s.batch * args.q_len * world / (ms_step * 1e-3)
     peaks = measured_peaks()
     achieved = b["decode_total"] / (dec_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -512,7 +521,7 @@ def run_ours(args) -> None:
 
     if rank == 0:
         cpu = None
-        if world == 1 and not args.no_cpu_baseline:
+        if world == 1 and not args.no_cpu_baseline and args.q_len == 1:
             cpu = oracle_baseline(s, args.cpu_budget, args.ref_seqs)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
@@ -898,6 +907,8 @@ def main():
     ap.add_argument("--ref-seqs", type=int, default=None, help="sequences in the oracle sample")
     ap.add_argument("--op", choices=["decode", "copy_blocks", "swap", "prefill"], default="decode")
     ap.add_argument("--op-blocks", type=int, default=4096, help="blocks moved per step (--op copy_blocks|swap)")
+    ap.add_argument("--q-len", type=int, default=1,
+                    help="query tokens per sequence and step (> 1: multi-query decode, speculative verification)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -18,7 +18,8 @@
  *        "Prefix caching" and "Automatic prefix caching" (requests with a
  *        common prompt prefix reuse its KV blocks), "Preemption support"
  *        (swapping KV cache blocks out to CPU RAM), "CPU offloading" and
- *        "Chunked prefill" (long prompts processed in chunks).
+ *        "Chunked prefill" (long prompts processed in chunks) and "Speculative
+ *        decoding" (the target model verifies several proposed tokens at once).
  * Number formats follow the public OCP 8-bit Floating Point Specification
  * (OFP8: E4M3 "fn" with max 448 and no infinities, E5M2 with max 57344) and the
  * OCP Microscaling Formats specification (E2M1: values 0, .5, 1, 1.5, 2, 3, 4, 6).
@@ -198,6 +199,31 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
                                 float scale, int split_blocks, void* out,
                                 void* workspace, size_t workspace_bytes,
                                 int32_t* err_flag, pqkv_stream_t stream);
+
+/*
+ * Multi-query decode for speculative verification ([P3] "Speculative
+ * decoding": the target model verifies several proposed tokens in one pass).
+ * Each sequence has q_len query tokens, its last q_len positions (their K/V are
+ * written to the cache first and seq_lens[b] counts them): token i sits at
+ * position seq_lens[b] - q_len + i and attends to positions 0..that one. q and
+ * out are [batch][q_len][num_q_heads][head_dim] (device, contiguous). The
+ * decode kernels take the q_len x (num_q_heads / num_kv_heads) query rows of a
+ * KV head as the columns of one tensor-core tile, so that product must be at
+ * most 8 (longer chunks: pqkv_paged_prefill_attention). workspace: at least
+ * pqkv_decode_workspace_bytes(batch, num_q_heads * q_len, num_kv_heads,
+ * head_dim, max_blocks_per_seq, split_blocks) bytes. A sequence with
+ * 0 < seq_lens[b] < q_len gets zero rows and PQKV_DEVERR_SEQ_LEN. q_len = 1 is
+ * pqkv_paged_decode_attention. Other arguments, results and errors as there.
+ */
+int pqkv_paged_multi_query_decode_attention(const void* q, int q_dtype, int batch, int q_len,
+                                            int num_q_heads, const void* cache, const void* scales,
+                                            const void* outliers_idx, const void* outliers_val,
+                                            int kv_dtype, int num_blocks, int num_kv_heads,
+                                            int head_dim, const int32_t* block_tables,
+                                            int max_blocks_per_seq, const int32_t* seq_lens,
+                                            float scale, int split_blocks, void* out,
+                                            void* workspace, size_t workspace_bytes,
+                                            int32_t* err_flag, pqkv_stream_t stream);
 
 /*
  * pqkv_paged_decode_attention without a workspace argument, for callers that

@@ -38,6 +38,7 @@ EXPORTS = (
     "pqkv_paged_decode_attention_noalloc", "pqkv_pool_num_evictable", "pqkv_pool_num_cached",
     "pqkv_pool_prefix_lookup", "pqkv_pool_prefix_insert", "pqkv_pool_cow", "pqkv_copy_blocks",
     "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in", "pqkv_paged_prefill_attention",
+    "pqkv_paged_multi_query_decode_attention",
 )
 
 
@@ -83,6 +84,8 @@ def _load() -> ctypes.CDLL:
         "pqkv_swap_in": (I, [P, P, P, P, I, I, I, I, P, I, P, P, P]),
         "pqkv_paged_prefill_attention": (I, [P, I, I, I, I, P, P, P, P, P, I, I, I, I, P, I, P, ctypes.c_float,
                                              P, P, P]),
+        "pqkv_paged_multi_query_decode_attention": (I, [P, I, I, I, I, P, P, P, P, I, I, I, I, P, I, P,
+                                                        ctypes.c_float, I, P, P, Z, P, P]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -238,6 +241,30 @@ def paged_decode_attention(q: torch.Tensor, cache: KVCache, block_tables: torch.
         _dev_ptr(out, "out"), _dev_ptr(workspace, "workspace"), workspace.numel(),
         _dev_ptr(err_flag, "err_flag"), _stream_handle(stream, q.device))
     _check("pqkv_paged_decode_attention", st)
+
+
+def paged_multi_query_decode_attention(q: torch.Tensor, cache: KVCache, block_tables: torch.Tensor,
+                                      seq_lens: torch.Tensor, scale: float, out: torch.Tensor,
+                                      workspace: torch.Tensor, err_flag: torch.Tensor, split_blocks: int = 0,
+                                      stream=None) -> None:
+    """pqkv_paged_multi_query_decode_attention: q, out [B][q_len][Hq][D] (each sequence's last q_len
+    positions); workspace from decode_workspace(B, Hq * q_len, ...)."""
+    B, k, Hq, D = q.shape
+    if out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B][max_blocks_per_seq]")
+    if seq_lens.dtype != torch.int32 or seq_lens.numel() != B:
+        raise ValueError("seq_lens must be int32 [B]")
+    st = _lib.pqkv_paged_multi_query_decode_attention(
+        _dev_ptr(q, "q"), _dt_of(q, "q"), B, k, Hq, _dev_ptr(cache.cache, "cache"),
+        _dev_ptr(cache.scales, "scales"), _dev_ptr(cache.outliers_idx, "outliers_idx"),
+        _dev_ptr(cache.outliers_val, "outliers_val"), cache.kv_dtype, cache.num_blocks,
+        cache.num_kv_heads, cache.head_dim, _dev_ptr(block_tables, "block_tables"),
+        block_tables.shape[1], _dev_ptr(seq_lens, "seq_lens"), ctypes.c_float(scale), split_blocks,
+        _dev_ptr(out, "out"), _dev_ptr(workspace, "workspace"), workspace.numel(),
+        _dev_ptr(err_flag, "err_flag"), _stream_handle(stream, q.device))
+    _check("pqkv_paged_multi_query_decode_attention", st)
 
 
 def paged_prefill_attention(q: torch.Tensor, cu_q_lens: torch.Tensor, max_q_len: int, cache: KVCache,

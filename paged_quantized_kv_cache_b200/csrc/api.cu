@@ -214,16 +214,16 @@ int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_str
              : PQKV_ERR_CUDA;
 }
 
-int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads, const void* cache,
-                                const void* scales, const void* outliers_idx, const void* outliers_val,
-                                int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
-                                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
-                                float scale, int split_blocks, void* out, void* workspace,
-                                size_t workspace_bytes, int32_t* err_flag, pqkv_stream_t stream) {
+static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num_q_heads, const void* cache,
+                       const void* scales, const void* outliers_idx, const void* outliers_val, int kv_dtype,
+                       int num_blocks, int num_kv_heads, int head_dim, const int32_t* block_tables,
+                       int max_blocks_per_seq, const int32_t* seq_lens, float scale, int split_blocks, void* out,
+                       void* workspace, size_t workspace_bytes, int32_t* err_flag, pqkv_stream_t stream) {
   if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
   if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
   if (batch < 0 || batch > PQKV_MAX_BATCH || num_kv_heads < 1 || num_q_heads < 1 ||
-      num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > 8 || (head_dim != 64 && head_dim != 128) ||
+      num_q_heads % num_kv_heads != 0 || q_len < 1 || (int64_t)(num_q_heads / num_kv_heads) * q_len > 8 ||
+      (head_dim != 64 && head_dim != 128) ||
       num_blocks < 1 || max_blocks_per_seq < 1 || split_blocks < 0)
     return PQKV_ERR_ARG;
   if (batch == 0) return PQKV_OK;
@@ -237,8 +237,9 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   if ((int64_t)batch * num_kv_heads * max_blocks_per_seq >= INT32_MAX ||
       (int64_t)num_blocks * num_kv_heads * 32 >= INT32_MAX)
     return PQKV_ERR_ARG;
-  const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
-                                                  split_blocks);
+  // the pieces hold one row per MMA column: q_len x (num_q_heads / num_kv_heads)
+  const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads * q_len, num_kv_heads, head_dim,
+                                                  max_blocks_per_seq, split_blocks);
   if (need == 0 || workspace_bytes < need) return PQKV_ERR_ARG;
   DeviceInfo di;
   if (!device_info(di)) return PQKV_ERR_CUDA;
@@ -258,7 +259,9 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
-  p.G = num_q_heads / num_kv_heads;
+  p.Gh = num_q_heads / num_kv_heads;
+  p.k = q_len;
+  p.G = p.Gh * q_len;
   p.nb = num_blocks;
   p.maxblk = max_blocks_per_seq;
   p.split_blocks = split_blocks;
@@ -276,12 +279,37 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
   mp.Hq = num_q_heads;
   mp.Hkv = num_kv_heads;
   mp.G = p.G;
+  mp.k = p.k;
+  mp.Gh = p.Gh;
   mp.maxblk = max_blocks_per_seq;
   mp.warps = di.sms * decode_warps(kv_dtype, head_dim);
   mp.split_blocks = split_blocks;
   mp.slot_floats = p.slot_floats;
   e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads, const void* cache,
+                                const void* scales, const void* outliers_idx, const void* outliers_val,
+                                int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                                const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                                float scale, int split_blocks, void* out, void* workspace,
+                                size_t workspace_bytes, int32_t* err_flag, pqkv_stream_t stream) {
+  return decode_impl(q, q_dtype, batch, 1, num_q_heads, cache, scales, outliers_idx, outliers_val, kv_dtype,
+                     num_blocks, num_kv_heads, head_dim, block_tables, max_blocks_per_seq, seq_lens, scale,
+                     split_blocks, out, workspace, workspace_bytes, err_flag, stream);
+}
+
+int pqkv_paged_multi_query_decode_attention(const void* q, int q_dtype, int batch, int q_len, int num_q_heads,
+                                            const void* cache, const void* scales, const void* outliers_idx,
+                                            const void* outliers_val, int kv_dtype, int num_blocks,
+                                            int num_kv_heads, int head_dim, const int32_t* block_tables,
+                                            int max_blocks_per_seq, const int32_t* seq_lens, float scale,
+                                            int split_blocks, void* out, void* workspace, size_t workspace_bytes,
+                                            int32_t* err_flag, pqkv_stream_t stream) {
+  return decode_impl(q, q_dtype, batch, q_len, num_q_heads, cache, scales, outliers_idx, outliers_val, kv_dtype,
+                     num_blocks, num_kv_heads, head_dim, block_tables, max_blocks_per_seq, seq_lens, scale,
+                     split_blocks, out, workspace, workspace_bytes, err_flag, stream);
 }
 
 size_t pqkv_block_record_bytes(int kv_dtype, int num_kv_heads, int head_dim) {

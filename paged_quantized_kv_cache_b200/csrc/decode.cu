@@ -37,6 +37,12 @@ __device__ __forceinline__ float ex2(float x) {
   return r;
 }
 
+// Element offset of the q / out row of MMA column c of KV head h of sequence
+// b: q and out are [B][k][Hq][D], column c = (token c / Gh, head c % Gh).
+__device__ __forceinline__ size_t col_row(int b, int h, int c, int k, int Gh, int Hq, int D) {
+  return ((size_t)(b * k + c / Gh) * Hq + (size_t)h * Gh + c % Gh) * D;
+}
+
 template <bool QBF16>
 __device__ __forceinline__ float q_at(const void* q, size_t i) {
   if constexpr (QBF16)
@@ -361,7 +367,7 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     int local = 0;
     for (int i = lo; i < hi; ++i) {
       const int L = p.seq_lens[i];
-      local += (L < 0 || L > lim) ? 0 : (L + kBlock - 1) / kBlock;
+      local += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
     }
     int incl = local;
 #pragma unroll
@@ -376,7 +382,7 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     if (tid == 0) P[0] = 0;
     for (int i = lo; i < hi; ++i) {
       const int L = p.seq_lens[i];
-      run += (L < 0 || L > lim) ? 0 : (L + kBlock - 1) / kBlock;
+      run += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
       P[i + 1] = run;
     }
     __syncthreads();
@@ -384,9 +390,9 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
   const int T = p.Hkv * P[p.B];
   const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + p.warps - 1) / p.warps);
   const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (wid >= (long)p.B * p.Hq) return;
-  const int b = (int)(wid / p.Hq), hq = (int)(wid % p.Hq);
-  const int h = hq / p.G, n = hq % p.G;
+  if (wid >= (long)p.B * p.Hkv * p.G) return;
+  const int b = (int)(wid / ((long)p.Hkv * p.G));
+  const int h = (int)((wid / p.G) % p.Hkv), n = (int)(wid % p.G);
   const int nblk = P[b + 1] - P[b];
   if (nblk == 0) return;
   const int s0 = p.Hkv * P[b] + h * nblk;
@@ -451,7 +457,7 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  const size_t orow = ((size_t)b * p.Hq + hq) * D + lane * DPL;
+  const size_t orow = col_row(b, h, n, p.k, p.Gh, p.Hq, D) + lane * DPL;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
 }
@@ -480,6 +486,10 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int B = p.B, Hkv = p.Hkv, G = p.G, Hq = p.Hq;
   const int g = lane >> 2, qd = lane & 3;
+  // multi-query: positions at the end of the sequence hidden from this lane's
+  // two columns (query token c / Gh of k sits k - 1 - c / Gh before the end)
+  const int hid0 = (2 * qd < G) ? p.k - 1 - (2 * qd) / p.Gh : 0;
+  const int hid1 = (2 * qd + 1 < G) ? p.k - 1 - (2 * qd + 1) / p.Gh : 0;
   uint64_t* wbar = bars + warp * NS;
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
@@ -504,7 +514,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     int local = 0;
     for (int i = lo; i < hi; ++i) {
       const int L = p.seq_lens[i];
-      const bool bad = (L < 0 || L > lim);
+      const bool bad = (L < 0 || L > lim || (L > 0 && L < p.k));
       if (bad && blockIdx.x == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
       local += bad ? 0 : (L + kBlock - 1) / kBlock;
     }
@@ -521,7 +531,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     if (tid == 0) P[0] = 0;
     for (int i = lo; i < hi; ++i) {
       const int L = p.seq_lens[i];
-      const bool bad = (L < 0 || L > lim);
+      const bool bad = (L < 0 || L > lim || (L > 0 && L < p.k));
       run += bad ? 0 : (L + kBlock - 1) / kBlock;
       P[i + 1] = run;
     }
@@ -531,7 +541,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   // ---- sequences without blocks (empty or rejected): zero output rows ----
   for (int b = blockIdx.x; b < B; b += gridDim.x) {
     if (P[b + 1] != P[b]) continue;
-    for (int i = tid; i < Hq * D; i += blockDim.x) store_out<QBF16>(p.out, (size_t)b * Hq * D + i, 0.f);
+    for (int i = tid; i < p.k * Hq * D; i += blockDim.x) store_out<QBF16>(p.out, (size_t)b * p.k * Hq * D + i, 0.f);
   }
 
   const int T = Hkv * P[B];
@@ -635,8 +645,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       vref = 0.f;
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      const size_t qrow = ((size_t)b * Hq + (size_t)h * G + g) * D;
       const bool has = g < G;
+      const size_t qrow = has ? col_row(b, h, g, p.k, p.Gh, Hq, D) : 0;
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
         if constexpr (Gm::k16) {
@@ -664,7 +674,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         __syncwarp();
         for (int i = lane; i < 8 * D; i += 32) {
           const int n = i / D;
-          const float v = (n < G) ? q_at<QBF16>(p.q, ((size_t)b * Hq + (size_t)h * G + n) * D + (i % D)) : 0.f;
+          const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.Gh, Hq, D) + (i % D)) : 0.f;
           wq[n * Gm::kQStride + i % D] = __half_as_ushort(__float2half_rn(v));
         }
         __syncwarp();
@@ -695,17 +705,18 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       if (!started_before && !ends_after) {
         const float i0 = lt0 > 0.f ? vs / lt0 : 0.f;
         const float i1 = lt1 > 0.f ? vs / lt1 : 0.f;
-        const size_t ob = ((size_t)b * Hq + (size_t)h * G) * D;
+        const size_t ob0 = n0 < G ? col_row(b, h, n0, p.k, p.Gh, Hq, D) : 0;
+        const size_t ob1 = n1 < G ? col_row(b, h, n1, p.k, p.Gh, Hq, D) : 0;
 #pragma unroll
         for (int mt = 0; mt < KT; ++mt) {
           const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
           if (n0 < G) {
-            store_out<QBF16>(p.out, ob + (size_t)n0 * D + da, acc[mt][0] * i0);
-            store_out<QBF16>(p.out, ob + (size_t)n0 * D + db, acc[mt][2] * i0);
+            store_out<QBF16>(p.out, ob0 + da, acc[mt][0] * i0);
+            store_out<QBF16>(p.out, ob0 + db, acc[mt][2] * i0);
           }
           if (n1 < G) {
-            store_out<QBF16>(p.out, ob + (size_t)n1 * D + da, acc[mt][1] * i1);
-            store_out<QBF16>(p.out, ob + (size_t)n1 * D + db, acc[mt][3] * i1);
+            store_out<QBF16>(p.out, ob1 + da, acc[mt][1] * i1);
+            store_out<QBF16>(p.out, ob1 + db, acc[mt][3] * i1);
           }
         }
         return;
@@ -759,8 +770,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       }
       const bool useA = !((skip >> sA) & 1u);
       const bool useB = (n2 == 2) && !((skip >> sB) & 1u);
-      const int validA = min(kBlock, Lb - kBlock * j);
-      const int validB = min(kBlock, Lb - kBlock * (j + 1));
+      const int remA = Lb - kBlock * j, remB = remA - kBlock;  // tokens left from each block on
+      const int validA = min(kBlock, remA), validB = min(kBlock, remB);
       const uint32_t tbA = smem_u32(wtile + sA * Gm::kTile), tbB = smem_u32(wtile + sB * Gm::kTile);
       const uint8_t* sdA = wside + sA * Gm::kSideStride;
       const uint8_t* sdB = wside + sB * Gm::kSideStride;
@@ -779,10 +790,15 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       const float mA = p.scale_log2 * skA, mB = p.scale_log2 * skB;
       float xA0 = scA[0] * mA, xA1 = scA[1] * mA, xA2 = scA[2] * mA, xA3 = scA[3] * mA;
       float xB0 = scB[0] * mB, xB1 = scB[1] * mB, xB2 = scB[2] * mB, xB3 = scB[3] * mB;
-      if (!useA || g >= validA) xA0 = xA1 = kNegInf;
-      if (!useA || g + 8 >= validA) xA2 = xA3 = kNegInf;
-      if (!useB || g >= validB) xB0 = xB1 = kNegInf;
-      if (!useB || g + 8 >= validB) xB2 = xB3 = kNegInf;
+      // column n sees the tokens before the last hid_n ones (0 for one query token)
+      if (!useA || g >= remA - hid0) xA0 = kNegInf;
+      if (!useA || g >= remA - hid1) xA1 = kNegInf;
+      if (!useA || g + 8 >= remA - hid0) xA2 = kNegInf;
+      if (!useA || g + 8 >= remA - hid1) xA3 = kNegInf;
+      if (!useB || g >= remB - hid0) xB0 = kNegInf;
+      if (!useB || g >= remB - hid1) xB1 = kNegInf;
+      if (!useB || g + 8 >= remB - hid0) xB2 = kNegInf;
+      if (!useB || g + 8 >= remB - hid1) xB3 = kNegInf;
       float bm0 = fmaxf(fmaxf(xA0, xA2), fmaxf(xB0, xB2));
       float bm1 = fmaxf(fmaxf(xA1, xA3), fmaxf(xB1, xB3));
 #pragma unroll
@@ -932,7 +948,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
 // stream as a programmatic dependent (its launch overlaps the decode's tail;
 // griddepcontrol.wait inside it orders it after the decode grid).
 cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st) {
-  const long warps = (long)p.B * p.Hq;
+  const long warps = (long)p.B * p.Hkv * p.G;  // one per (sequence, KV head, column)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
   cfg.blockDim = dim3(128);

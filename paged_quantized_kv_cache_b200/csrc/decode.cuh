@@ -44,7 +44,11 @@ struct DecodeParams {
   const int32_t* seq_lens;      // [B]
   int32_t* err;
   float* partials;              // [2 * chunks][slot_floats]
+  // G = MMA columns per KV head = Gh query heads x k query tokens (column
+  // c = token c / Gh, head c % Gh); k > 1 is multi-query decode: token i of a
+  // sequence of length L sits at position L - k + i and sees positions <= it
   int B, Hq, Hkv, G, nb, maxblk;
+  int k, Gh;
   int split_blocks;
   int slot_floats;
   float scale_log2;             // softmax scale * log2(e)
@@ -56,6 +60,7 @@ struct MergeParams {
   const float* partials;
   void* out;
   int B, Hq, Hkv, G, maxblk;
+  int k, Gh;                 // as in DecodeParams
   int warps;         // warps of the decode grid (its balanced chunk length depends on it)
   int split_blocks;
   int slot_floats;

@@ -88,11 +88,12 @@ def spec(name: str, kv_dtype: Optional[int] = None, batch: Optional[int] = None)
 
 def _streams(s: Spec) -> List[np.random.SeedSequence]:
     # children 0..B-1: per-sequence K/V; B: lengths; B+1: physical ids; B+2: q;
-    # B+3: shared prefix K/V; B+4: outlier channel choice. The number of
-    # children depends only on the full batch of the named workload so that a
-    # batch cut keeps every sequence's stream.
+    # B+3: shared prefix K/V; B+4: outlier channel choice; B+5: multi-token q.
+    # The number of children depends only on the full batch of the named
+    # workload so that a batch cut keeps every sequence's stream (a child's
+    # stream depends on its index only).
     full = spec(s.name).batch
-    return np.random.SeedSequence(s.seed).spawn(full + 5)
+    return np.random.SeedSequence(s.seed).spawn(full + 6)
 
 
 def seq_lens(s: Spec) -> np.ndarray:
@@ -214,6 +215,15 @@ def input_dtype(s: Spec) -> int:
     if s.kv_dtype in (DT_FP16, DT_BF16):
         return s.kv_dtype
     return s.q_dtype
+
+
+def multi_query(s: Spec, q_len: int) -> torch.Tensor:
+    """q [B][q_len][Hq][D] ~ N(0,1) rounded to the query dtype (CPU), for the
+    multi-query (speculative verification) step; its own stream."""
+    full = spec(s.name).batch
+    rng = np.random.Generator(np.random.PCG64(_streams(s)[full + 5]))
+    q = _normal(rng, (full, q_len, s.num_q_heads, s.head_dim))[: s.batch]
+    return torch.from_numpy(np.ascontiguousarray(q)).to(TORCH_DTYPE[s.q_dtype])
 
 
 def query(s: Spec) -> torch.Tensor:
