@@ -38,11 +38,9 @@ namespace pqkv {
 
 namespace {
 
-constexpr int kM = 128;        // rows (query token, head) per CTA
+constexpr int kM = 128;        // rows (query token, head) per warpgroup tile
 constexpr int kN = 64;         // KV tokens per tile (4 blocks)
-constexpr int kComputeThreads = 128;              // 4 warps: one row (TMEM lane) per thread
-constexpr int kThreads = kComputeThreads + 32;     // + one producer warp
-constexpr int kStages = 4;     // KV tiles in flight
+constexpr int kWG = 128;       // threads of a compute warpgroup: one row (TMEM lane) per thread
 constexpr float kLazy = 8.f;   // O is rescaled only when a row max grows by more (log2 units)
 constexpr unsigned kFull = 0xFFFFFFFFu;
 
@@ -51,8 +49,14 @@ struct PrefillGeom {
   static constexpr bool k16 = (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16);
   static constexpr bool kFp8 = (KVF == PQKV_DTYPE_FP8_E4M3 || KVF == PQKV_DTYPE_FP8_E5M2);
   static constexpr bool kFp4 = (KVF == PQKV_DTYPE_FP4_E2M1);
+  // Compute warpgroups per CTA, each on its own 128-row query tile, sharing the
+  // K/V stages: two for 16-bit caches (one issues while the other stalls), one
+  // for quantized caches (their dequantized operand tiles take the room)
+  static constexpr int NWG = k16 ? 2 : 1;
+  static constexpr int kStages = k16 ? 3 : 4;     // KV tiles in flight
+  static constexpr int kThreads = NWG * kWG + 32; // + one producer warp
   static constexpr int NB = D / 64;                // 128-byte boxes per operand row
-  static constexpr int kQBytes = NB * kM * 128;    // Q operand [box][128 rows][128 B]
+  static constexpr int kQBytes = NB * kM * 128;    // Q operand of one warpgroup [box][128 rows][128 B]
   static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
   static constexpr int kPBytes = kM * 128;         // P operand: 64 tokens (2 B) per row
   // P = P_hi + P_lo, both rounded to the operand type, keeps ~16 significant
@@ -68,15 +72,17 @@ struct PrefillGeom {
   static constexpr int kStageBytes = (kRawStage + 1023) / 1024 * 1024;
   static constexpr int kKops = k16 ? 0 : 2;        // dequantized K tiles (S of tile t-1 may still read one)
   static constexpr int kVops = k16 ? 0 : 3;        // dequantized V tiles (PV of tile t-2 may still read one)
+  static constexpr int kPSet = (kSplitP ? 2 : 1) * kPBytes;  // P operands of one warpgroup
   static constexpr int oQ = 0;
-  static constexpr int oStage = oQ + kQBytes;
+  static constexpr int oStage = oQ + NWG * kQBytes;
   static constexpr int oKop = oStage + kStages * kStageBytes;
   static constexpr int oVop = oKop + kKops * kOpBytes;
   static constexpr int oP = oVop + kVops * kOpBytes;
-  static constexpr int oMisc = oP + (kSplitP ? 2 : 1) * kPBytes;
+  static constexpr int oMisc = oP + NWG * kPSet;
   static constexpr int kMiscBytes = 256;
   static constexpr int kSmem = oMisc + kMiscBytes + 1024;  // + alignment slack
-  static constexpr uint32_t kTmemCols = 256;      // O: columns [0, D); S buffers at D and D + 64
+  // per warpgroup 256 columns: O at [0, D), S buffers at D and D + 64
+  static constexpr uint32_t kTmemCols = 256 * NWG;
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -90,17 +96,17 @@ __device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Barrier of the 128 compute threads only (named barrier 1; the producer warp
-// runs on its own).
-__device__ __forceinline__ void compute_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// The same barrier, returning whether v held on every compute thread.
-__device__ __forceinline__ bool compute_all(bool v) {
+// Barrier of the 128 threads of one compute warpgroup (named barrier 1 + wg;
+// the other warpgroup and the producer warp run on their own).
+__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
+// The same barrier, returning whether v held on every thread of the warpgroup.
+__device__ __forceinline__ bool wg_all(int wg, bool v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, 128, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v)
+      : "r"((uint32_t)v), "r"(1 + wg)
       : "memory");
   return r != 0;
 }
@@ -119,27 +125,25 @@ __device__ __forceinline__ uint32_t hmul2u(uint32_t a, __half2 s) {
 }  // namespace
 
 template <int KVF, int D, bool QBF16>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap tmap, const PrefillParams p) {
   using Gm = PrefillGeom<KVF, D>;
+  constexpr int NWG = Gm::NWG, kStages = Gm::kStages;
   constexpr bool kBfMma = (KVF == PQKV_DTYPE_BF16);  // operand type: bf16 for a bf16 cache, else f16
   constexpr uint32_t kIdescS = tc::f16_idesc(kBfMma, kM, kN, false);
   constexpr uint32_t kIdescPV = tc::f16_idesc(kBfMma, kM, D, true);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* sQ = smem + Gm::oQ;
   uint8_t* sStage = smem + Gm::oStage;
   uint8_t* sKop = smem + Gm::oKop;
   uint8_t* sVop = smem + Gm::oVop;
-  uint8_t* sP = smem + Gm::oP;
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Gm::oMisc);  // [kStages] tile landed
   uint64_t* bar_empty = bar_full + kStages;                             // [kStages] stage free again
-  uint64_t* bar_s = bar_empty + kStages;                                // [2] S(t) computed
-  uint64_t* bar_pv = bar_s + 2;                                         // [1] PV(t) computed
-  int* stage_mask = reinterpret_cast<int*>(bar_pv + 1);                 // [kStages] blocks loaded
-  int* tile_mask = stage_mask + kStages;                                // [2] blocks holding valid tokens
-  float* tile_sk = reinterpret_cast<float*>(tile_mask + 2);             // [2][4] FP8 K scales
+  uint64_t* bar_s_all = bar_empty + kStages;                            // [NWG][2] S(t) computed
+  uint64_t* bar_pv_all = bar_s_all + 2 * NWG;                           // [NWG] PV(t) computed
+  int* stage_mask = reinterpret_cast<int*>(bar_pv_all + NWG);           // [kStages] blocks loaded
+  float* tile_sk = reinterpret_cast<float*>(stage_mask + kStages);      // [2][4] FP8 K scales
   float* tile_sv = tile_sk + 8;                                         // [2][4] FP8 V scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -148,21 +152,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the chunk's K/V may come from the previous kernel
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int h = blockIdx.y;
-  const int b = blockIdx.x / p.tiles_per_seq;
-  const int mt = p.tiles_per_seq - 1 - (int)(blockIdx.x % p.tiles_per_seq);  // long tiles first
   const int G = p.G, TOK = kM / G;
+  const int ctas = (p.tiles_per_seq + NWG - 1) / NWG;  // CTAs per sequence
+  const int b = blockIdx.x / ctas;
+  const int mt0 = NWG * (ctas - 1 - (int)(blockIdx.x % ctas));  // first query tile; long ones first
   const int q0 = p.cu_q[b], qn = p.cu_q[b + 1] - q0;
   const int L = p.seq_lens[b];
-  const int i0 = mt * TOK;
-  if (i0 == 0 && h == 0 && tid == 0 && qn > p.tiles_per_seq * TOK)
+  if (mt0 == 0 && h == 0 && tid == 0 && qn > p.tiles_per_seq * TOK)
     raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
-  if (qn <= 0 || i0 >= qn) return;
-  const int r = tid & (kM - 1);  // compute thread tid = row r (the producer warp has no row)
+  if (qn <= 0 || mt0 * TOK >= qn) return;
+  const bool is_compute = tid < NWG * kWG;
+  const int wg = is_compute ? tid / kWG : 0;
+  const int r = tid % kWG;                           // row of this thread in its warpgroup's tile
+  const int i0 = (mt0 + wg) * TOK;                   // first query token of the warpgroup's tile
   const int my_i = i0 + r / G, my_n = r % G;
-  const bool row_ok = tid < kComputeThreads && my_i < qn;
+  const bool row_ok = is_compute && my_i < qn && i0 < p.tiles_per_seq * TOK;
   const size_t orow = ((size_t)(q0 + (row_ok ? my_i : 0)) * p.Hq + (size_t)h * G + my_n) * D;
   if (L < 0 || L > kBlock * p.maxblk || qn > L) {
-    if (i0 == 0 && h == 0 && tid == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
+    if (mt0 == 0 && h == 0 && tid == 0) raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);
     if (row_ok) {
       uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint8_t*>(p.out) + orow * 2);
       for (int c = 0; c < D / 8; ++c) o[c] = make_uint4(0, 0, 0, 0);
@@ -171,28 +178,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const int pos0 = L - qn;                          // position of query token 0
   const int my_pos = pos0 + my_i;                   // this row attends to [0, my_pos]
-  const int n_kv = pos0 + min(i0 + TOK, qn);        // positions the tile reads
+  // the CTA reads positions up to its last row: every warpgroup walks all its tiles
+  const int n_kv = pos0 + min(min(mt0 + NWG, p.tiles_per_seq) * TOK, qn);
   const int T = (n_kv + kN - 1) / kN;
   const int32_t* table = p.block_tables + (size_t)b * p.maxblk;
 
-  // ---- setup: tensor memory, barriers, Q tile ----
+  // ---- setup: tensor memory, barriers, Q tiles ----
   if (warp == 0) tc::tmem_alloc(tmem_slot, Gm::kTmemCols);
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1);
+      mbar_init(&bar_empty[s], NWG);
     }
-    mbar_init(&bar_s[0], 1);
-    mbar_init(&bar_s[1], 1);
-    mbar_init(bar_pv, 1);
+    for (int i = 0; i < 2 * NWG; ++i) mbar_init(&bar_s_all[i], 1);
+    for (int i = 0; i < NWG; ++i) mbar_init(&bar_pv_all[i], 1);
     *abort_flag = 0;
     *n_issued_slot = 0;
     fence_mbar_init();
   }
   if constexpr (Gm::k16)
-    if (tid == kComputeThreads) prefetch_tensormap(&tmap);
-  if (tid < kComputeThreads) {
-    // row r of Q, converted to the operand type, 16-byte chunks swizzled
+    if (tid == NWG * kWG) prefetch_tensormap(&tmap);
+  if (is_compute) {
+    // row r of the warpgroup's Q tile, converted to the operand type, 16-byte chunks swizzled
+    uint8_t* sQ = smem + Gm::oQ + wg * Gm::kQBytes;
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.q) + orow * 2);
 #pragma unroll 4
     for (int c = 0; c < D / 8; ++c) {
@@ -213,9 +221,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  int n_prepared = 0;  // KV tiles consumed by the compute warps
+  int n_prepared = 0;  // KV tiles consumed by this thread's warpgroup
 
-  if (warp == kComputeThreads / 32) {
+  if (!is_compute) {
     // ================= producer warp: KV tiles into the stage ring =================
     if (lane == 0) {
       int t = 0;
@@ -274,18 +282,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       *n_issued_slot = t;
     }
   } else {
-    // ================= compute warpgroup: one row per thread =================
-    const uint32_t t_row = tmem + ((uint32_t)(32 * warp) << 16);
+    // ================= compute warpgroup wg: one row per thread =================
+    const uint32_t t_row = tmem + 256u * wg + ((uint32_t)(32 * (warp & 3)) << 16);
+    const uint32_t t_base = tmem + 256u * wg;
+    uint64_t* bar_s = bar_s_all + 2 * wg;
+    uint64_t* bar_pv = bar_pv_all + wg;
+    uint8_t* sQ = smem + Gm::oQ + wg * Gm::kQBytes;
+    uint8_t* sP = smem + Gm::oP + wg * Gm::kPSet;
     uint32_t ph_full = 0, ph_s = 0, ph_pv = 0;  // parity bits per barrier
+    bool ok = true;                             // no wait of this thread has timed out
     bool aborted = false;
-    // operations issued and waited for (the same on every thread), so that a
-    // timeout can let the ones still in flight finish before the CTA exits
+    // operations issued and waited for (the same on every thread of the
+    // warpgroup), so that a timeout can let the ones in flight finish
     int n_s = 0, n_s_waited = 0, n_pv_waited = 0;
+    int mask_cur = 0, mask_next = 0;  // blocks of tile t / t + 1 holding data
 
-    // ---- make KV tile t's operands ready; false on a timeout ----
-    auto prepare = [&](int t) -> bool {
+    // ---- make KV tile t's operands ready; returns its block mask ----
+    auto prepare = [&](int t) -> int {
       const int s = t % kStages;
-      if (!compute_all(mbar_wait_bounded(&bar_full[s], (ph_full >> s) & 1u, p.timeout_ns))) return false;
+      ok = mbar_wait_bounded(&bar_full[s], (ph_full >> s) & 1u, p.timeout_ns) && ok;
       ph_full ^= 1u << s;
       ++n_prepared;
       const int mask = stage_mask[s];
@@ -293,24 +308,27 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* st = sStage + s * Gm::kStageBytes;
       if constexpr (Gm::k16) {
         // V rows without valid data (past the sequence, or a block not loaded)
-        // are zeroed: P is 0 there, and 0 x NaN would poison O
+        // are zeroed: P is 0 there, and 0 x NaN would poison O. Each warpgroup
+        // zeroes before its own products (the same zeros).
         if (mask != 0xF || base + kN > L) {
-          for (int u = r; u < kN * Gm::NB * 8; u += kComputeThreads) {
+          for (int u = r; u < kN * Gm::NB * 8; u += kWG) {
             const int rr = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
             if (((mask >> (rr >> 4)) & 1) && base + rr < L) continue;
             *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + rr * 128 + ((k & 7) << 4)) =
                 make_uint4(0, 0, 0, 0);
           }
+          tc::fence_smem_to_async();
+          wg_sync(wg);
         }
       } else {
         uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
         uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
         constexpr int CPR = D / 8;  // 16-byte operand chunks per row
-        for (int u = r; u < kN * CPR; u += kComputeThreads) {
+        for (int u = r; u < kN * CPR; u += kWG) {
           const int rr = u / CPR, c = u % CPR, j = rr >> 4, tr = rr & 15;
-          const bool ok = ((mask >> j) & 1) && base + rr < L;
+          const bool okr = ((mask >> j) & 1) && base + rr < L;
           uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
-          if (ok) {
+          if (okr) {
             const uint8_t* tile = st + j * Gm::kRawTile;
             if constexpr (Gm::kFp8) {
               const uint2 kc = *reinterpret_cast<const uint2*>(tile + tr * D + 8 * c);
@@ -351,51 +369,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if constexpr (Gm::kFp4) {
           // outlier channels (their codes are 0): write the fp16 values over them;
-          // thread = (block j, K|V, slot, half of the tokens)
-          compute_sync();
-          {
-            const int j = r >> 5, kv = (r >> 4) & 1, slot = (r >> 2) & 3, part = r & 3;
-            if ((mask >> j) & 1) {
-              const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
-              const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
-              if (ch < D) {
-                const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes) + kv * 64;
-                uint8_t* op = kv ? vop : kop;
-                const int c = ch >> 3;
+          // thread = (block j, K|V, slot, quarter of the tokens)
+          wg_sync(wg);
+          const int j = r >> 5, kv = (r >> 4) & 1, slot = (r >> 2) & 3, part = r & 3;
+          if ((mask >> j) & 1) {
+            const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+            const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
+            if (ch < D) {
+              const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes) + kv * 64;
+              uint8_t* op = kv ? vop : kop;
+              const int c = ch >> 3;
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                  const int tr = 4 * part + q4, rr = 16 * j + tr;
-                  if (base + rr < L)
-                    *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 +
-                                                 (((c & 7) ^ (rr & 7)) << 4) + (ch & 7) * 2) = val[tr * 4 + slot];
-                }
+              for (int q4 = 0; q4 < 4; ++q4) {
+                const int tr = 4 * part + q4, rr = 16 * j + tr;
+                if (base + rr < L)
+                  *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4) +
+                                               (ch & 7) * 2) = val[tr * 4 + slot];
               }
             }
           }
         }
         if constexpr (Gm::kFp8) {
           if (r < 4) {
-            const bool ok = (mask >> r) & 1;
+            const bool okb = (mask >> r) & 1;
             const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + r * Gm::kSide);
-            tile_sk[(t & 1) * 4 + r] = ok ? sc[0] : 0.f;
-            tile_sv[(t & 1) * 4 + r] = ok ? sc[1] : 0.f;
+            tile_sk[(t & 1) * 4 + r] = okb ? sc[0] : 0.f;
+            tile_sv[(t & 1) * 4 + r] = okb ? sc[1] : 0.f;
           }
         }
-      }
-      if (r == 0) tile_mask[t & 1] = mask;
-      tc::fence_smem_to_async();
-      tc::fence_before_sync();
-      compute_sync();
-      // a raw stage is free as soon as it is dequantized
-      if constexpr (!Gm::k16)
+        tc::fence_smem_to_async();
+        tc::fence_before_sync();
+        // the products may read the operands once every thread wrote its part;
+        // the consensus also carries timeouts
+        if (!wg_all(wg, ok)) ok = false;
+        // a raw stage is free as soon as it is dequantized
         if (r == 0) mbar_arrive(&bar_empty[s]);
-      return true;
+      }
+      return mask;
     };
 
-    // ---- MMA issue (thread 0) ----
+    // ---- MMA issue (thread 0 of the warpgroup) ----
     auto issue_s = [&](int t) {
       tc::fence_after_sync();
-      const uint32_t d = tmem + D + 64 * (t & 1);
+      const uint32_t d = t_base + D + 64 * (t & 1);
       const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
       const uint32_t qa = smem_u32(sQ), ka = smem_u32(kop);
 #pragma unroll
@@ -414,9 +430,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < kN / 16; ++kk) {
         const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
-        tc::mma_ss(tmem, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
+        tc::mma_ss(t_base, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
         if constexpr (Gm::kSplitP)
-          tc::mma_ss(tmem, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
+          tc::mma_ss(t_base, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
       }
       tc::commit(bar_pv);
       // a 16-bit stage holds the operands themselves: free once S(t) and PV(t) are done
@@ -426,22 +442,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- main loop ----
     float m = -INFINITY, l = 0.f, vref = 0.f;
     int pv_done = 0;  // PV products issued so far
-    if (!prepare(0)) aborted = true;
+    mask_next = prepare(0);
+    if (!ok) aborted = true;
     else {
       if (r == 0) issue_s(0);
       n_s = 1;
     }
 
     for (int t = 0; t < T && !aborted; ++t) {
+      mask_cur = mask_next;
       if (t + 1 < T) {
-        if (!prepare(t + 1)) { aborted = true; break; }
-        if (r == 0) issue_s(t + 1);
-        ++n_s;
+        mask_next = prepare(t + 1);
+        if (Gm::k16 ? true : ok) {
+          if (r == 0) issue_s(t + 1);
+          ++n_s;
+        } else {
+          aborted = true;
+          break;
+        }
       }
-      if (!compute_all(mbar_wait_bounded(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns))) {
-        aborted = true;
-        break;
-      }
+      ok = mbar_wait_bounded(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns) && ok;
       ph_s ^= 1u << (t & 1);
       ++n_s_waited;
       tc::fence_after_sync();
@@ -458,10 +478,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           sv[32 + i] = c2[i];
         }
       }
-      const int mask = tile_mask[t & 1];
-      // no column of this tile is masked for any row: all 4 blocks valid and the
-      // tile ends at or before the first row's position (rows past the chunk
-      // keep a zero query and are never stored)
+      const int mask = mask_cur;
+      // no column of this tile is masked for any row of the warpgroup: all 4
+      // blocks valid and the tile ends at or before the first row's position
+      // (rows past the chunk keep a zero query and are never stored)
       const bool full = mask == 0xF && t * kN + kN - 1 <= pos0 + i0;
       float vs[4] = {1.f, 1.f, 1.f, 1.f};
       float xs[64];  // FP8: scores in log2 units; otherwise raw scores (scale applied in the exponent)
@@ -544,10 +564,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
       // PV(t-1) must be done before O is rescaled or P is overwritten
       if (t > 0) {
-        if (!compute_all(mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns))) {
-          aborted = true;
-          break;
-        }
+        ok = mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns) && ok;
         ph_pv ^= 1u;
         ++n_pv_waited;
         tc::fence_after_sync();
@@ -573,13 +590,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_smem_to_async();
       tc::fence_before_sync();
-      compute_sync();
+      // one barrier per tile: P complete, S read, and no wait timed out anywhere
+      if (!wg_all(wg, ok)) {
+        aborted = true;
+        break;
+      }
       if (r == 0) issue_pv(t, pv_done == 0);
       ++pv_done;
     }
 
     if (!aborted && pv_done > 0) {
-      if (!compute_all(mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns))) aborted = true;
+      ok = mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns) && ok;
+      if (!wg_all(wg, ok)) aborted = true;
       else {
         ph_pv ^= 1u;
         ++n_pv_waited;
@@ -647,8 +669,9 @@ static cudaError_t launch_prefill_t(const CUtensorMap& tmap, const PrefillParams
     configured.fetch_or(bit);
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.B * p.tiles_per_seq), (unsigned)p.Hkv);
-  cfg.blockDim = dim3(kThreads);
+  constexpr int NWG = PrefillGeom<KVF, D>::NWG;
+  cfg.gridDim = dim3((unsigned)(p.B * ((p.tiles_per_seq + NWG - 1) / NWG)), (unsigned)p.Hkv);
+  cfg.blockDim = dim3(PrefillGeom<KVF, D>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
