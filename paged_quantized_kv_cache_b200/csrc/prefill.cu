@@ -20,7 +20,7 @@
 //   S(t) = Q K(t)^T            tcgen05.mma M=128 N=64, two S buffers in TMEM
 //   online softmax of S(t)     one row per thread, no shuffles, lazy rescale
 //   O += P(t) V(t)             tcgen05.mma M=128 N=D, P from shared memory
-//                              (P = P_hi + P_lo in two products, except FP4)
+//                              (P = P_hi + P_lo in two products for bf16)
 // S(t+1) is issued before the softmax of tile t, so the tensor cores compute
 // while the threads exponentiate. Operands are 128-byte-swizzled shared-memory
 // tiles: 16-bit K/V land there directly by TMA; FP8 / FP4 tiles are fetched raw
@@ -49,20 +49,21 @@ struct PrefillGeom {
   static constexpr bool k16 = (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16);
   static constexpr bool kFp8 = (KVF == PQKV_DTYPE_FP8_E4M3 || KVF == PQKV_DTYPE_FP8_E5M2);
   static constexpr bool kFp4 = (KVF == PQKV_DTYPE_FP4_E2M1);
-  // Compute warpgroups per CTA, each on its own 128-row query tile, sharing the
-  // K/V stages: two for 16-bit caches (one issues while the other stalls), one
-  // for quantized caches (their dequantized operand tiles take the room)
-  static constexpr int NWG = k16 ? 2 : 1;
-  static constexpr int kStages = k16 ? 3 : 4;     // KV tiles in flight
+  // Two compute warpgroups per CTA, each on its own 128-row query tile, sharing
+  // the K/V stages (one issues while the other stalls; a K/V tile serves 256
+  // rows). Quantized tiles are dequantized by both together.
+  static constexpr int NWG = 2;
+  static constexpr int kStages = (kFp8 && D == 128) ? 2 : 3;  // KV tiles in flight (shared memory)
   static constexpr int kThreads = NWG * kWG + 32; // + one producer warp
   static constexpr int NB = D / 64;                // 128-byte boxes per operand row
   static constexpr int kQBytes = NB * kM * 128;    // Q operand of one warpgroup [box][128 rows][128 B]
   static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
   static constexpr int kPBytes = kM * 128;         // P operand: 64 tokens (2 B) per row
-  // P = P_hi + P_lo, both rounded to the operand type, keeps ~16 significant
-  // bits of the probabilities (a bf16 P alone errs by up to |v| 2^-9); FP4's
-  // tolerance allows a single f16 P
-  static constexpr bool kSplitP = !kFp4;
+  // bf16 operands: P = P_hi + P_lo, both rounded to bf16, keeps ~16 significant
+  // bits of the probabilities (a bf16 P alone errs by up to |v| 2^-9, too much
+  // for the 2e-3 tolerance); f16 operands (fp16, FP8, FP4 caches) take a single
+  // f16 P (|v| 2^-11 at most)
+  static constexpr bool kSplitP = (KVF == PQKV_DTYPE_BF16);
   static constexpr int kRawTile = 32 * row_bytes(KVF, D);  // one block's K|V codes
   static constexpr int kScaleBytes = kFp8 ? 16 : (kFp4 ? 2 * 16 * (D / 16) : 0);
   static constexpr int kValBytes = kFp4 ? 2 * 16 * 4 * 2 : 0;
@@ -99,7 +100,21 @@ __device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
 // Barrier of the 128 threads of one compute warpgroup (named barrier 1 + wg;
 // the other warpgroup and the producer warp run on their own).
 __device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
-// The same barrier, returning whether v held on every thread of the warpgroup.
+// Barrier of all compute threads (named barrier 3), and its and-reduction.
+template <int NWG>
+__device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 3, %0;" ::"n"(NWG * 128) : "memory"); }
+template <int NWG>
+__device__ __forceinline__ bool cta_all(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 3, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(NWG * 128)
+      : "memory");
+  return r != 0;
+}
+// The warpgroup barrier, returning whether v held on every thread of the warpgroup.
 __device__ __forceinline__ bool wg_all(int wg, bool v) {
   uint32_t r;
   asm volatile(
@@ -142,8 +157,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   uint64_t* bar_empty = bar_full + kStages;                             // [kStages] stage free again
   uint64_t* bar_s_all = bar_empty + kStages;                            // [NWG][2] S(t) computed
   uint64_t* bar_pv_all = bar_s_all + 2 * NWG;                           // [NWG] PV(t) computed
-  int* stage_mask = reinterpret_cast<int*>(bar_pv_all + NWG);           // [kStages] blocks loaded
-  float* tile_sk = reinterpret_cast<float*>(stage_mask + kStages);      // [2][4] FP8 K scales
+  float* tile_sk = reinterpret_cast<float*>(bar_pv_all + NWG);          // [2][4] FP8 K scales
   float* tile_sv = tile_sk + 8;                                         // [2][4] FP8 V scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -188,7 +202,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], NWG);
+      mbar_init(&bar_empty[s], Gm::k16 ? NWG : 1);  // 16-bit: each warpgroup's commit; else one arrival
     }
     for (int i = 0; i < 2 * NWG; ++i) mbar_init(&bar_s_all[i], 1);
     for (int i = 0; i < NWG; ++i) mbar_init(&bar_pv_all[i], 1);
@@ -252,7 +266,6 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
             }
           }
         }
-        stage_mask[s] = mask;
         mbar_arrive_expect_tx(&bar_full[s], bytes);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -303,7 +316,17 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       ok = mbar_wait_bounded(&bar_full[s], (ph_full >> s) & 1u, p.timeout_ns) && ok;
       ph_full ^= 1u << s;
       ++n_prepared;
-      const int mask = stage_mask[s];
+      // blocks of the tile that were fetched (as the producer decided), from the
+      // block table itself so that every thread agrees even after a timeout
+      int mask = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int blk = 4 * t + j;
+        if (blk * kBlock < n_kv) {
+          const int id = __ldg(table + blk);
+          if (id >= 0 && id < p.nb) mask |= 1 << j;
+        }
+      }
       const int base = t * kN;
       uint8_t* st = sStage + s * Gm::kStageBytes;
       if constexpr (Gm::k16) {
@@ -321,10 +344,14 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           wg_sync(wg);
         }
       } else {
+        // both warpgroups are past the previous tile (its products read the
+        // operand buffers written below), then dequantize half of the tile each
+        cta_sync<NWG>();
+        const int gt = wg * kWG + r;
         uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
         uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
         constexpr int CPR = D / 8;  // 16-byte operand chunks per row
-        for (int u = r; u < kN * CPR; u += kWG) {
+        for (int u = gt; u < kN * CPR; u += NWG * kWG) {
           const int rr = u / CPR, c = u % CPR, j = rr >> 4, tr = rr & 15;
           const bool okr = ((mask >> j) & 1) && base + rr < L;
           uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
@@ -369,9 +396,9 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         }
         if constexpr (Gm::kFp4) {
           // outlier channels (their codes are 0): write the fp16 values over them;
-          // thread = (block j, K|V, slot, quarter of the tokens)
-          wg_sync(wg);
-          const int j = r >> 5, kv = (r >> 4) & 1, slot = (r >> 2) & 3, part = r & 3;
+          // thread = (block j, K|V, slot, eighth of the tokens)
+          cta_sync<NWG>();
+          const int j = gt >> 6, kv = (gt >> 5) & 1, slot = (gt >> 3) & 3, part = gt & 7;
           if ((mask >> j) & 1) {
             const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
             const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
@@ -380,8 +407,8 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
               uint8_t* op = kv ? vop : kop;
               const int c = ch >> 3;
 #pragma unroll
-              for (int q4 = 0; q4 < 4; ++q4) {
-                const int tr = 4 * part + q4, rr = 16 * j + tr;
+              for (int q4 = 0; q4 < 2; ++q4) {
+                const int tr = 2 * part + q4, rr = 16 * j + tr;
                 if (base + rr < L)
                   *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4) +
                                                (ch & 7) * 2) = val[tr * 4 + slot];
@@ -390,20 +417,21 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           }
         }
         if constexpr (Gm::kFp8) {
-          if (r < 4) {
-            const bool okb = (mask >> r) & 1;
-            const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + r * Gm::kSide);
-            tile_sk[(t & 1) * 4 + r] = okb ? sc[0] : 0.f;
-            tile_sv[(t & 1) * 4 + r] = okb ? sc[1] : 0.f;
+          if (gt < 4) {
+            const bool okb = (mask >> gt) & 1;
+            const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + gt * Gm::kSide);
+            tile_sk[(t & 1) * 4 + gt] = okb ? sc[0] : 0.f;
+            tile_sv[(t & 1) * 4 + gt] = okb ? sc[1] : 0.f;
           }
         }
         tc::fence_smem_to_async();
         tc::fence_before_sync();
         // the products may read the operands once every thread wrote its part;
-        // the consensus also carries timeouts
-        if (!wg_all(wg, ok)) ok = false;
+        // the consensus over both warpgroups also carries timeouts (quantized
+        // caches abort only here, so that neither warpgroup is left waiting)
+        ok = cta_all<NWG>(ok);
         // a raw stage is free as soon as it is dequantized
-        if (r == 0) mbar_arrive(&bar_empty[s]);
+        if (gt == 0) mbar_arrive(&bar_empty[s]);
       }
       return mask;
     };
@@ -443,7 +471,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     float m = -INFINITY, l = 0.f, vref = 0.f;
     int pv_done = 0;  // PV products issued so far
     mask_next = prepare(0);
-    if (!ok) aborted = true;
+    if (!(Gm::k16 ? wg_all(wg, ok) : ok)) aborted = true;
     else {
       if (r == 0) issue_s(0);
       n_s = 1;
@@ -590,10 +618,15 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       }
       tc::fence_smem_to_async();
       tc::fence_before_sync();
-      // one barrier per tile: P complete, S read, and no wait timed out anywhere
-      if (!wg_all(wg, ok)) {
-        aborted = true;
-        break;
+      // one barrier per tile: P complete and S read; for 16-bit caches it also
+      // decides on a timeout (quantized caches decide at the next dequantization)
+      if constexpr (Gm::k16) {
+        if (!wg_all(wg, ok)) {
+          aborted = true;
+          break;
+        }
+      } else {
+        wg_sync(wg);
       }
       if (r == 0) issue_pv(t, pv_done == 0);
       ++pv_done;
@@ -601,7 +634,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
 
     if (!aborted && pv_done > 0) {
       ok = mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns) && ok;
-      if (!wg_all(wg, ok)) aborted = true;
+      if (!(Gm::k16 ? wg_all(wg, ok) : cta_all<NWG>(ok))) aborted = true;
       else {
         ph_pv ^= 1u;
         ++n_pv_waited;
