@@ -112,7 +112,7 @@ def generate_kv(s: W.Spec, seqs, threads: int = 0, ahead: int = 8):
 class Setup:
     """Cache prefilled with the workload, plus one decode step's inputs, on `device`."""
 
-    def __init__(self, s: W.Spec, device, split_blocks: int, q_len: int = 1):
+    def __init__(self, s: W.Spec, device, split_blocks: int, q_len: int = 1, prefill: bool = False):
         import paged_quantized_kv_cache_b200 as pq
         self.pq = pq
         self.s = s
@@ -122,6 +122,7 @@ class Setup:
         self.lens0 = W.seq_lens(s)
         self.lens = W.decode_lens(s)
         self.q_len = q_len
+        self.prefill = prefill  # the step's q_len tokens attend by the chunked-prefill kernel
         self.cache = pq.allocate_cache(s.kv_dtype, tab.num_blocks, s.num_kv_heads, s.head_dim, device=device,
                                        fill=0xFF)
         self.err = torch.zeros(1, dtype=torch.int32, device=device)
@@ -173,20 +174,36 @@ class Setup:
         self.d_slots, self.d_bt, self.d_lens = views["slots"], views["bt"], views["lens"]
         self.h2d_bytes = sum(t.numel() * t.element_size() for _, t in parts)
         self.d_out = torch.empty_like(self.d_q)
-        self.ws = pq.decode_workspace(s.batch, s.num_q_heads * q_len, s.num_kv_heads, s.head_dim,
-                                      tab.max_blocks, split_blocks, device=device)
+        if prefill:
+            self.ws = None
+            self.cu = torch.arange(0, (s.batch + 1) * q_len, q_len, dtype=torch.int32, device=device)
+        else:
+            self.ws = pq.decode_workspace(s.batch, s.num_q_heads * q_len, s.num_kv_heads, s.head_dim,
+                                          tab.max_blocks, split_blocks, device=device)
 
     def write(self):
         self.pq.kv_cache_write(self.d_k, self.d_v, self.d_slots, self.cache, self.err)
 
     def decode(self):
-        if self.q_len == 1:
+        if self.prefill:
+            s = self.s
+            self.pq.paged_prefill_attention(self.d_q.view(-1, s.num_q_heads, s.head_dim), self.cu, self.q_len,
+                                            self.cache, self.d_bt, self.d_lens, self.scale,
+                                            self.d_out.view(-1, s.num_q_heads, s.head_dim), self.err)
+        elif self.q_len == 1:
             self.pq.paged_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale, self.d_out,
                                            self.ws, self.err, split_blocks=self.split_blocks)
         else:
             self.pq.paged_multi_query_decode_attention(self.d_q, self.cache, self.d_bt, self.d_lens, self.scale,
                                                        self.d_out, self.ws, self.err,
                                                        split_blocks=self.split_blocks)
+
+    def prefill_flops(self) -> float:
+        """Causal attention flops of the step's query chunk: 4 * Hq * D per
+        (query token, visible position)."""
+        s, C = self.s, self.q_len
+        pre = self.lens.astype(np.int64) - C
+        return 4.0 * s.num_q_heads * s.head_dim * float(np.sum(C * pre + C * (C + 1) // 2))
 
     def unique_tokens(self) -> int:
         s = self.s
@@ -544,7 +561,7 @@ def run_ours(args) -> None:
         dist.destroy_process_group()
 
 
-def run_e2e(st: Setup, args, world: int) -> dict:
+def run_e2e(st: Setup, args, world: int, per_step=None, unit: str = UNIT, scale: float = 1e9) -> dict:
     """Same step through the public API from pinned host buffers: copy the
     step's inputs in (q, the new tokens' k / v, slots, block tables, lengths),
     write + decode, copy the output back, every step."""
@@ -575,8 +592,8 @@ def run_e2e(st: Setup, args, world: int) -> dict:
     torch.cuda.synchronize(dev)
     barrier(world)
     ms = max_over_ranks(e0.elapsed_time(e1), world) / K
-    b = st.step_bytes()
-    return {"value": b["kv"] * world / (ms * 1e-3) / 1e9, "unit": UNIT, "ms_per_step": ms,
+    work = st.step_bytes()["kv"] if per_step is None else per_step
+    return {"value": work * world / (ms * 1e-3) / scale, "unit": unit, "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
 
@@ -725,135 +742,68 @@ PREFILL_DESCR = ("chunked prefill, Llama-3-8B-shaped layer: 16 seqs, prefix U[0,
 
 
 def run_prefill(args) -> None:
+    """One step = kv_cache_write of each sequence's 512-token chunk + the
+    chunked-prefill attention of its queries over prefix + chunk."""
     import oracle
-    import paged_quantized_kv_cache_b200 as pq
     rank, world, local = dist_env()
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU")
     torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
+    device = torch.device("cuda", local)
     if world > 1:
         import datetime
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    kv = KV_NAMES[args.kv_dtype or "bf16"]
-    B, Hq, Hkv, D, C = args.batch or 16, 32, 8, 128, 512
-    rng = np.random.default_rng(7 + rank)
-    prefix = rng.integers(0, 7681, size=B)
-    lens = (prefix + C).astype(np.int32)
-    nblk = (lens + 15) // 16
-    maxblk = int(nblk.max())
-    nb = int(nblk.sum()) + 64
-    perm = rng.permutation(nb).astype(np.int32)
-    tables = np.full((B, maxblk), -1, dtype=np.int32)
-    o = 0
-    for b in range(B):
-        tables[b, :nblk[b]] = perm[o:o + nblk[b]]
-        o += nblk[b]
-    in_dt = torch.float16 if kv == W.DT_FP16 else torch.bfloat16
-    g = pq.allocate_cache(kv, nb, Hkv, D, device=dev, fill=0)
-    err = torch.zeros(1, dtype=torch.int32, device=dev)
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(11 + rank)
-    # prefixes: written once, untimed
-    for b in range(B):
-        if prefix[b]:
-            k = torch.randn((int(prefix[b]), Hkv, D), generator=gen, device=dev).to(in_dt)
-            v = torch.randn((int(prefix[b]), Hkv, D), generator=gen, device=dev).to(in_dt)
-            sl = pq.build_slot_mapping(tables[b:b + 1], [0], [int(prefix[b])])
-            pq.kv_cache_write(k, v, torch.from_numpy(sl).to(dev), g, err)
-    # the step's inputs: chunk K/V, slots, queries, metadata (packed pinned host copy for e2e)
-    ck = torch.randn((B * C, Hkv, D), generator=gen, device=dev).to(in_dt)
-    cv = torch.randn((B * C, Hkv, D), generator=gen, device=dev).to(in_dt)
-    q = torch.randn((B * C, Hq, D), generator=gen, device=dev).to(in_dt)
-    slots = torch.from_numpy(pq.build_slot_mapping(tables, prefix, [C] * B)).to(dev)
-    cu = torch.from_numpy(np.arange(0, (B + 1) * C, C, dtype=np.int32)).to(dev)
-    bt = torch.from_numpy(tables).to(dev)
-    sl = torch.from_numpy(lens).to(dev)
-    out = torch.empty_like(q)
-    scale = 1.0 / math.sqrt(D)
-    stream = torch.cuda.current_stream(dev)
-
-    def write():
-        pq.kv_cache_write(ck, cv, slots, g, err)
-
-    def attend():
-        pq.paged_prefill_attention(q, cu, C, g, bt, sl, scale, out, err)
-
+    s = bench_spec("prefill", args.kv_dtype, args.batch, args.pool_blocks, q_len=512)
+    st = Setup(s, device, 0, q_len=512, prefill=True)
+    stream = torch.cuda.current_stream(device)
     for _ in range(max(args.warmup, 3)):
-        write()
-        attend()
-    torch.cuda.synchronize(dev)
+        st.write()
+        st.decode()
+    torch.cuda.synchronize(device)
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier(world)
-    torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(device)
     clocks.start()
     e0.record(stream)
     for i in range(K):
         ev[i][0].record(stream)
-        write()
+        st.write()
         ev[i][1].record(stream)
-        attend()
+        st.decode()
         ev[i][2].record(stream)
     e1.record(stream)
-    torch.cuda.synchronize(dev)
+    torch.cuda.synchronize(device)
     clocks.stop()
     barrier(world)
-    if int(err.item()) != 0:
-        raise RuntimeError("device error bits %d" % int(err.item()))
+    if int(st.err.item()) != 0:
+        raise RuntimeError("device error bits %d" % int(st.err.item()))
     ms = max_over_ranks(e0.elapsed_time(e1), world) / K
     att_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
     wr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
-    # causal attention flops: 4 * Hq * D per (query token, visible position)
-    flops = 4.0 * Hq * D * float(sum(C * int(prefix[b]) + C * (C + 1) // 2 for b in range(B)))
+    flops = st.prefill_flops()
     value = flops * world / (ms * 1e-3) / 1e12
     peaks = measured_peaks()
-    peak = peaks["bf16_tflops"]
     achieved = flops / (att_ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                "traffic": None, "kernel": "paged_prefill_kernel",
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None, "kernel": "paged_prefill_kernel",
                 "peak_source": peaks["source"] + " (MEASURED_PEAKS.json bf16_tflops, cuBLAS bf16 burst; the f16 "
                 "operands of quantized caches run at the same dense rate)",
                 "flops_per_launch": flops, "avg_launch_ms": att_ms}
-    # e2e: the step's inputs from pinned host memory, the output back, every step
-    h_q, h_k, h_v = q.cpu().pin_memory(), ck.cpu().pin_memory(), cv.cpu().pin_memory()
-    h_slots = slots.cpu().pin_memory()
-    h_meta = torch.cat([cu.cpu(), sl.cpu(), bt.cpu().ravel()]).pin_memory()
-    d_meta = torch.empty_like(h_meta, device=dev)
-    h_out = torch.empty_like(out, device="cpu").pin_memory()
-
-    def e2e_step():
-        q.copy_(h_q, non_blocking=True)
-        ck.copy_(h_k, non_blocking=True)
-        cv.copy_(h_v, non_blocking=True)
-        slots.copy_(h_slots, non_blocking=True)
-        d_meta.copy_(h_meta, non_blocking=True)
-        write()
-        attend()
-        h_out.copy_(out, non_blocking=True)
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize(dev)
-    Ke = max(1, min(K, 50))
-    e0.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize(dev)
-    ms_e2e = max_over_ranks(e0.elapsed_time(e1), world) / Ke
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_meta))
-    e2e = {"value": flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h_out.numel() * h_out.element_size()}
+    e2e = None if args.no_e2e else run_e2e(st, argparse.Namespace(steps=min(K, 50)), world, per_step=flops,
+                                            unit="TFLOP/s", scale=1e12)
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             # the oracle's prefill of one sequence: a 64-token chunk after 1024 cached tokens
             r2 = np.random.default_rng(3)
+            Hq, Hkv, D = s.num_q_heads, s.num_kv_heads, s.head_dim
             L, qn = 1088, 64
-            oc = oracle.Cache(kv, (L + 15) // 16, Hkv, D, poison=False)
+            in_dt = W.TORCH_DTYPE[W.input_dtype(s)]
+            oc = oracle.Cache(s.kv_dtype, (L + 15) // 16, Hkv, D, poison=False)
             tab = np.arange((L + 15) // 16, dtype=np.int32)[None]
             kk = torch.from_numpy(r2.standard_normal((L, Hkv, D)).astype(np.float32)).to(in_dt)
             vv = torch.from_numpy(r2.standard_normal((L, Hkv, D)).astype(np.float32)).to(in_dt)
@@ -863,22 +813,24 @@ def run_prefill(args) -> None:
             f1 = 4.0 * Hq * D * (qn * (L - qn) + qn * (qn + 1) // 2)
             reps, t0 = 0, time.perf_counter()
             while time.perf_counter() - t0 < min(args.cpu_budget, 10.0):
-                oracle.paged_prefill(oc, qq, cuq, tab, np.array([L], np.int32), scale)
+                oracle.paged_prefill(oc, qq, cuq, tab, np.array([L], np.int32), st.scale)
                 reps += 1
             dt = time.perf_counter() - t0
             cpu = {"value": f1 * reps / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
                    "sample": "%d runs of one sequence: a %d-token chunk after %d cached tokens, %s cache, %.1f s"
-                             % (reps, qn, L - qn, DT_LABEL[kv], dt)}
+                             % (reps, qn, L - qn, DT_LABEL[s.kv_dtype], dt)}
         line = {
             "metric": "chunked-prefill attention TFLOP/s (causal, paged cache)", "value": value, "unit": "TFLOP/s",
             "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16" if kv == W.DT_BF16 else ("fp16" if kv == W.DT_FP16 else DT_LABEL[kv] + "->f16"),
+            "dtype": "bf16" if s.kv_dtype == W.DT_BF16 else ("fp16" if s.kv_dtype == W.DT_FP16 else
+                                                             DT_LABEL[s.kv_dtype] + "->f16"),
             "data": "synthetic",
-            "config": {"workload": PREFILL_DESCR + "; KV " + DT_LABEL[kv], "batch": B, "chunk": C,
-                       "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": D, "context_tokens": int(lens.sum()),
-                       "l2": "KV read per step %.0f MB (prefix + chunk, once per query tile) vs 126 MB L2; no flush"
-                             % (float(lens.sum()) * Hkv * 2 * D * (2 if kv <= 1 else 1) / 1e6)},
+            "config": {"workload": PREFILL_DESCR + "; KV " + DT_LABEL[s.kv_dtype], "batch": s.batch, "chunk": 512,
+                       "num_q_heads": s.num_q_heads, "num_kv_heads": s.num_kv_heads, "head_dim": s.head_dim,
+                       "context_tokens": int(st.lens.sum()),
+                       "l2": "KV read per step %.0f MB (prefix + chunk) vs 126 MB L2; no flush"
+                             % (st.step_bytes()["kv"] / 1e6)},
             "attention_kernel_ms": att_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": 2 * K, "clocks": clocks.summary(),

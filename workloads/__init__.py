@@ -77,6 +77,11 @@ def spec(name: str, kv_dtype: Optional[int] = None, batch: Optional[int] = None)
     elif name == "fp4":
         s = Spec("fp4", 5, 256, 32, 8, 128, DT_FP4, DT_BF16, "loguniform", 1024, 65536,
                  pool_blocks=1048576, outlier_channels=2, chunk_tokens=512)
+    elif name == "prefill":
+        # chunked prefill: a cached prefix of U[0, 7680] tokens (written in
+        # 512-token chunks) and one more 512-token chunk whose queries attend
+        s = Spec("prefill", 6, 16, 32, 8, 128, DT_BF16, DT_BF16, "uniform", 0, 7680,
+                 pool_blocks=9000, append_tokens=512, chunk_tokens=512)
     else:
         raise KeyError(name)
     if kv_dtype is not None:
