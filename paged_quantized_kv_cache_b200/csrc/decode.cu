@@ -118,6 +118,39 @@ __device__ __forceinline__ int dmap(int mt, int rr) {
   }
 }
 
+// FP4 outlier channels: per-warp state carried from block to block. The
+// outlier channels of consecutive blocks of one KV head usually agree, so the
+// query fragment at the K outlier channels and the V outlier product are kept
+// in registers while the channel set stays the same; the V product goes to the
+// shared-memory accumulator of outlier channels only when the set changes or
+// the piece ends.
+struct OutlierState {
+  static constexpr uint32_t kNone = 0xFEFEFEFEu;  // no valid channel byte (they are < 128 or 0xFF)
+  uint32_t kidx;      // K outlier channels the cached query fragment belongs to
+  uint32_t kq;        // query fragment (B of the K outlier MMA) for them
+  uint32_t vidx;      // V outlier channels vacc belongs to
+  float vacc[4];      // V outlier product (rows = slots, lanes g < 4) not yet flushed
+  __device__ __forceinline__ void reset() {
+    kidx = vidx = kNone;
+    kq = 0;
+    vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.f;
+  }
+  // add vacc into the accumulator of outlier channels and clear it
+  template <int STRIDE>
+  __device__ __forceinline__ void flush(float* oext, int lane, int D) {
+    const int g = lane >> 2, qd = lane & 3;
+    if (vidx != kNone && g < 4) {
+      const int dch = (vidx >> (8 * g)) & 0xFF;
+      if (dch < D) {
+        oext[(2 * qd) * STRIDE + dch] += vacc[0];
+        oext[(2 * qd + 1) * STRIDE + dch] += vacc[1];
+      }
+    }
+    __syncwarp();
+    vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.f;
+  }
+};
+
 // ---------------------------------------------------------------------------
 // S^T (16 tokens x 8 query heads) += K Q^T for one block in shared memory.
 // Lane (g, qd) ends with rows (tokens) g, g + 8 and columns (heads) 2qd, 2qd + 1.
@@ -125,7 +158,7 @@ __device__ __forceinline__ int dmap(int mt, int rr) {
 template <int KVF, int D>
 __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, const uint32_t (&qf)[D / 16][2],
                                              const uint16_t* wq, const LdsmOffsets<KVF, D>& lo, int lane,
-                                             float (&sc)[4]) {
+                                             float (&sc)[4], OutlierState& ost) {
   using Gm = DecodeGeom<KVF, D>;
   constexpr int KT = D / 16;
   const int g = lane >> 2, qd = lane & 3;
@@ -197,22 +230,25 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
         mma16816<false>(so, ha[2], hb[2], ha[3], hb[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
       }
     }
-    // outlier channels (their codes are 0): S^T += Kout (16 tokens x 4 slots) Qout^T
+    // outlier channels (their codes are 0): S^T += Kout (16 tokens x 4 slots) Qout^T.
+    // Empty slots hold +0 values and get a zero query, so they add nothing.
     {
-      const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes;                      // K idx [8]
-      const uint16_t* kv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes);   // K vals [16][4]
-      uint32_t a0 = 0, a1 = 0, b0 = 0;
-      if (qd < 2) {
-        const int r0i = idx[2 * qd], r1i = idx[2 * qd + 1];
-        a0 = (uint32_t)kv[g * 4 + 2 * qd] | ((uint32_t)kv[g * 4 + 2 * qd + 1] << 16);
-        a1 = (uint32_t)kv[(g + 8) * 4 + 2 * qd] | ((uint32_t)kv[(g + 8) * 4 + 2 * qd + 1] << 16);
-        const uint32_t q0 = (r0i < D) ? wq[g * Gm::kQStride + r0i] : 0u;
-        const uint32_t q1 = (r1i < D) ? wq[g * Gm::kQStride + r1i] : 0u;
-        b0 = q0 | (q1 << 16);
-        if (r0i >= D) { a0 &= 0xFFFF0000u; a1 &= 0xFFFF0000u; }
-        if (r1i >= D) { a0 &= 0x0000FFFFu; a1 &= 0x0000FFFFu; }
+      const uint32_t kw = *reinterpret_cast<const uint32_t*>(side + Gm::kScaleBytes + Gm::kValBytes);  // K idx
+      const uint32_t* kv = reinterpret_cast<const uint32_t*>(side + Gm::kScaleBytes);  // K vals [16][4] fp16
+      if (kw != ost.kidx) {  // same for the whole warp
+        uint32_t b0 = 0;
+        if (qd < 2) {
+          const int r0i = (kw >> (16 * qd)) & 0xFF, r1i = (kw >> (16 * qd + 8)) & 0xFF;
+          const uint32_t q0 = (r0i < D) ? wq[g * Gm::kQStride + r0i] : 0u;
+          const uint32_t q1 = (r1i < D) ? wq[g * Gm::kQStride + r1i] : 0u;
+          b0 = q0 | (q1 << 16);
+        }
+        ost.kidx = kw;
+        ost.kq = b0;
       }
-      mma16816<false>(so, a0, a1, 0u, 0u, b0, 0u);
+      const uint32_t a0 = (qd < 2) ? kv[g * 2 + qd] : 0u;
+      const uint32_t a1 = (qd < 2) ? kv[(g + 8) * 2 + qd] : 0u;
+      mma16816<false>(so, a0, a1, 0u, 0u, ost.kq, 0u);
     }
   }
 #pragma unroll
@@ -226,7 +262,7 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
 template <int KVF, int D>
 __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const LdsmOffsets<KVF, D>& lo, int lane,
                                          int valid, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
-                                         float (&acc)[D / 16][4], float* oext) {
+                                         float (&acc)[D / 16][4], float* oext, OutlierState& ost) {
   using Gm = DecodeGeom<KVF, D>;
   constexpr int KT = D / 16;
   constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
@@ -314,12 +350,18 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
       }
     }
     // outlier channels: Oext[n][idx_r] += (Vout^T (4 slots x 16 tokens) P^T)[r][n].
-    // The result of slot r sits in lanes 4r..4r+3 (heads 2qd, 2qd+1); it is
-    // added to the warp's shared-memory accumulator of outlier channels, which
-    // follows O's rescaling and is folded into O when the piece ends.
+    // The result of slot r sits in lanes 4r..4r+3 (heads 2qd, 2qd+1); it stays
+    // in registers while the block's V outlier channels match the previous
+    // block's, and goes to the warp's shared-memory accumulator of outlier
+    // channels (which follows O's rescaling and is folded into O when the piece
+    // ends) when they change.
     {
-      const uint8_t* idx = side + Gm::kScaleBytes + Gm::kValBytes + 8;                         // V idx
+      const uint32_t vw = *reinterpret_cast<const uint32_t*>(side + Gm::kScaleBytes + Gm::kValBytes + 8);  // V idx
       const uint16_t* vv = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes + 128);    // V vals
+      if (vw != ost.vidx) {  // same for the whole warp
+        ost.template flush<Gm::kOStride>(oext, lane, D);
+        ost.vidx = vw;
+      }
       uint32_t a0 = 0, a2 = 0;
       if (g < 4) {
         a0 = (uint32_t)vv[t0 * 4 + g] | ((uint32_t)vv[(t0 + 1) * 4 + g] << 16);
@@ -329,16 +371,7 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
           a2 = mask_pair(a2, t1, valid);
         }
       }
-      float ex[4] = {0.f, 0.f, 0.f, 0.f};
-      mma_pv(ex, a0, 0u, a2, 0u);
-      if (g < 4) {
-        const int dch = idx[g];
-        if (dch < D) {
-          oext[(2 * qd) * Gm::kOStride + dch] += ex[0];
-          oext[(2 * qd + 1) * Gm::kOStride + dch] += ex[1];
-        }
-      }
-      __syncwarp();
+      mma_pv(ost.vacc, a0, 0u, a2, 0u);
     }
   }
 }
@@ -638,11 +671,13 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     uint32_t qf[KT][2];
     float acc[KT][4];
     float m0, m1, l0, l1, vref;
+    OutlierState ost;  // FP4 only
 
     auto begin_piece = [&]() {
       m0 = m1 = kNegInf;
       l0 = l1 = 0.f;
       vref = 0.f;
+      ost.reset();  // the query changes with the piece
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       const bool has = g < G;
@@ -691,7 +726,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       const float vs = Gm::kFp8 ? vref : 1.f;
       const int n0 = 2 * qd, n1 = 2 * qd + 1;
       if constexpr (Gm::kFp4) {  // fold the outlier channels' O in and clear it
-        __syncwarp();
+        ost.template flush<Gm::kOStride>(woext, lane, D);
 #pragma unroll
         for (int mt = 0; mt < KT; ++mt)
 #pragma unroll
@@ -778,8 +813,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
 
       // ---- scores of both blocks (independent MMA chains) ----
       float scA[4] = {0.f, 0.f, 0.f, 0.f}, scB[4] = {0.f, 0.f, 0.f, 0.f};
-      if (useA) block_scores<KVF, D>(tbA, sdA, qf, wq, lofs, lane, scA);
-      if (useB) block_scores<KVF, D>(tbB, sdB, qf, wq, lofs, lane, scB);
+      if (useA) block_scores<KVF, D>(tbA, sdA, qf, wq, lofs, lane, scA, ost);
+      if (useB) block_scores<KVF, D>(tbB, sdB, qf, wq, lofs, lane, scB, ost);
       float skA = 1.f, skB = 1.f, svA = 1.f, svB = 1.f;
       if constexpr (Gm::kFp8) {
         if (useA) { skA = reinterpret_cast<const float*>(sdA)[0]; svA = reinterpret_cast<const float*>(sdA)[1]; }
@@ -840,6 +875,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
           acc[mt][3] *= f1c;
         }
         if constexpr (Gm::kFp4) {  // the outlier channels' O follows the same rescale
+          ost.vacc[0] *= f0c;
+          ost.vacc[1] *= f1c;
           __syncwarp();
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt)
@@ -861,12 +898,12 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       auto pv = [&](uint32_t tb, const uint8_t* sd, int valid, float w0, float w1, float w2, float w3) {
         const uint32_t hA = pack_f32x2(w0, w1, kBf16Mma), hB = pack_f32x2(w2, w3, kBf16Mma);
         if constexpr (Gm::kFp4) {
-          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), 0u, 0u, acc, woext);
+          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), 0u, 0u, acc, woext, ost);
         } else {
           const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
           const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
           block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), movmatrix_t(lA),
-                           movmatrix_t(lB), acc, woext);
+                           movmatrix_t(lB), acc, woext, ost);
         }
       };
       if (useA && (!Gm::kFp8 || prA > 0.f))
