@@ -178,7 +178,8 @@ class Setup:
             self.ws = None
             self.cu = torch.arange(0, (s.batch + 1) * q_len, q_len, dtype=torch.int32, device=device)
         else:
-            self.ws = pq.decode_workspace(s.batch, s.num_q_heads * q_len, s.num_kv_heads, s.head_dim,
+            kp = min(q_len, max(1, 8 // (s.num_q_heads // s.num_kv_heads)))  # query tokens per decode pass
+            self.ws = pq.decode_workspace(s.batch, s.num_q_heads * kp, s.num_kv_heads, s.head_dim,
                                           tab.max_blocks, split_blocks, device=device)
 
     def write(self):

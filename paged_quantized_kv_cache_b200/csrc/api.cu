@@ -222,7 +222,7 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
   if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
   if (batch < 0 || batch > PQKV_MAX_BATCH || num_kv_heads < 1 || num_q_heads < 1 ||
-      num_q_heads % num_kv_heads != 0 || q_len < 1 || (int64_t)(num_q_heads / num_kv_heads) * q_len > 8 ||
+      num_q_heads % num_kv_heads != 0 || q_len < 1 || q_len > 64 || num_q_heads / num_kv_heads > 8 ||
       (head_dim != 64 && head_dim != 128) ||
       num_blocks < 1 || max_blocks_per_seq < 1 || split_blocks < 0)
     return PQKV_ERR_ARG;
@@ -237,8 +237,12 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   if ((int64_t)batch * num_kv_heads * max_blocks_per_seq >= INT32_MAX ||
       (int64_t)num_blocks * num_kv_heads * 32 >= INT32_MAX)
     return PQKV_ERR_ARG;
-  // the pieces hold one row per MMA column: q_len x (num_q_heads / num_kv_heads)
-  const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads * q_len, num_kv_heads, head_dim,
+  // A pass takes up to 8 MMA columns: the G query heads of kp consecutive query
+  // tokens; more tokens take several passes, each reading the KV once. The
+  // pieces hold one row per column of a pass.
+  const int Gh = num_q_heads / num_kv_heads;
+  const int kp = std::min(q_len, std::max(1, 8 / Gh));
+  const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads * kp, num_kv_heads, head_dim,
                                                   max_blocks_per_seq, split_blocks);
   if (need == 0 || workspace_bytes < need) return PQKV_ERR_ARG;
   DeviceInfo di;
@@ -259,18 +263,15 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   p.B = batch;
   p.Hq = num_q_heads;
   p.Hkv = num_kv_heads;
-  p.Gh = num_q_heads / num_kv_heads;
+  p.Gh = Gh;
   p.k = q_len;
-  p.G = p.Gh * q_len;
   p.nb = num_blocks;
   p.maxblk = max_blocks_per_seq;
   p.split_blocks = split_blocks;
-  p.slot_floats = (int)round_up((size_t)p.G * head_dim + 2 * p.G, 4);
+  p.slot_floats = (int)round_up((size_t)Gh * kp * head_dim + 2 * Gh * kp, 4);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms, st);
-  if (e != cudaSuccess) return PQKV_ERR_CUDA;
   MergeParams mp;
   mp.seq_lens = seq_lens;
   mp.partials = p.partials;
@@ -278,15 +279,23 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   mp.B = batch;
   mp.Hq = num_q_heads;
   mp.Hkv = num_kv_heads;
-  mp.G = p.G;
   mp.k = p.k;
   mp.Gh = p.Gh;
   mp.maxblk = max_blocks_per_seq;
   mp.warps = di.sms * decode_warps(kv_dtype, head_dim);
   mp.split_blocks = split_blocks;
   mp.slot_floats = p.slot_floats;
-  e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
-  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+  // passes run in stream order; each kernel waits for the previous one before
+  // touching the workspace (programmatic dependents wait for the full grid)
+  for (int q0 = 0; q0 < q_len; q0 += kp) {
+    p.q0 = mp.q0 = q0;
+    p.G = mp.G = Gh * std::min(kp, q_len - q0);
+    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms, st);
+    if (e != cudaSuccess) return PQKV_ERR_CUDA;
+    e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
+    if (e != cudaSuccess) return PQKV_ERR_CUDA;
+  }
+  return PQKV_OK;
 }
 
 int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads, const void* cache,

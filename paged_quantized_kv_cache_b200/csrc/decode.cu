@@ -38,9 +38,9 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // Element offset of the q / out row of MMA column c of KV head h of sequence
-// b: q and out are [B][k][Hq][D], column c = (token c / Gh, head c % Gh).
-__device__ __forceinline__ size_t col_row(int b, int h, int c, int k, int Gh, int Hq, int D) {
-  return ((size_t)(b * k + c / Gh) * Hq + (size_t)h * Gh + c % Gh) * D;
+// b: q and out are [B][k][Hq][D], column c = (token q0 + c / Gh, head c % Gh).
+__device__ __forceinline__ size_t col_row(int b, int h, int c, int k, int q0, int Gh, int Hq, int D) {
+  return ((size_t)(b * k + q0 + c / Gh) * Hq + (size_t)h * Gh + c % Gh) * D;
 }
 
 template <bool QBF16>
@@ -490,7 +490,7 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  const size_t orow = col_row(b, h, n, p.k, p.Gh, p.Hq, D) + lane * DPL;
+  const size_t orow = col_row(b, h, n, p.k, p.q0, p.Gh, p.Hq, D) + lane * DPL;
 #pragma unroll
   for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
 }
@@ -520,9 +520,9 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   const int B = p.B, Hkv = p.Hkv, G = p.G, Hq = p.Hq;
   const int g = lane >> 2, qd = lane & 3;
   // multi-query: positions at the end of the sequence hidden from this lane's
-  // two columns (query token c / Gh of k sits k - 1 - c / Gh before the end)
-  const int hid0 = (2 * qd < G) ? p.k - 1 - (2 * qd) / p.Gh : 0;
-  const int hid1 = (2 * qd + 1 < G) ? p.k - 1 - (2 * qd + 1) / p.Gh : 0;
+  // two columns (query token q0 + c / Gh of k sits k - 1 - q0 - c / Gh before the end)
+  const int hid0 = (2 * qd < G) ? p.k - 1 - p.q0 - (2 * qd) / p.Gh : 0;
+  const int hid1 = (2 * qd + 1 < G) ? p.k - 1 - p.q0 - (2 * qd + 1) / p.Gh : 0;
   uint64_t* wbar = bars + warp * NS;
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
@@ -681,7 +681,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
 #pragma unroll
       for (int mt = 0; mt < KT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
       const bool has = g < G;
-      const size_t qrow = has ? col_row(b, h, g, p.k, p.Gh, Hq, D) : 0;
+      const size_t qrow = has ? col_row(b, h, g, p.k, p.q0, p.Gh, Hq, D) : 0;
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
         if constexpr (Gm::k16) {
@@ -709,7 +709,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         __syncwarp();
         for (int i = lane; i < 8 * D; i += 32) {
           const int n = i / D;
-          const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.Gh, Hq, D) + (i % D)) : 0.f;
+          const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.q0, p.Gh, Hq, D) + (i % D)) : 0.f;
           wq[n * Gm::kQStride + i % D] = __half_as_ushort(__float2half_rn(v));
         }
         __syncwarp();
@@ -740,8 +740,8 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       if (!started_before && !ends_after) {
         const float i0 = lt0 > 0.f ? vs / lt0 : 0.f;
         const float i1 = lt1 > 0.f ? vs / lt1 : 0.f;
-        const size_t ob0 = n0 < G ? col_row(b, h, n0, p.k, p.Gh, Hq, D) : 0;
-        const size_t ob1 = n1 < G ? col_row(b, h, n1, p.k, p.Gh, Hq, D) : 0;
+        const size_t ob0 = n0 < G ? col_row(b, h, n0, p.k, p.q0, p.Gh, Hq, D) : 0;
+        const size_t ob1 = n1 < G ? col_row(b, h, n1, p.k, p.q0, p.Gh, Hq, D) : 0;
 #pragma unroll
         for (int mt = 0; mt < KT; ++mt) {
           const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);

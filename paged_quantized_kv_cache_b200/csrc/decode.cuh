@@ -44,11 +44,12 @@ struct DecodeParams {
   const int32_t* seq_lens;      // [B]
   int32_t* err;
   float* partials;              // [2 * chunks][slot_floats]
-  // G = MMA columns per KV head = Gh query heads x k query tokens (column
-  // c = token c / Gh, head c % Gh); k > 1 is multi-query decode: token i of a
-  // sequence of length L sits at position L - k + i and sees positions <= it
+  // G = MMA columns per KV head = Gh query heads x the query tokens q0,
+  // q0 + 1, ... of this pass (column c = token q0 + c / Gh, head c % Gh); k > 1
+  // is multi-query decode: token i of a sequence of length L sits at position
+  // L - k + i and sees positions <= it
   int B, Hq, Hkv, G, nb, maxblk;
-  int k, Gh;
+  int k, Gh, q0;
   int split_blocks;
   int slot_floats;
   float scale_log2;             // softmax scale * log2(e)
@@ -60,7 +61,7 @@ struct MergeParams {
   const float* partials;
   void* out;
   int B, Hq, Hkv, G, maxblk;
-  int k, Gh;                 // as in DecodeParams
+  int k, Gh, q0;             // as in DecodeParams
   int warps;         // warps of the decode grid (its balanced chunk length depends on it)
   int split_blocks;
   int slot_floats;

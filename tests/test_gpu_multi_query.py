@@ -2,8 +2,8 @@
 "Speculative decoding") against the oracle: each sequence's last q_len
 positions attend causally, which is the oracle's chunked prefill with chunks
 of q_len tokens. The decode kernels put the q_len x G query rows of a KV head in
-the columns of one tensor-core tile; q_len = 1 must reproduce
-pqkv_paged_decode_attention bit for bit."""
+the columns of one tensor-core tile (several passes when q_len x G > 8);
+q_len = 1 must reproduce pqkv_paged_decode_attention bit for bit."""
 import numpy as np
 import pytest
 import torch
@@ -25,6 +25,10 @@ CASES = [
     (pq.FP8_E5M2, torch.float16, 64, 16, 8, 4, 0),
     (pq.FP4_E2M1, torch.bfloat16, 128, 32, 8, 2, 0),
     (pq.FP4_E2M1, torch.float16, 64, 8, 4, 3, 2),
+    # more query tokens than one tile's 8 columns: several passes over the KV
+    (pq.BF16, torch.bfloat16, 128, 32, 8, 4, 0),
+    (pq.FP8_E4M3, torch.bfloat16, 128, 32, 8, 5, 3),
+    (pq.FP4_E2M1, torch.bfloat16, 64, 32, 4, 3, 0),
 ]
 
 
@@ -53,7 +57,8 @@ def _build(kv_dtype, qdt, D, Hq, Hkv, k, lens, seed):
 def _mq(g, q, bt, lens, scale, split=0):
     B, k, Hq, D = q.shape
     out = torch.full_like(q.cuda(), float("nan"))
-    ws = pq.decode_workspace(B, Hq * k, g.num_kv_heads, D, bt.shape[1], split)
+    kp = min(k, max(1, 8 // (Hq // g.num_kv_heads)))  # query tokens per pass
+    ws = pq.decode_workspace(B, Hq * kp, g.num_kv_heads, D, bt.shape[1], split)
     ws.fill_(0xAB)
     e = gh.err_flag()
     pq.paged_multi_query_decode_attention(q.cuda(), g, torch.from_numpy(np.ascontiguousarray(bt, np.int32)).cuda(),
@@ -98,10 +103,12 @@ def test_sequence_shorter_than_its_query_tokens_and_limits():
     ref, _ = oracle.paged_prefill(o, q[keep].reshape(-1, Hq, D), np.arange(0, 3 * k, k, dtype=np.int32),
                                   bt[keep], np.array([lens[i] for i in keep], np.int32), 0.125)
     gh.assert_close(out[keep].reshape(-1, Hq, D), ref, kv_dtype, tag="valid sequences")
-    # q_len x G above one tensor-core tile is rejected before anything runs
-    big = torch.zeros((1, 5, 8, 64), dtype=torch.float16, device="cuda")  # 5 x 2 columns
+    # more than 64 query tokens, or a workspace sized for too few columns, is
+    # rejected before anything runs
     ws = pq.decode_workspace(1, 8, 4, 64, bt.shape[1])
-    with pytest.raises(pq.PqkvError):
-        pq.paged_multi_query_decode_attention(big, g, torch.from_numpy(bt[:1].copy()).cuda(),
-                                              torch.tensor([40], dtype=torch.int32, device="cuda"), 0.1,
-                                              torch.empty_like(big), ws, gh.err_flag())
+    for kq, w in ((65, pq.decode_workspace(1, 8 * 4, 4, 64, bt.shape[1])), (4, ws[:16])):
+        big = torch.zeros((1, kq, 8, 64), dtype=torch.float16, device="cuda")
+        with pytest.raises(pq.PqkvError):
+            pq.paged_multi_query_decode_attention(big, g, torch.from_numpy(bt[:1].copy()).cuda(),
+                                                  torch.tensor([100], dtype=torch.int32, device="cuda"), 0.1,
+                                                  torch.empty_like(big), w, gh.err_flag())
