@@ -136,6 +136,7 @@ static float bf16_to_f32(uint16_t b) {
 /* Exported format helpers (for the oracle's own pins). */
 void oracle_encode(int dt, const float* x, int64_t n, uint8_t* out) {
   const minifloat* f = fmt_of(dt);
+#pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) out[i] = (uint8_t)mf_encode(f, x[i]);
 }
 

@@ -44,3 +44,16 @@ def test_random_bit_patterns_and_specials(code, odt):
     x = x[np.isfinite(x)]
     specials = np.array([0.0, -0.0, 1e-45, -1e-45, 1e-38, 3e38, -3e38, 1.0, -1.0], np.float32)
     _check(np.concatenate([x, specials]).astype(np.float32), code, odt)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("code,odt", FMTS, ids=["e4m3", "e5m2", "e2m1"])
+def test_all_two_to_the_32_inputs(code, odt):
+    """Every float32 bit pattern except NaNs (outside the encoders' domain),
+    in chunks of 2^26: GPU and oracle codes equal bit for bit."""
+    chunk = 1 << 26
+    for c0 in range(0, 1 << 32, chunk):
+        bits = np.arange(c0, c0 + chunk, dtype=np.uint64).astype(np.uint32)
+        x = bits.view(np.float32)
+        x = x[~np.isnan(x)]
+        _check(x, code, odt)
