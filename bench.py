@@ -163,17 +163,24 @@ class Setup:
             offs[name] = total
             total += (t.numel() * t.element_size() + 255) // 256 * 256
         self.h_in = torch.empty(total, dtype=torch.uint8).pin_memory()
-        self.d_in = torch.empty(total, dtype=torch.uint8, device=device)
-        views = {}
         for name, t in parts:
             n = t.numel() * t.element_size()
             self.h_in[offs[name]:offs[name] + n].copy_(t.contiguous().view(-1).view(torch.uint8))
-            views[name] = self.d_in[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
-        self.d_in.copy_(self.h_in)
-        self.d_q, self.d_k, self.d_v = views["q"], views["k"], views["v"]
-        self.d_slots, self.d_bt, self.d_lens = views["slots"], views["bt"], views["lens"]
+        # two device copies of the inputs and outputs, so that the end-to-end
+        # leg can copy one step's inputs in while the previous step computes
+        self.d_in_sets, self._views = [], []
+        for _ in range(2):
+            d_in = torch.empty(total, dtype=torch.uint8, device=device)
+            d_in.copy_(self.h_in)
+            views = {}
+            for name, t in parts:
+                n = t.numel() * t.element_size()
+                views[name] = d_in[offs[name]:offs[name] + n].view(t.dtype).view(t.shape)
+            self.d_in_sets.append(d_in)
+            self._views.append(views)
         self.h2d_bytes = sum(t.numel() * t.element_size() for _, t in parts)
-        self.d_out = torch.empty_like(self.d_q)
+        self.d_outs = [torch.empty_like(self._views[0]["q"]) for _ in range(2)]
+        self.use(0)
         if prefill:
             self.ws = None
             self.cu = torch.arange(0, (s.batch + 1) * q_len, q_len, dtype=torch.int32, device=device)
@@ -181,6 +188,14 @@ class Setup:
             kp = min(q_len, max(1, 8 // (s.num_q_heads // s.num_kv_heads)))  # query tokens per decode pass
             self.ws = pq.decode_workspace(s.batch, s.num_q_heads * kp, s.num_kv_heads, s.head_dim,
                                           tab.max_blocks, split_blocks, device=device)
+
+    def use(self, i: int):
+        """Make input / output set i the one write() and decode() use."""
+        v = self._views[i]
+        self.d_in = self.d_in_sets[i]
+        self.d_q, self.d_k, self.d_v = v["q"], v["k"], v["v"]
+        self.d_slots, self.d_bt, self.d_lens = v["slots"], v["bt"], v["lens"]
+        self.d_out = self.d_outs[i]
 
     def write(self):
         self.pq.kv_cache_write(self.d_k, self.d_v, self.d_slots, self.cache, self.err)
@@ -499,20 +514,18 @@ def run_ours(args) -> None:
     torch.cuda.synchronize(device)
 
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    # the timed region: K steps back to back (nothing between the kernels, so
+    # each launch overlaps the previous kernel's tail as programmed)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(device)
     clocks.start()
     e0.record(stream)
     for i in range(K):
-        ev[i][0].record(stream)
         st.write()
-        ev[i][1].record(stream)
         st.decode()
-        ev[i][2].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     clocks.stop()
@@ -521,6 +534,15 @@ def run_ours(args) -> None:
         raise RuntimeError("device error bits %d during the timed steps" % int(st.err.item()))
     total_ms = max_over_ranks(e0.elapsed_time(e1), world)
     ms_step = total_ms / K
+    # then K more steps with events around each call, for the kernels' own times
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record(stream)
+        st.write()
+        ev[i][1].record(stream)
+        st.decode()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(device)
     dec_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
     wr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
 
@@ -533,7 +555,8 @@ def run_ours(args) -> None:
                 "frac": achieved / peaks["hbm_gbs"],
                 "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype]),
                 "kernel": "paged_decode_kernel", "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, "
-                "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms}
+                "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms,
+                "timing": "CUDA events around each decode call (decode + merge kernels) over K further steps"}
 
     e2e = run_e2e(st, args, world) if not args.no_e2e else None
 
@@ -552,8 +575,9 @@ def run_ours(args) -> None:
             "decode_tok_s_per_layer": tok_s,
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            # per step: cache write, split decode, log-sum-exp merge
-            "gpu_launches": 3 * K, "clocks": clocks.summary(),
+            # per step: cache write, then per decode pass a split decode and its log-sum-exp merge
+            "gpu_launches": (1 + 2 * -(-args.q_len // max(1, min(args.q_len, 8 // (s.num_q_heads // s.num_kv_heads)))))
+            * K, "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -563,40 +587,61 @@ def run_ours(args) -> None:
 
 
 def run_e2e(st: Setup, args, world: int, per_step=None, unit: str = UNIT, scale: float = 1e9) -> dict:
-    """Same step through the public API from pinned host buffers: copy the
-    step's inputs in (q, the new tokens' k / v, slots, block tables, lengths),
-    write + decode, copy the output back, every step."""
+    """Same step through the public API from pinned host buffers, as a serving
+    loop runs it: every step copies its inputs in (q, the new tokens' k / v,
+    slots, block tables, lengths; one packed copy) and its output back. The
+    copies run on their own streams, so step i + 1's inputs travel in and step
+    i's output travels out while step i computes (two device buffer sets);
+    the timed region spans the first input copy to the last output copy."""
     dev = st.device
-    stream = torch.cuda.current_stream(dev)
-    h_out = torch.empty(st.d_out.shape, dtype=st.d_out.dtype).pin_memory()
+    comp = torch.cuda.current_stream(dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    h_outs = [torch.empty(st.d_outs[0].shape, dtype=st.d_outs[0].dtype).pin_memory() for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
     h2d = st.h2d_bytes
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = h_outs[0].numel() * h_outs[0].element_size()
 
-    def step():
-        st.d_in.copy_(st.h_in, non_blocking=True)
+    def step(i):
+        b = i & 1
+        if i >= 2:
+            s_in.wait_event(ev_comp[b])  # step i - 2 has read this input set
+        with torch.cuda.stream(s_in):
+            st.d_in_sets[b].copy_(st.h_in, non_blocking=True)
+        ev_in[b].record(s_in)
+        comp.wait_event(ev_in[b])
+        if i >= 2:
+            comp.wait_event(ev_out[b])  # step i - 2's output has left this buffer
+        st.use(b)
         st.write()
         st.decode()
-        h_out.copy_(st.d_out, non_blocking=True)
+        ev_comp[b].record(comp)
+        s_out.wait_event(ev_comp[b])
+        with torch.cuda.stream(s_out):
+            h_outs[b].copy_(st.d_outs[b], non_blocking=True)
+        ev_out[b].record(s_out)
 
-    for _ in range(3):
-        step()
+    for i in range(3):
+        step(i)
     torch.cuda.synchronize(dev)
     K = max(1, args.steps)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
-    e0.record(stream)
-    for _ in range(K):
-        step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(K):
+        step(i)
+    e1.record(s_out)
     torch.cuda.synchronize(dev)
     barrier(world)
+    st.use(0)
     ms = max_over_ranks(e0.elapsed_time(e1), world) / K
     work = st.step_bytes()["kv"] if per_step is None else per_step
     return {"value": work * world / (ms * 1e-3) / scale, "unit": unit, "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "inputs of step i+1 copied in and output of step i copied out while step i computes"}
 
 def run_block_op(args) -> None:
     """copy_blocks: n random (src, dst) pairs of the workload's pool per step.
@@ -763,7 +808,6 @@ def run_prefill(args) -> None:
         st.decode()
     torch.cuda.synchronize(device)
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier(world)
@@ -771,11 +815,8 @@ def run_prefill(args) -> None:
     clocks.start()
     e0.record(stream)
     for i in range(K):
-        ev[i][0].record(stream)
         st.write()
-        ev[i][1].record(stream)
         st.decode()
-        ev[i][2].record(stream)
     e1.record(stream)
     torch.cuda.synchronize(device)
     clocks.stop()
@@ -783,6 +824,15 @@ def run_prefill(args) -> None:
     if int(st.err.item()) != 0:
         raise RuntimeError("device error bits %d" % int(st.err.item()))
     ms = max_over_ranks(e0.elapsed_time(e1), world) / K
+    # then K more steps with events around each call, for the kernels' own times
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    for i in range(K):
+        ev[i][0].record(stream)
+        st.write()
+        ev[i][1].record(stream)
+        st.decode()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(device)
     att_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
     wr_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
     flops = st.prefill_flops()
