@@ -84,6 +84,12 @@ def bench_spec(name: str, kv_name: str | None, batch: int | None = None, pool: i
     return s
 
 
+def decode_passes(q_len: int, G: int) -> int:
+    """Decode passes of a multi-query step: up to 16 query rows (G heads x tokens) per KV read."""
+    kp = min(q_len, max(1, 16 // G))
+    return -(-q_len // kp)
+
+
 def per_token_bytes(s: W.Spec) -> int:
     """Algorithmic KV bytes of one token (all KV heads, K and V, with its share of
     the scales / outlier buffers of the cache layout)."""
@@ -185,9 +191,8 @@ class Setup:
             self.ws = None
             self.cu = torch.arange(0, (s.batch + 1) * q_len, q_len, dtype=torch.int32, device=device)
         else:
-            kp = min(q_len, max(1, 8 // (s.num_q_heads // s.num_kv_heads)))  # query tokens per decode pass
-            self.ws = pq.decode_workspace(s.batch, s.num_q_heads * kp, s.num_kv_heads, s.head_dim,
-                                          tab.max_blocks, split_blocks, device=device)
+            self.ws = pq.multi_query_decode_workspace(s.batch, q_len, s.num_q_heads, s.num_kv_heads, s.head_dim,
+                                                      tab.max_blocks, split_blocks, device=device)
 
     def use(self, i: int):
         """Make input / output set i the one write() and decode() use."""
@@ -576,8 +581,8 @@ def run_ours(args) -> None:
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             # per step: cache write, then per decode pass a split decode and its log-sum-exp merge
-            "gpu_launches": (1 + 2 * -(-args.q_len // max(1, min(args.q_len, 8 // (s.num_q_heads // s.num_kv_heads)))))
-            * K, "clocks": clocks.summary(),
+            "gpu_launches": (1 + 2 * decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
+            "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -163,7 +163,8 @@ int pqkv_kv_cache_write(const void* k, const void* v, int in_dtype, int num_toke
 /*
  * Device workspace needed by pqkv_paged_decode_attention for these sizes, on
  * the current device. split_blocks as in pqkv_paged_decode_attention. Returns 0
- * for invalid sizes.
+ * for invalid sizes. num_q_heads / num_kv_heads may be up to 16 here (the
+ * columns of one multi-query pass); the decode itself takes up to 8.
  */
 size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
                                    int head_dim, int max_blocks_per_seq,
@@ -207,17 +208,20 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
  * written to the cache first and seq_lens[b] counts them): token i sits at
  * position seq_lens[b] - q_len + i and attends to positions 0..that one. q and
  * out are [batch][q_len][num_q_heads][head_dim] (device, contiguous). The
- * decode kernels take the query rows of a KV head as the columns of one
- * tensor-core tile: kp = min(q_len, max(1, 8 / G)) consecutive query tokens
- * (G = num_q_heads / num_kv_heads <= 8) share each read of the KV; more tokens
- * take ceil(q_len / kp) passes, each reading the KV once more (long chunks:
- * pqkv_paged_prefill_attention). 1 <= q_len <= 64. workspace: at least
- * pqkv_decode_workspace_bytes(batch, num_q_heads * kp, num_kv_heads, head_dim,
- * max_blocks_per_seq, split_blocks) bytes (num_q_heads * q_len is always
- * enough when q_len x G <= 8). A sequence with 0 < seq_lens[b] < q_len gets
- * zero rows and PQKV_DEVERR_SEQ_LEN. q_len = 1 is pqkv_paged_decode_attention.
- * Other arguments, results and errors as there.
+ * decode kernels take the query rows of a KV head as the columns of one or two
+ * 8-column tensor-core tiles: kp = min(q_len, 16 / G) consecutive query tokens
+ * (G = num_q_heads / num_kv_heads <= 8) share each read of the KV, in one tile
+ * when kp x G <= 8, else two; more tokens take ceil(q_len / kp) passes, each
+ * reading the KV once more (long chunks: pqkv_paged_prefill_attention).
+ * 1 <= q_len <= 64. workspace: at least
+ * pqkv_multi_query_decode_workspace_bytes(batch, q_len, ...) bytes. A sequence
+ * with 0 < seq_lens[b] < q_len gets zero rows and PQKV_DEVERR_SEQ_LEN.
+ * q_len = 1 is pqkv_paged_decode_attention, bit for bit. Other arguments,
+ * results and errors as there.
  */
+size_t pqkv_multi_query_decode_workspace_bytes(int batch, int q_len, int num_q_heads,
+                                               int num_kv_heads, int head_dim,
+                                               int max_blocks_per_seq, int split_blocks);
 int pqkv_paged_multi_query_decode_attention(const void* q, int q_dtype, int batch, int q_len,
                                             int num_q_heads, const void* cache, const void* scales,
                                             const void* outliers_idx, const void* outliers_val,

@@ -38,7 +38,7 @@ EXPORTS = (
     "pqkv_paged_decode_attention_noalloc", "pqkv_pool_num_evictable", "pqkv_pool_num_cached",
     "pqkv_pool_prefix_lookup", "pqkv_pool_prefix_insert", "pqkv_pool_cow", "pqkv_copy_blocks",
     "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in", "pqkv_paged_prefill_attention",
-    "pqkv_paged_multi_query_decode_attention",
+    "pqkv_paged_multi_query_decode_attention", "pqkv_multi_query_decode_workspace_bytes",
 )
 
 
@@ -59,6 +59,7 @@ def _load() -> ctypes.CDLL:
         "pqkv_cache_layout": (I, [I, I, I, I, P]),
         "pqkv_kv_cache_write": (I, [P, P, I, I, P, P, P, P, P, I, I, I, I, P, P]),
         "pqkv_decode_workspace_bytes": (Z, [I, I, I, I, I, I]),
+        "pqkv_multi_query_decode_workspace_bytes": (Z, [I, I, I, I, I, I, I]),
         "pqkv_paged_decode_attention": (I, [P, I, I, I, P, P, P, P, I, I, I, I, P, I, P, ctypes.c_float, I,
                                             P, P, Z, P, P]),
         "pqkv_decode_workspace_init": (I, [P, Z, P]),
@@ -214,6 +215,16 @@ def decode_workspace(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: 
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
+def multi_query_decode_workspace(batch: int, q_len: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                                 max_blocks_per_seq: int, split_blocks: int = 0, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for paged_multi_query_decode_attention (torch allocation)."""
+    n = int(_lib.pqkv_multi_query_decode_workspace_bytes(batch, q_len, num_q_heads, num_kv_heads, head_dim,
+                                                         max_blocks_per_seq, split_blocks))
+    if n == 0:
+        raise PqkvError("pqkv_multi_query_decode_workspace_bytes", ERR_ARG)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
 def decode_workspace_init(workspace: torch.Tensor, stream=None) -> None:
     _check("pqkv_decode_workspace_init", _lib.pqkv_decode_workspace_init(
         _dev_ptr(workspace, "workspace"), workspace.numel(), _stream_handle(stream, workspace.device)))
@@ -248,7 +259,7 @@ def paged_multi_query_decode_attention(q: torch.Tensor, cache: KVCache, block_ta
                                       workspace: torch.Tensor, err_flag: torch.Tensor, split_blocks: int = 0,
                                       stream=None) -> None:
     """pqkv_paged_multi_query_decode_attention: q, out [B][q_len][Hq][D] (each sequence's last q_len
-    positions); workspace from decode_workspace(B, Hq * q_len, ...)."""
+    positions); workspace from multi_query_decode_workspace(B, q_len, Hq, ...)."""
     B, k, Hq, D = q.shape
     if out.shape != q.shape or out.dtype != q.dtype:
         raise ValueError("out must match q")

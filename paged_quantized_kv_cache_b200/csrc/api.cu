@@ -11,11 +11,11 @@
 #include "write.cuh"
 
 namespace pqkv {
-cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap, const DecodeParams& p,
+cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st);
 cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
-size_t decode_smem_bytes(int kv_dtype, int D, int B);
-int decode_warps(int kv_dtype, int D);
+size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt);
+int decode_warps(int kv_dtype, int D, int nt);
 }  // namespace pqkv
 
 using namespace pqkv;
@@ -196,7 +196,7 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
       (head_dim != 64 && head_dim != 128) || max_blocks_per_seq < 1 || split_blocks < 0)
     return 0;
   const int G = num_q_heads / num_kv_heads;
-  if (G > 8) return 0;
+  if (G > 16) return 0;  // columns of one pass: up to two tiles of 8
   DeviceInfo di;
   if (!device_info(di)) return 0;
   const size_t slot = round_up((size_t)G * head_dim + 2 * G, 4) * 4;
@@ -212,6 +212,20 @@ int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_str
   return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
              ? PQKV_OK
              : PQKV_ERR_CUDA;
+}
+
+// Query tokens per decode pass: the G query heads of kp consecutive tokens fill
+// up to 16 MMA columns (two tiles of 8 when more than 8 are used).
+static int mq_tokens_per_pass(int q_len, int G) { return std::min(q_len, std::max(1, 16 / G)); }
+
+size_t pqkv_multi_query_decode_workspace_bytes(int batch, int q_len, int num_q_heads, int num_kv_heads,
+                                               int head_dim, int max_blocks_per_seq, int split_blocks) {
+  if (q_len < 1 || q_len > 64 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
+      num_q_heads / num_kv_heads > 8)
+    return 0;
+  const int kp = mq_tokens_per_pass(q_len, num_q_heads / num_kv_heads);
+  return pqkv_decode_workspace_bytes(batch, num_q_heads * kp, num_kv_heads, head_dim, max_blocks_per_seq,
+                                     split_blocks);
 }
 
 static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num_q_heads, const void* cache,
@@ -237,17 +251,18 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   if ((int64_t)batch * num_kv_heads * max_blocks_per_seq >= INT32_MAX ||
       (int64_t)num_blocks * num_kv_heads * 32 >= INT32_MAX)
     return PQKV_ERR_ARG;
-  // A pass takes up to 8 MMA columns: the G query heads of kp consecutive query
-  // tokens; more tokens take several passes, each reading the KV once. The
-  // pieces hold one row per column of a pass.
+  // A pass takes up to 16 MMA columns: the G query heads of kp consecutive
+  // query tokens; more tokens take several passes, each reading the KV once.
+  // The pieces hold one row per column of a pass.
   const int Gh = num_q_heads / num_kv_heads;
-  const int kp = std::min(q_len, std::max(1, 8 / Gh));
+  const int kp = mq_tokens_per_pass(q_len, Gh);
   const size_t need = pqkv_decode_workspace_bytes(batch, num_q_heads * kp, num_kv_heads, head_dim,
                                                   max_blocks_per_seq, split_blocks);
   if (need == 0 || workspace_bytes < need) return PQKV_ERR_ARG;
   DeviceInfo di;
   if (!device_info(di)) return PQKV_ERR_CUDA;
-  if (decode_smem_bytes(kv_dtype, head_dim, batch) > (size_t)di.max_smem) return PQKV_ERR_ARG;
+  for (int nt = 1; nt <= (Gh * kp > 8 ? 2 : 1); ++nt)
+    if (decode_smem_bytes(kv_dtype, head_dim, batch, nt) > (size_t)di.max_smem) return PQKV_ERR_ARG;
   CUtensorMap tmap;
   if (!cached_cache_map(&tmap, cache, kv_dtype, num_blocks, num_kv_heads, head_dim)) return PQKV_ERR_CUDA;
   DecodeParams p;
@@ -282,7 +297,6 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   mp.k = p.k;
   mp.Gh = p.Gh;
   mp.maxblk = max_blocks_per_seq;
-  mp.warps = di.sms * decode_warps(kv_dtype, head_dim);
   mp.split_blocks = split_blocks;
   mp.slot_floats = p.slot_floats;
   // passes run in stream order; each kernel waits for the previous one before
@@ -290,7 +304,9 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   for (int q0 = 0; q0 < q_len; q0 += kp) {
     p.q0 = mp.q0 = q0;
     p.G = mp.G = Gh * std::min(kp, q_len - q0);
-    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p, di.sms, st);
+    const int nt = p.G > 8 ? 2 : 1;  // tiles of 8 columns
+    mp.warps = di.sms * decode_warps(kv_dtype, head_dim, nt);
+    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
     if (e != cudaSuccess) return PQKV_ERR_CUDA;
     e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
     if (e != cudaSuccess) return PQKV_ERR_CUDA;

@@ -124,16 +124,20 @@ __device__ __forceinline__ int dmap(int mt, int rr) {
 // in registers while the channel set stays the same; the V product goes to the
 // shared-memory accumulator of outlier channels only when the set changes or
 // the piece ends.
+template <int NT>
 struct OutlierState {
   static constexpr uint32_t kNone = 0xFEFEFEFEu;  // no valid channel byte (they are < 128 or 0xFF)
-  uint32_t kidx;      // K outlier channels the cached query fragment belongs to
-  uint32_t kq;        // query fragment (B of the K outlier MMA) for them
-  uint32_t vidx;      // V outlier channels vacc belongs to
-  float vacc[4];      // V outlier product (rows = slots, lanes g < 4) not yet flushed
+  uint32_t kidx;        // K outlier channels the cached query fragments belong to
+  uint32_t kq[NT];      // query fragments (B of the K outlier MMA), per column tile
+  uint32_t vidx;        // V outlier channels vacc belongs to
+  float vacc[NT][4];    // V outlier product (rows = slots, lanes g < 4) not yet flushed
   __device__ __forceinline__ void reset() {
     kidx = vidx = kNone;
-    kq = 0;
-    vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      kq[nt] = 0;
+      vacc[nt][0] = vacc[nt][1] = vacc[nt][2] = vacc[nt][3] = 0.f;
+    }
   }
   // add vacc into the accumulator of outlier channels and clear it
   template <int STRIDE>
@@ -142,35 +146,48 @@ struct OutlierState {
     if (vidx != kNone && g < 4) {
       const int dch = (vidx >> (8 * g)) & 0xFF;
       if (dch < D) {
-        oext[(2 * qd) * STRIDE + dch] += vacc[0];
-        oext[(2 * qd + 1) * STRIDE + dch] += vacc[1];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          oext[(8 * nt + 2 * qd) * STRIDE + dch] += vacc[nt][0];
+          oext[(8 * nt + 2 * qd + 1) * STRIDE + dch] += vacc[nt][1];
+        }
       }
     }
     __syncwarp();
-    vacc[0] = vacc[1] = vacc[2] = vacc[3] = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) vacc[nt][0] = vacc[nt][1] = vacc[nt][2] = vacc[nt][3] = 0.f;
   }
 };
 
 // ---------------------------------------------------------------------------
-// S^T (16 tokens x 8 query heads) += K Q^T for one block in shared memory.
-// Lane (g, qd) ends with rows (tokens) g, g + 8 and columns (heads) 2qd, 2qd + 1.
+// S^T (16 tokens x 8 NT query rows) += K Q^T for one block in shared memory.
+// Lane (g, qd) ends with rows (tokens) g, g + 8 and columns 8nt + 2qd, 8nt +
+// 2qd + 1 of each column tile nt; the K fragments are dequantized once for all.
 // ---------------------------------------------------------------------------
-template <int KVF, int D>
-__device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, const uint32_t (&qf)[D / 16][2],
-                                             const uint16_t* wq, const LdsmOffsets<KVF, D>& lo, int lane,
-                                             float (&sc)[4], OutlierState& ost) {
-  using Gm = DecodeGeom<KVF, D>;
+template <int KVF, int D, int NT>
+__device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side,
+                                             const uint32_t (&qf)[NT][D / 16][2], const uint16_t* wq,
+                                             const LdsmOffsets<KVF, D>& lo, int lane, float (&sc)[NT][4],
+                                             OutlierState<NT>& ost) {
+  using Gm = DecodeGeom<KVF, D, NT>;
   constexpr int KT = D / 16;
   const int g = lane >> 2, qd = lane & 3;
-  float se[4] = {0.f, 0.f, 0.f, 0.f}, so[4] = {0.f, 0.f, 0.f, 0.f};  // two independent chains
+  float se[NT][4], so[NT][4];  // two independent chains per column tile
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) se[nt][i] = so[nt][i] = 0.f;
   if constexpr (Gm::k16) {
     constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
 #pragma unroll
     for (int kk = 0; kk < KT; ++kk) {
       uint32_t a0, a1, a2, a3;
       ldsm_x4(tb + lo.k[kk], a0, a1, a2, a3);
-      if (kk & 1) mma16816<kBf>(so, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
-      else mma16816<kBf>(se, a0, a1, a2, a3, qf[kk][0], qf[kk][1]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        if (kk & 1) mma16816<kBf>(so[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+        else mma16816<kBf>(se[nt], a0, a1, a2, a3, qf[nt][kk][0], qf[nt][kk][1]);
+      }
     }
   } else if constexpr (Gm::kFp8) {
     // ldmatrix on byte data: lane (g, qd) receives bytes 4qd..4qd+3 of a token
@@ -184,8 +201,11 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
       dec4<KVF>(r1, x1l, x1h);
       dec4<KVF>(r2, x2l, x2h);
       dec4<KVF>(r3, x3l, x3h);
-      mma16816<false>(se, x0l, x1l, x0h, x1h, qf[2 * cp][0], qf[2 * cp][1]);
-      mma16816<false>(so, x2l, x3l, x2h, x3h, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mma16816<false>(se[nt], x0l, x1l, x0h, x1h, qf[nt][2 * cp][0], qf[nt][2 * cp][1]);
+        mma16816<false>(so[nt], x2l, x3l, x2h, x3h, qf[nt][2 * cp + 1][0], qf[nt][2 * cp + 1][1]);
+      }
     }
   } else {
     // FP4: one 16-byte chunk = 32 d; lane (g, qd) receives the 8 codes
@@ -226,8 +246,11 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
           ha[i] = *reinterpret_cast<uint32_t*>(&xa);
           hb[i] = *reinterpret_cast<uint32_t*>(&yb);
         }
-        mma16816<false>(se, ha[0], hb[0], ha[1], hb[1], qf[2 * c][0], qf[2 * c][1]);
-        mma16816<false>(so, ha[2], hb[2], ha[3], hb[3], qf[2 * c + 1][0], qf[2 * c + 1][1]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          mma16816<false>(se[nt], ha[0], hb[0], ha[1], hb[1], qf[nt][2 * c][0], qf[nt][2 * c][1]);
+          mma16816<false>(so[nt], ha[2], hb[2], ha[3], hb[3], qf[nt][2 * c + 1][0], qf[nt][2 * c + 1][1]);
+        }
       }
     }
     // outlier channels (their codes are 0): S^T += Kout (16 tokens x 4 slots) Qout^T.
@@ -236,43 +259,52 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side, c
       const uint32_t kw = *reinterpret_cast<const uint32_t*>(side + Gm::kScaleBytes + Gm::kValBytes);  // K idx
       const uint32_t* kv = reinterpret_cast<const uint32_t*>(side + Gm::kScaleBytes);  // K vals [16][4] fp16
       if (kw != ost.kidx) {  // same for the whole warp
-        uint32_t b0 = 0;
-        if (qd < 2) {
-          const int r0i = (kw >> (16 * qd)) & 0xFF, r1i = (kw >> (16 * qd + 8)) & 0xFF;
-          const uint32_t q0 = (r0i < D) ? wq[g * Gm::kQStride + r0i] : 0u;
-          const uint32_t q1 = (r1i < D) ? wq[g * Gm::kQStride + r1i] : 0u;
-          b0 = q0 | (q1 << 16);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t b0 = 0;
+          if (qd < 2) {
+            const int r0i = (kw >> (16 * qd)) & 0xFF, r1i = (kw >> (16 * qd + 8)) & 0xFF;
+            const uint16_t* row = wq + (8 * nt + g) * Gm::kQStride;
+            const uint32_t q0 = (r0i < D) ? row[r0i] : 0u;
+            const uint32_t q1 = (r1i < D) ? row[r1i] : 0u;
+            b0 = q0 | (q1 << 16);
+          }
+          ost.kq[nt] = b0;
         }
         ost.kidx = kw;
-        ost.kq = b0;
       }
       const uint32_t a0 = (qd < 2) ? kv[g * 2 + qd] : 0u;
       const uint32_t a1 = (qd < 2) ? kv[(g + 8) * 2 + qd] : 0u;
-      mma16816<false>(so, a0, a1, 0u, 0u, ost.kq, 0u);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma16816<false>(so[nt], a0, a1, 0u, 0u, ost.kq[nt], 0u);
     }
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) sc[i] = se[i] + so[i];
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sc[nt][i] = se[nt][i] + so[nt][i];
 }
 
 // ---------------------------------------------------------------------------
-// O^T (D x 8 query heads) += V^T P^T for one block. P^T arrives as two B
-// fragments (hi and lo parts, P = P_hi + P_lo rounded to the operand type).
+// O^T (D x 8 NT query rows) += V^T P^T for one block. P^T arrives per column
+// tile as two B fragments (hi and lo parts, P = P_hi + P_lo rounded to the
+// operand type); the V fragments are dequantized once for all tiles.
 // ---------------------------------------------------------------------------
-template <int KVF, int D>
+template <int KVF, int D, int NT>
 __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const LdsmOffsets<KVF, D>& lo, int lane,
-                                         int valid, uint32_t b0, uint32_t b1, uint32_t c0, uint32_t c1,
-                                         float (&acc)[D / 16][4], float* oext, OutlierState& ost) {
-  using Gm = DecodeGeom<KVF, D>;
+                                         int valid, const uint32_t (&b0)[NT], const uint32_t (&b1)[NT],
+                                         const uint32_t (&c0)[NT], const uint32_t (&c1)[NT],
+                                         float (&acc)[NT][D / 16][4], float* oext, OutlierState<NT>& ost) {
+  using Gm = DecodeGeom<KVF, D, NT>;
   constexpr int KT = D / 16;
   constexpr bool kBf = (KVF == PQKV_DTYPE_BF16);
   const int g = lane >> 2, qd = lane & 3;
   const int t0 = 2 * qd, t1 = 2 * qd + 8;
   // FP4 keeps P in f16 only (its tolerance allows it); the others add P_lo.
   constexpr bool kSplitP = !Gm::kFp4;
-  auto mma_pv = [&](float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
-    mma16816<kBf>(d, a0, a1, a2, a3, b0, b1);
-    if constexpr (kSplitP) mma16816<kBf>(d, a0, a1, a2, a3, c0, c1);
+  auto mma_pv = [&](int nt, float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3) {
+    mma16816<kBf>(d, a0, a1, a2, a3, b0[nt], b1[nt]);
+    if constexpr (kSplitP) mma16816<kBf>(d, a0, a1, a2, a3, c0[nt], c1[nt]);
   };
   if constexpr (Gm::k16) {
 #pragma unroll
@@ -285,7 +317,8 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
         a2 = mask_pair(a2, t1, valid);
         a3 = mask_pair(a3, t1, valid);
       }
-      mma_pv(acc[mt], a0, a1, a2, a3);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_pv(nt, acc[nt][mt], a0, a1, a2, a3);
     }
   } else if constexpr (Gm::kFp8) {
     // ldmatrix.trans on byte data: lane (g, qd) receives d0 = 16c + 2g and d0 + 1
@@ -307,7 +340,8 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
           a2 = mask_pair(a2, t1, valid);
           a3 = mask_pair(a3, t1, valid);
         }
-        mma_pv(acc[2 * cp + e], a0, a1, a2, a3);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma_pv(nt, acc[nt][2 * cp + e], a0, a1, a2, a3);
       }
     }
   } else {
@@ -343,10 +377,15 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
         const int c = 4 * i + e;
         uint32_t a[4];
         dec_e2m1x8(r[e], a);
-        const __half2 p0 = __hmul2(*reinterpret_cast<const __half2*>(&b0), *reinterpret_cast<const __half2*>(&sp[0][c]));
-        const __half2 p1 = __hmul2(*reinterpret_cast<const __half2*>(&b1), *reinterpret_cast<const __half2*>(&sp[1][c]));
-        mma16816<false>(acc[c], a[0], a[1], a[2], a[3], *reinterpret_cast<const uint32_t*>(&p0),
-                        *reinterpret_cast<const uint32_t*>(&p1));
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const __half2 p0 =
+              __hmul2(*reinterpret_cast<const __half2*>(&b0[nt]), *reinterpret_cast<const __half2*>(&sp[0][c]));
+          const __half2 p1 =
+              __hmul2(*reinterpret_cast<const __half2*>(&b1[nt]), *reinterpret_cast<const __half2*>(&sp[1][c]));
+          mma16816<false>(acc[nt][c], a[0], a[1], a[2], a[3], *reinterpret_cast<const uint32_t*>(&p0),
+                          *reinterpret_cast<const uint32_t*>(&p1));
+        }
       }
     }
     // outlier channels: Oext[n][idx_r] += (Vout^T (4 slots x 16 tokens) P^T)[r][n].
@@ -371,7 +410,8 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
           a2 = mask_pair(a2, t1, valid);
         }
       }
-      mma_pv(ost.vacc, a0, 0u, a2, 0u);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_pv(nt, ost.vacc[nt], a0, 0u, a2, 0u);
     }
   }
 }
@@ -495,11 +535,12 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
   for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
 }
 
-template <int KVF, int D, bool QBF16>
-__global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
+template <int KVF, int D, bool QBF16, int NT>
+__global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p) {
-  using Gm = DecodeGeom<KVF, D>;
-  using Sm = DecodeSmem<KVF, D>;
+  using Gm = DecodeGeom<KVF, D, NT>;
+  using Sm = DecodeSmem<KVF, D, NT>;
+  constexpr int NC = Gm::kCols;  // MMA columns (query rows of one KV head) per warp
   constexpr int NW = Gm::kWarps;
   asm volatile("griddepcontrol.wait;" ::: "memory");  // inputs may come from the previous kernel
   constexpr int NS = Gm::kStages;
@@ -520,16 +561,23 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
   const int B = p.B, Hkv = p.Hkv, G = p.G, Hq = p.Hq;
   const int g = lane >> 2, qd = lane & 3;
   // multi-query: positions at the end of the sequence hidden from this lane's
-  // two columns (query token q0 + c / Gh of k sits k - 1 - q0 - c / Gh before the end)
-  const int hid0 = (2 * qd < G) ? p.k - 1 - p.q0 - (2 * qd) / p.Gh : 0;
-  const int hid1 = (2 * qd + 1 < G) ? p.k - 1 - p.q0 - (2 * qd + 1) / p.Gh : 0;
+  // columns n = 8nt + 2qd + c (query token q0 + n / Gh of k sits k - 1 - q0 -
+  // n / Gh before the end)
+  int hid[NT][2];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int c = 0; c < 2; ++c) {
+      const int n = 8 * nt + 2 * qd + c;
+      hid[nt][c] = (n < G) ? p.k - 1 - p.q0 - n / p.Gh : 0;
+    }
   uint64_t* wbar = bars + warp * NS;
   uint8_t* wtile = tiles + warp * NS * Gm::kTile;
   uint8_t* wside = sides + warp * NS * Gm::kSideStride;
-  uint16_t* wq = qcopy + warp * 8 * Gm::kQStride;
-  float* woext = oext_all + warp * 8 * Gm::kOStride;  // FP4: O of outlier channels [8 heads][D (+pad)]
+  uint16_t* wq = qcopy + warp * NC * Gm::kQStride;
+  float* woext = oext_all + warp * NC * Gm::kOStride;  // FP4: O of outlier channels [NC rows][D (+pad)]
   if constexpr (Gm::kFp4)
-    for (int i = lane; i < 8 * Gm::kOStride; i += 32) woext[i] = 0.f;
+    for (int i = lane; i < NC * Gm::kOStride; i += 32) woext[i] = 0.f;
   const LdsmOffsets<KVF, D> lofs(lane);
 
   if (lane == 0) {
@@ -668,26 +716,31 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     int nblk = P[b + 1] - P[b];
     int Lb = p.seq_lens[b];
     bool started_before = j > 0;
-    uint32_t qf[KT][2];
-    float acc[KT][4];
-    float m0, m1, l0, l1, vref;
-    OutlierState ost;  // FP4 only
+    uint32_t qf[NT][KT][2];
+    float acc[NT][KT][4];
+    float mm[NT][2], ll[NT][2], vref;  // running max and sum of each of the lane's columns
+    OutlierState<NT> ost;  // FP4 only
 
     auto begin_piece = [&]() {
-      m0 = m1 = kNegInf;
-      l0 = l1 = 0.f;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        mm[nt][0] = mm[nt][1] = kNegInf;
+        ll[nt][0] = ll[nt][1] = 0.f;
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
+      }
       vref = 0.f;
       ost.reset();  // the query changes with the piece
 #pragma unroll
-      for (int mt = 0; mt < KT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-      const bool has = g < G;
-      const size_t qrow = has ? col_row(b, h, g, p.k, p.q0, p.Gh, Hq, D) : 0;
+      for (int nt = 0; nt < NT; ++nt) {
+      const bool has = 8 * nt + g < G;
+      const size_t qrow = has ? col_row(b, h, 8 * nt + g, p.k, p.q0, p.Gh, Hq, D) : 0;
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
         if constexpr (Gm::k16) {
           const uint32_t* q32 = reinterpret_cast<const uint32_t*>(p.q);
-          qf[kk][0] = has ? __ldg(q32 + (qrow + 16 * kk + 2 * qd) / 2) : 0u;
-          qf[kk][1] = has ? __ldg(q32 + (qrow + 16 * kk + 8 + 2 * qd) / 2) : 0u;
+          qf[nt][kk][0] = has ? __ldg(q32 + (qrow + 16 * kk + 2 * qd) / 2) : 0u;
+          qf[nt][kk][1] = has ? __ldg(q32 + (qrow + 16 * kk + 8 + 2 * qd) / 2) : 0u;
         } else {
           // k-slot order of the dequantized K fragments: FP8 k-step kk holds
           // d = 16kk + 4qd + {0,1 | 2,3}; FP4 k-step (c, s) = (kk/2, kk%2) holds
@@ -700,14 +753,15 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
             v2 = q_at<QBF16>(p.q, qrow + d0 + 2);
             v3 = q_at<QBF16>(p.q, qrow + d0 + 3);
           }
-          qf[kk][0] = f16x2_from(v0, v1);
-          qf[kk][1] = f16x2_from(v2, v3);
+          qf[nt][kk][0] = f16x2_from(v0, v1);
+          qf[nt][kk][1] = f16x2_from(v2, v3);
         }
+      }
       }
       if constexpr (Gm::kFp4) {
         // f16 copy of this warp's query rows for the outlier channels
         __syncwarp();
-        for (int i = lane; i < 8 * D; i += 32) {
+        for (int i = lane; i < NC * D; i += 32) {
           const int n = i / D;
           const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.q0, p.Gh, Hq, D) + (i % D)) : 0.f;
           wq[n * Gm::kQStride + i % D] = __half_as_ushort(__float2half_rn(v));
@@ -717,41 +771,51 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
     };
 
     auto finish_piece = [&](bool ends_after) {
-      float lt0 = l0, lt1 = l1;
+      float lt[NT][2];
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        lt0 += __shfl_xor_sync(kFull, lt0, o);
-        lt1 += __shfl_xor_sync(kFull, lt1, o);
+      for (int nt = 0; nt < NT; ++nt) {
+        lt[nt][0] = ll[nt][0];
+        lt[nt][1] = ll[nt][1];
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          lt[nt][0] += __shfl_xor_sync(kFull, lt[nt][0], o);
+          lt[nt][1] += __shfl_xor_sync(kFull, lt[nt][1], o);
+        }
       }
       const float vs = Gm::kFp8 ? vref : 1.f;
-      const int n0 = 2 * qd, n1 = 2 * qd + 1;
       if constexpr (Gm::kFp4) {  // fold the outlier channels' O in and clear it
         ost.template flush<Gm::kOStride>(woext, lane, D);
 #pragma unroll
-        for (int mt = 0; mt < KT; ++mt)
+        for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            float* slot = woext + (2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1));
-            acc[mt][e] += *slot;
-            *slot = 0.f;
-          }
+          for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float* slot = woext + (8 * nt + 2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1));
+              acc[nt][mt][e] += *slot;
+              *slot = 0.f;
+            }
         __syncwarp();
       }
       if (!started_before && !ends_after) {
-        const float i0 = lt0 > 0.f ? vs / lt0 : 0.f;
-        const float i1 = lt1 > 0.f ? vs / lt1 : 0.f;
-        const size_t ob0 = n0 < G ? col_row(b, h, n0, p.k, p.q0, p.Gh, Hq, D) : 0;
-        const size_t ob1 = n1 < G ? col_row(b, h, n1, p.k, p.q0, p.Gh, Hq, D) : 0;
 #pragma unroll
-        for (int mt = 0; mt < KT; ++mt) {
-          const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
-          if (n0 < G) {
-            store_out<QBF16>(p.out, ob0 + da, acc[mt][0] * i0);
-            store_out<QBF16>(p.out, ob0 + db, acc[mt][2] * i0);
-          }
-          if (n1 < G) {
-            store_out<QBF16>(p.out, ob1 + da, acc[mt][1] * i1);
-            store_out<QBF16>(p.out, ob1 + db, acc[mt][3] * i1);
+        for (int nt = 0; nt < NT; ++nt) {
+          const int n0 = 8 * nt + 2 * qd, n1 = n0 + 1;
+          const float i0 = lt[nt][0] > 0.f ? vs / lt[nt][0] : 0.f;
+          const float i1 = lt[nt][1] > 0.f ? vs / lt[nt][1] : 0.f;
+          const size_t ob0 = n0 < G ? col_row(b, h, n0, p.k, p.q0, p.Gh, Hq, D) : 0;
+          const size_t ob1 = n1 < G ? col_row(b, h, n1, p.k, p.q0, p.Gh, Hq, D) : 0;
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
+            if (n0 < G) {
+              store_out<QBF16>(p.out, ob0 + da, acc[nt][mt][0] * i0);
+              store_out<QBF16>(p.out, ob0 + db, acc[nt][mt][2] * i0);
+            }
+            if (n1 < G) {
+              store_out<QBF16>(p.out, ob1 + da, acc[nt][mt][1] * i1);
+              store_out<QBF16>(p.out, ob1 + db, acc[nt][mt][3] * i1);
+            }
           }
         }
         return;
@@ -759,25 +823,29 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       const int slot = started_before ? 2 * k : 2 * k + 1;
       float* base = p.partials + (size_t)slot * p.slot_floats;
 #pragma unroll
-      for (int mt = 0; mt < KT; ++mt) {
-        const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
-        if (n0 < G) {
-          base[n0 * D + da] = acc[mt][0] * vs;
-          base[n0 * D + db] = acc[mt][2] * vs;
+      for (int nt = 0; nt < NT; ++nt) {
+        const int n0 = 8 * nt + 2 * qd, n1 = n0 + 1;
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) {
+          const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
+          if (n0 < G) {
+            base[n0 * D + da] = acc[nt][mt][0] * vs;
+            base[n0 * D + db] = acc[nt][mt][2] * vs;
+          }
+          if (n1 < G) {
+            base[n1 * D + da] = acc[nt][mt][1] * vs;
+            base[n1 * D + db] = acc[nt][mt][3] * vs;
+          }
         }
-        if (n1 < G) {
-          base[n1 * D + da] = acc[mt][1] * vs;
-          base[n1 * D + db] = acc[mt][3] * vs;
-        }
-      }
-      if (g == 0) {
-        if (n0 < G) {
-          base[G * D + n0] = m0;
-          base[G * D + G + n0] = lt0;
-        }
-        if (n1 < G) {
-          base[G * D + n1] = m1;
-          base[G * D + G + n1] = lt1;
+        if (g == 0) {
+          if (n0 < G) {
+            base[G * D + n0] = mm[nt][0];
+            base[G * D + G + n0] = lt[nt][0];
+          }
+          if (n1 < G) {
+            base[G * D + n1] = mm[nt][1];
+            base[G * D + G + n1] = lt[nt][1];
+          }
         }
       }
     };
@@ -812,9 +880,13 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       const uint8_t* sdB = wside + sB * Gm::kSideStride;
 
       // ---- scores of both blocks (independent MMA chains) ----
-      float scA[4] = {0.f, 0.f, 0.f, 0.f}, scB[4] = {0.f, 0.f, 0.f, 0.f};
-      if (useA) block_scores<KVF, D>(tbA, sdA, qf, wq, lofs, lane, scA, ost);
-      if (useB) block_scores<KVF, D>(tbB, sdB, qf, wq, lofs, lane, scB, ost);
+      float scA[NT][4], scB[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) scA[nt][e] = scB[nt][e] = 0.f;
+      if (useA) block_scores<KVF, D, NT>(tbA, sdA, qf, wq, lofs, lane, scA, ost);
+      if (useB) block_scores<KVF, D, NT>(tbB, sdB, qf, wq, lofs, lane, scB, ost);
       float skA = 1.f, skB = 1.f, svA = 1.f, svB = 1.f;
       if constexpr (Gm::kFp8) {
         if (useA) { skA = reinterpret_cast<const float*>(sdA)[0]; svA = reinterpret_cast<const float*>(sdA)[1]; }
@@ -822,34 +894,44 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       }
 
       // ---- online softmax over up to 32 tokens (log2 domain) ----
+      // x[nt][e]: row (token) g + 8 (e >> 1), column 8nt + 2qd + (e & 1)
       const float mA = p.scale_log2 * skA, mB = p.scale_log2 * skB;
-      float xA0 = scA[0] * mA, xA1 = scA[1] * mA, xA2 = scA[2] * mA, xA3 = scA[3] * mA;
-      float xB0 = scB[0] * mB, xB1 = scB[1] * mB, xB2 = scB[2] * mB, xB3 = scB[3] * mB;
-      // column n sees the tokens before the last hid_n ones (0 for one query token)
-      if (!useA || g >= remA - hid0) xA0 = kNegInf;
-      if (!useA || g >= remA - hid1) xA1 = kNegInf;
-      if (!useA || g + 8 >= remA - hid0) xA2 = kNegInf;
-      if (!useA || g + 8 >= remA - hid1) xA3 = kNegInf;
-      if (!useB || g >= remB - hid0) xB0 = kNegInf;
-      if (!useB || g >= remB - hid1) xB1 = kNegInf;
-      if (!useB || g + 8 >= remB - hid0) xB2 = kNegInf;
-      if (!useB || g + 8 >= remB - hid1) xB3 = kNegInf;
-      float bm0 = fmaxf(fmaxf(xA0, xA2), fmaxf(xB0, xB2));
-      float bm1 = fmaxf(fmaxf(xA1, xA3), fmaxf(xB1, xB3));
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        bm0 = fmaxf(bm0, __shfl_xor_sync(kFull, bm0, o));
-        bm1 = fmaxf(bm1, __shfl_xor_sync(kFull, bm1, o));
-      }
+      float xA[NT][4], xB[NT][4], bm[NT][2];
+      bool need_any = false;
       constexpr float kLazy = lazy_of<KVF>();
-      const bool need0 = bm0 > m0 + kLazy, need1 = bm1 > m1 + kLazy;
-      float f0c = 1.f, f1c = 1.f;
-      bool rescale = __any_sync(kFull, need0 || need1);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = g + 8 * (e >> 1), hd = hid[nt][e & 1];
+          // column n sees the tokens before the last hid ones (0 for one query token)
+          xA[nt][e] = (!useA || r >= remA - hd) ? kNegInf : scA[nt][e] * mA;
+          xB[nt][e] = (!useB || r >= remB - hd) ? kNegInf : scB[nt][e] * mB;
+        }
+        bm[nt][0] = fmaxf(fmaxf(xA[nt][0], xA[nt][2]), fmaxf(xB[nt][0], xB[nt][2]));
+        bm[nt][1] = fmaxf(fmaxf(xA[nt][1], xA[nt][3]), fmaxf(xB[nt][1], xB[nt][3]));
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+          bm[nt][0] = fmaxf(bm[nt][0], __shfl_xor_sync(kFull, bm[nt][0], o));
+          bm[nt][1] = fmaxf(bm[nt][1], __shfl_xor_sync(kFull, bm[nt][1], o));
+        }
+        need_any |= (bm[nt][0] > mm[nt][0] + kLazy) || (bm[nt][1] > mm[nt][1] + kLazy);
+      }
+      float fc[NT][2];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) fc[nt][0] = fc[nt][1] = 1.f;
+      bool rescale = __any_sync(kFull, need_any);
       if (rescale) {
-        if (need0) { f0c = ex2(m0 - bm0); m0 = bm0; }
-        if (need1) { f1c = ex2(m1 - bm1); m1 = bm1; }
-        l0 *= f0c;
-        l1 *= f1c;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            if (bm[nt][c] > mm[nt][c] + kLazy) {
+              fc[nt][c] = ex2(mm[nt][c] - bm[nt][c]);
+              mm[nt][c] = bm[nt][c];
+            }
+            ll[nt][c] *= fc[nt][c];
+          }
       }
       // FP8 V scales: O is kept in units of vref, the largest V scale so far;
       // a block with a smaller scale enters with P scaled by sv / vref <= 1.
@@ -858,8 +940,11 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
         const float svm = fmaxf(useA ? svA : 0.f, useB ? svB : 0.f);
         if (svm > vref) {
           const float rs = vref / svm;
-          f0c *= rs;
-          f1c *= rs;
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            fc[nt][0] *= rs;
+            fc[nt][1] *= rs;
+          }
           vref = svm;
           rescale = true;
         }
@@ -868,48 +953,66 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
       }
       if (rescale) {
 #pragma unroll
-        for (int mt = 0; mt < KT; ++mt) {
-          acc[mt][0] *= f0c;
-          acc[mt][1] *= f1c;
-          acc[mt][2] *= f0c;
-          acc[mt][3] *= f1c;
-        }
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            acc[nt][mt][0] *= fc[nt][0];
+            acc[nt][mt][1] *= fc[nt][1];
+            acc[nt][mt][2] *= fc[nt][0];
+            acc[nt][mt][3] *= fc[nt][1];
+          }
         if constexpr (Gm::kFp4) {  // the outlier channels' O follows the same rescale
-          ost.vacc[0] *= f0c;
-          ost.vacc[1] *= f1c;
           __syncwarp();
 #pragma unroll
-          for (int mt = 0; mt < KT; ++mt)
+          for (int nt = 0; nt < NT; ++nt) {
+            ost.vacc[nt][0] *= fc[nt][0];
+            ost.vacc[nt][1] *= fc[nt][1];
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              woext[(2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1))] *= (e & 1) ? f1c : f0c;
+            for (int mt = 0; mt < KT; ++mt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                woext[(8 * nt + 2 * qd + (e & 1)) * Gm::kOStride + dmap<KVF>(mt, g + 8 * (e >> 1))] *=
+                    fc[nt][e & 1];
+          }
           __syncwarp();
         }
       }
-      const bool live0 = m0 != kNegInf, live1 = m1 != kNegInf;
-      const float pA0 = live0 ? ex2(xA0 - m0) : 0.f, pA2 = live0 ? ex2(xA2 - m0) : 0.f;
-      const float pA1 = live1 ? ex2(xA1 - m1) : 0.f, pA3 = live1 ? ex2(xA3 - m1) : 0.f;
-      const float pB0 = live0 ? ex2(xB0 - m0) : 0.f, pB2 = live0 ? ex2(xB2 - m0) : 0.f;
-      const float pB1 = live1 ? ex2(xB1 - m1) : 0.f, pB3 = live1 ? ex2(xB3 - m1) : 0.f;
-      l0 += (pA0 + pA2) + (pB0 + pB2);
-      l1 += (pA1 + pA3) + (pB1 + pB3);
+      float pA[NT][4], pB[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float mc = mm[nt][e & 1];
+          const bool live = mc != kNegInf;
+          pA[nt][e] = live ? ex2(xA[nt][e] - mc) : 0.f;
+          pB[nt][e] = live ? ex2(xB[nt][e] - mc) : 0.f;
+        }
+        ll[nt][0] += (pA[nt][0] + pA[nt][2]) + (pB[nt][0] + pB[nt][2]);
+        ll[nt][1] += (pA[nt][1] + pA[nt][3]) + (pB[nt][1] + pB[nt][3]);
+      }
 
       // ---- O^T += V^T P^T; P = P_hi + P_lo (except FP4) so ~16 significant bits survive ----
-      auto pv = [&](uint32_t tb, const uint8_t* sd, int valid, float w0, float w1, float w2, float w3) {
-        const uint32_t hA = pack_f32x2(w0, w1, kBf16Mma), hB = pack_f32x2(w2, w3, kBf16Mma);
-        if constexpr (Gm::kFp4) {
-          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), 0u, 0u, acc, woext, ost);
-        } else {
-          const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
-          const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
-          block_pv<KVF, D>(tb, sd, lofs, lane, valid, movmatrix_t(hA), movmatrix_t(hB), movmatrix_t(lA),
-                           movmatrix_t(lB), acc, woext, ost);
+      auto pv = [&](uint32_t tb, const uint8_t* sd, int valid, const float (&w)[NT][4], float pr) {
+        uint32_t b0[NT], b1[NT], c0[NT], c1[NT];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const float w0 = w[nt][0] * pr, w1 = w[nt][1] * pr, w2 = w[nt][2] * pr, w3 = w[nt][3] * pr;
+          const uint32_t hA = pack_f32x2(w0, w1, kBf16Mma), hB = pack_f32x2(w2, w3, kBf16Mma);
+          b0[nt] = movmatrix_t(hA);
+          b1[nt] = movmatrix_t(hB);
+          if constexpr (Gm::kFp4) {
+            c0[nt] = c1[nt] = 0u;
+          } else {
+            const uint32_t lA = pack_f32x2(w0 - unpack_lo(hA, kBf16Mma), w1 - unpack_hi(hA, kBf16Mma), kBf16Mma);
+            const uint32_t lB = pack_f32x2(w2 - unpack_lo(hB, kBf16Mma), w3 - unpack_hi(hB, kBf16Mma), kBf16Mma);
+            c0[nt] = movmatrix_t(lA);
+            c1[nt] = movmatrix_t(lB);
+          }
         }
+        block_pv<KVF, D, NT>(tb, sd, lofs, lane, valid, b0, b1, c0, c1, acc, woext, ost);
       };
-      if (useA && (!Gm::kFp8 || prA > 0.f))
-        pv(tbA, sdA, validA, pA0 * prA, pA1 * prA, pA2 * prA, pA3 * prA);
-      if (useB && (!Gm::kFp8 || prB > 0.f))
-        pv(tbB, sdB, validB, pB0 * prB, pB1 * prB, pB2 * prB, pB3 * prB);
+      if (useA && (!Gm::kFp8 || prA > 0.f)) pv(tbA, sdA, validA, pA, prA);
+      if (useB && (!Gm::kFp8 || prB > 0.f)) pv(tbB, sdB, validB, pB, prB);
 
       __syncwarp();
       if (f + NS < f1) issue(sA, f + NS);
@@ -948,10 +1051,10 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D>::kWarps * 32, 1)
 
 // ---- instantiation + launch --------------------------------------------------
 
-template <int KVF, int D, bool QBF16>
+template <int KVF, int D, bool QBF16, int NT>
 static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& p, int grid, cudaStream_t st) {
-  auto kern = paged_decode_kernel<KVF, D, QBF16>;
-  const size_t smem = DecodeSmem<KVF, D>::bytes(p.B);
+  auto kern = paged_decode_kernel<KVF, D, QBF16, NT>;
+  const size_t smem = DecodeSmem<KVF, D, NT>::bytes(p.B);
   // opt in once per device to the largest size any batch can need
   static std::atomic<uint64_t> configured{0};
   int dev = 0;
@@ -959,7 +1062,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
   const uint64_t bit = 1ull << (dev & 63);
   if (!(configured.load() & bit)) {
     const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               (int)DecodeSmem<KVF, D>::bytes(PQKV_MAX_BATCH));
+                                               (int)DecodeSmem<KVF, D, NT>::bytes(PQKV_MAX_BATCH));
     if (e != cudaSuccess) return e;
     configured.fetch_or(bit);
   }
@@ -968,7 +1071,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
   // only the launch overlaps
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(DecodeGeom<KVF, D>::kWarps * 32);
+  cfg.blockDim = dim3(DecodeGeom<KVF, D, NT>::kWarps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -1003,36 +1106,53 @@ cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t 
                 : cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, false>, p);
 }
 
-int decode_warps(int kv_dtype, int D) {
+// nt = tiles of 8 MMA columns per warp (1, or 2 for up to 16 query rows per KV head)
+template <int NT>
+static int decode_warps_t(int kv_dtype, int D) {
   switch (kv_dtype) {
     case PQKV_DTYPE_FP16:
     case PQKV_DTYPE_BF16:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_BF16, 128>::kWarps : DecodeGeom<PQKV_DTYPE_BF16, 64>::kWarps;
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_BF16, 128, NT>::kWarps : DecodeGeom<PQKV_DTYPE_BF16, 64, NT>::kWarps;
     case PQKV_DTYPE_FP8_E4M3:
     case PQKV_DTYPE_FP8_E5M2:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP8_E4M3, 128>::kWarps : DecodeGeom<PQKV_DTYPE_FP8_E4M3, 64>::kWarps;
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP8_E4M3, 128, NT>::kWarps
+                      : DecodeGeom<PQKV_DTYPE_FP8_E4M3, 64, NT>::kWarps;
     default:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP4_E2M1, 128>::kWarps : DecodeGeom<PQKV_DTYPE_FP4_E2M1, 64>::kWarps;
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP4_E2M1, 128, NT>::kWarps
+                      : DecodeGeom<PQKV_DTYPE_FP4_E2M1, 64, NT>::kWarps;
   }
 }
 
-size_t decode_smem_bytes(int kv_dtype, int D, int B) {
+int decode_warps(int kv_dtype, int D, int nt) {
+  return nt == 2 ? decode_warps_t<2>(kv_dtype, D) : decode_warps_t<1>(kv_dtype, D);
+}
+
+template <int NT>
+static size_t decode_smem_bytes_t(int kv_dtype, int D, int B) {
   switch (kv_dtype) {
     case PQKV_DTYPE_FP16:
     case PQKV_DTYPE_BF16:
-      return D == 128 ? DecodeSmem<PQKV_DTYPE_BF16, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_BF16, 64>::bytes(B);
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_BF16, 128, NT>::bytes(B) : DecodeSmem<PQKV_DTYPE_BF16, 64, NT>::bytes(B);
     case PQKV_DTYPE_FP8_E4M3:
     case PQKV_DTYPE_FP8_E5M2:
-      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP8_E4M3, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_FP8_E4M3, 64>::bytes(B);
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP8_E4M3, 128, NT>::bytes(B)
+                      : DecodeSmem<PQKV_DTYPE_FP8_E4M3, 64, NT>::bytes(B);
     default:
-      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP4_E2M1, 128>::bytes(B) : DecodeSmem<PQKV_DTYPE_FP4_E2M1, 64>::bytes(B);
+      return D == 128 ? DecodeSmem<PQKV_DTYPE_FP4_E2M1, 128, NT>::bytes(B)
+                      : DecodeSmem<PQKV_DTYPE_FP4_E2M1, 64, NT>::bytes(B);
   }
 }
 
-cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap, const DecodeParams& p,
+size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt) {
+  return nt == 2 ? decode_smem_bytes_t<2>(kv_dtype, D, B) : decode_smem_bytes_t<1>(kv_dtype, D, B);
+}
+
+cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st) {
-#define PQKV_DEC(KVF, DD, QB) \
-  if (kv_dtype == KVF && D == DD && q_bf16 == QB) return launch_decode_t<KVF, DD, QB>(tmap, p, grid, st);
+#define PQKV_DEC(KVF, DD, QB)                                                                        \
+  if (kv_dtype == KVF && D == DD && q_bf16 == QB)                                                    \
+    return nt == 2 ? launch_decode_t<KVF, DD, QB, 2>(tmap, p, grid, st)                              \
+                   : launch_decode_t<KVF, DD, QB, 1>(tmap, p, grid, st);
   PQKV_DEC(PQKV_DTYPE_FP16, 128, false)
   PQKV_DEC(PQKV_DTYPE_FP16, 64, false)
   PQKV_DEC(PQKV_DTYPE_BF16, 128, true)

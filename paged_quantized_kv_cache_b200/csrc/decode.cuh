@@ -67,8 +67,9 @@ struct MergeParams {
   int slot_floats;
 };
 
-// Compile-time geometry of one format.
-template <int KVF, int D>
+// Compile-time geometry of one format; NT = tiles of 8 MMA columns (query rows)
+// per KV head: 1, or 2 for multi-query decode with up to 16 rows.
+template <int KVF, int D, int NT = 1>
 struct DecodeGeom {
   static constexpr bool k16 = (KVF == PQKV_DTYPE_FP16 || KVF == PQKV_DTYPE_BF16);
   static constexpr bool kFp8 = (KVF == PQKV_DTYPE_FP8_E4M3 || KVF == PQKV_DTYPE_FP8_E5M2);
@@ -84,7 +85,9 @@ struct DecodeGeom {
   static constexpr int kSideStride = kSide == 0 ? 0 : ((kSide + 127) / 128) * 128;
   // Warps per CTA and shared-memory stages per warp (even: blocks are consumed
   // in pairs while the next pair is in flight); about 192 KB of stages per SM.
-  static constexpr int kWarps = k16 ? (D == 128 ? 6 : 8) : 12;
+  // (two column tiles double the accumulators: quantized formats drop to 8 warps)
+  static constexpr int kWarps = k16 ? (D == 128 ? 6 : 8) : (NT == 1 ? 12 : 8);
+  static constexpr int kCols = 8 * NT;                          // MMA columns per KV head
   static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 4 : 6) : (D == 128 ? 4 : 6));
   static constexpr uint32_t kTx = kTile + kSide;
   // FP4 per-warp shared rows, padded so that the 8 rows fall in different banks
@@ -102,14 +105,14 @@ struct DecodeGeom {
   }
 };
 
-template <int KVF, int D>
+template <int KVF, int D, int NT = 1>
 struct DecodeSmem {
-  using Gm = DecodeGeom<KVF, D>;
+  using Gm = DecodeGeom<KVF, D, NT>;
   static constexpr int kTilesBytes = Gm::kWarps * Gm::kStages * Gm::kTile;
   static constexpr int kSideBytes = Gm::kWarps * Gm::kStages * Gm::kSideStride;
   static constexpr int kBarBytes = Gm::kWarps * Gm::kStages * 8;
-  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * 8 * Gm::kQStride * 2 : 0;     // per-warp f16 q copy
-  static constexpr int kOextBytes = Gm::kFp4 ? Gm::kWarps * 8 * Gm::kOStride * 4 : 0;  // per-warp outlier-channel O
+  static constexpr int kQBytes = Gm::kFp4 ? Gm::kWarps * Gm::kCols * Gm::kQStride * 2 : 0;     // per-warp f16 q copy
+  static constexpr int kOextBytes = Gm::kFp4 ? Gm::kWarps * Gm::kCols * Gm::kOStride * 4 : 0;  // outlier-channel O
   static size_t bytes(int B) {
     return 1024 + (size_t)kTilesBytes + kSideBytes + kBarBytes + kQBytes + kOextBytes + (size_t)(B + 1) * 4;
   }

@@ -2,8 +2,9 @@
 "Speculative decoding") against the oracle: each sequence's last q_len
 positions attend causally, which is the oracle's chunked prefill with chunks
 of q_len tokens. The decode kernels put the q_len x G query rows of a KV head in
-the columns of one tensor-core tile (several passes when q_len x G > 8);
-q_len = 1 must reproduce pqkv_paged_decode_attention bit for bit."""
+the columns of one or two 8-column tensor-core tiles (several passes when
+q_len x G > 16); q_len = 1 must reproduce pqkv_paged_decode_attention bit for
+bit."""
 import numpy as np
 import pytest
 import torch
@@ -25,10 +26,17 @@ CASES = [
     (pq.FP8_E5M2, torch.float16, 64, 16, 8, 4, 0),
     (pq.FP4_E2M1, torch.bfloat16, 128, 32, 8, 2, 0),
     (pq.FP4_E2M1, torch.float16, 64, 8, 4, 3, 2),
-    # more query tokens than one tile's 8 columns: several passes over the KV
+    # 9..16 query rows per KV head: one pass with two column tiles
     (pq.BF16, torch.bfloat16, 128, 32, 8, 4, 0),
+    (pq.FP16, torch.float16, 64, 8, 8, 16, 0),
+    (pq.BF16, torch.bfloat16, 128, 24, 8, 5, 2),     # G = 3: 15 rows, the second tile part-filled
+    (pq.FP8_E5M2, torch.float16, 64, 16, 8, 8, 0),
+    (pq.FP4_E2M1, torch.bfloat16, 128, 32, 8, 4, 0),
+    (pq.FP4_E2M1, torch.float16, 64, 32, 4, 2, 2),
+    # more rows than two tiles hold: several passes over the KV, the last one narrower
     (pq.FP8_E4M3, torch.bfloat16, 128, 32, 8, 5, 3),
     (pq.FP4_E2M1, torch.bfloat16, 64, 32, 4, 3, 0),
+    (pq.BF16, torch.bfloat16, 128, 32, 8, 11, 0),
 ]
 
 
@@ -57,8 +65,7 @@ def _build(kv_dtype, qdt, D, Hq, Hkv, k, lens, seed):
 def _mq(g, q, bt, lens, scale, split=0):
     B, k, Hq, D = q.shape
     out = torch.full_like(q.cuda(), float("nan"))
-    kp = min(k, max(1, 8 // (Hq // g.num_kv_heads)))  # query tokens per pass
-    ws = pq.decode_workspace(B, Hq * kp, g.num_kv_heads, D, bt.shape[1], split)
+    ws = pq.multi_query_decode_workspace(B, k, Hq, g.num_kv_heads, D, bt.shape[1], split)
     ws.fill_(0xAB)
     e = gh.err_flag()
     pq.paged_multi_query_decode_attention(q.cuda(), g, torch.from_numpy(np.ascontiguousarray(bt, np.int32)).cuda(),
@@ -71,7 +78,7 @@ def _mq(g, q, bt, lens, scale, split=0):
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "kv%d-D%d-G%d-k%d-s%d" % (c[0], c[2], c[3] // c[4], c[5], c[6]))
 def test_multi_query_decode_matches_oracle(case):
     kv_dtype, qdt, D, Hq, Hkv, k, split = case
-    lens = [37, 200, 16, 1000, 9]
+    lens = [max(L, k) for L in (37, 200, 16, 1000, 9)]  # each sequence holds its q_len query tokens
     g, o, bt, q = _build(kv_dtype, qdt, D, Hq, Hkv, k, lens, seed=70 + kv_dtype + k)
     scale = 1.0 / np.sqrt(D)
     out, err = _mq(g, q, bt, lens, scale, split)
@@ -105,8 +112,8 @@ def test_sequence_shorter_than_its_query_tokens_and_limits():
     gh.assert_close(out[keep].reshape(-1, Hq, D), ref, kv_dtype, tag="valid sequences")
     # more than 64 query tokens, or a workspace sized for too few columns, is
     # rejected before anything runs
-    ws = pq.decode_workspace(1, 8, 4, 64, bt.shape[1])
-    for kq, w in ((65, pq.decode_workspace(1, 8 * 4, 4, 64, bt.shape[1])), (4, ws[:16])):
+    ws = pq.multi_query_decode_workspace(1, 4, 8, 4, 64, bt.shape[1])
+    for kq, w in ((65, ws), (4, ws[:16])):
         big = torch.zeros((1, kq, 8, 64), dtype=torch.float16, device="cuda")
         with pytest.raises(pq.PqkvError):
             pq.paged_multi_query_decode_attention(big, g, torch.from_numpy(bt[:1].copy()).cuda(),
