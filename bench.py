@@ -580,8 +580,8 @@ def run_ours(args) -> None:
             "decode_tok_s_per_layer": tok_s,
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            # per step: cache write, then per decode pass a split decode and its log-sum-exp merge
-            "gpu_launches": (1 + 2 * decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
+            # per step: cache write, then one decode kernel per pass (split pairs merged inside it)
+            "gpu_launches": (1 + decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

@@ -186,10 +186,13 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
  * GPU; > 0 = process the KV of all (sequence, head) pairs, laid end to end, in
  * chunks of exactly that many 16-token blocks. Results differ only by rounding.
  * workspace: device buffer of at least pqkv_decode_workspace_bytes(...) bytes,
- * scratch for the split pieces (no initialization needed). Two kernels run on
- * `stream`: the split decode, then the log-sum-exp merge of split pairs
- * (launched as a programmatic dependent of the first). Calls that share a
- * workspace must be ordered. batch <= PQKV_MAX_BATCH.
+ * scratch for the split pieces and one arrival word per chunk. One kernel runs
+ * on `stream`; the warp that writes the last piece of a split pair merges the
+ * pieces by log-sum-exp in chunk order. The arrival words carry a 40-bit tag
+ * of the launch, so the buffer needs no clearing between calls; on a buffer's
+ * first use its old bytes could match a tag with probability 2^-40 per split
+ * pair, which pqkv_decode_workspace_init (zero fill) removes. Calls that share
+ * a workspace must be ordered. batch <= PQKV_MAX_BATCH.
  */
 int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads,
                                 const void* cache, const void* scales,
@@ -330,8 +333,9 @@ int pqkv_swap_in(void* cache, void* scales, void* outliers_idx, void* outliers_v
                  const int32_t* block_ids, int num, const void* host_records,
                  int32_t* err_flag, pqkv_stream_t stream);
 
-/* Zero-fill a decode workspace on `stream` (optional; results never depend on
- * the workspace's prior contents). */
+/* Zero-fill a decode workspace on `stream`. Optional: it only removes the
+ * 2^-40 chance per split pair that a never-used buffer's old bytes match a
+ * launch tag (see pqkv_paged_decode_attention). */
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
                                pqkv_stream_t stream);
 

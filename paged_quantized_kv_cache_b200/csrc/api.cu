@@ -2,6 +2,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -13,9 +14,7 @@
 namespace pqkv {
 cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st);
-cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
 size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt);
-int decode_warps(int kv_dtype, int D, int nt);
 }  // namespace pqkv
 
 using namespace pqkv;
@@ -123,9 +122,10 @@ bool cached_cache_map(CUtensorMap* map, const void* cache, int kv_dtype, int nb,
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace = two partial-result slots per chunk of the split, written by the
-// decode kernel before the merge kernel reads them; nothing in it needs to be
-// initialized by the caller.
+// Workspace = two partial-result slots per chunk of the split and one arrival
+// word per chunk, all written by the decode kernel before it reads them (the
+// words carry a per-launch tag); nothing in it needs to be initialized by the
+// caller.
 
 }  // namespace
 
@@ -190,6 +190,23 @@ int pqkv_kv_cache_write(const void* k, const void* v, int in_dtype, int num_toke
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
 }
 
+// Upper bound of the decode's chunks (each has two partial slots and one
+// arrival word in the workspace).
+static size_t decode_chunks(int batch, int num_kv_heads, int max_blocks_per_seq, int split_blocks, int sms) {
+  const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
+  return split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks : (size_t)sms * kDecodeWarps;
+}
+
+// Launch tags of the decode's arrival words: 40 bits, never 0, so a zeroed
+// word never matches.
+static unsigned long long next_decode_epoch() {
+  static std::atomic<unsigned long long> n{0};
+  for (;;) {
+    const unsigned long long e = (n.fetch_add(1) + 1) & ((1ull << 40) - 1);
+    if (e != 0) return e;
+  }
+}
+
 size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads, int head_dim,
                                    int max_blocks_per_seq, int split_blocks) {
   if (batch < 1 || num_kv_heads < 1 || num_q_heads < 1 || num_q_heads % num_kv_heads != 0 ||
@@ -200,10 +217,8 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
   DeviceInfo di;
   if (!device_info(di)) return 0;
   const size_t slot = round_up((size_t)G * head_dim + 2 * G, 4) * 4;
-  const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
-  const size_t chunks = split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks
-                                         : (size_t)di.sms * kDecodeWarps;
-  return 2 * chunks * slot;
+  const size_t chunks = decode_chunks(batch, num_kv_heads, max_blocks_per_seq, split_blocks, di.sms);
+  return 2 * chunks * slot + chunks * sizeof(unsigned long long);  // partial slots, then arrival words
 }
 
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes, pqkv_stream_t stream) {
@@ -286,29 +301,19 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   p.slot_floats = (int)round_up((size_t)Gh * kp * head_dim + 2 * Gh * kp, 4);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
+  // the arrival words follow the partial slots (16-byte aligned: slot_floats is a multiple of 4)
+  const size_t chunks = decode_chunks(batch, num_kv_heads, max_blocks_per_seq, split_blocks, di.sms);
+  p.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
+                                                     2 * chunks * (size_t)p.slot_floats * sizeof(float));
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  MergeParams mp;
-  mp.seq_lens = seq_lens;
-  mp.partials = p.partials;
-  mp.out = out;
-  mp.B = batch;
-  mp.Hq = num_q_heads;
-  mp.Hkv = num_kv_heads;
-  mp.k = p.k;
-  mp.Gh = p.Gh;
-  mp.maxblk = max_blocks_per_seq;
-  mp.split_blocks = split_blocks;
-  mp.slot_floats = p.slot_floats;
   // passes run in stream order; each kernel waits for the previous one before
   // touching the workspace (programmatic dependents wait for the full grid)
   for (int q0 = 0; q0 < q_len; q0 += kp) {
-    p.q0 = mp.q0 = q0;
-    p.G = mp.G = Gh * std::min(kp, q_len - q0);
+    p.q0 = q0;
+    p.G = Gh * std::min(kp, q_len - q0);
+    p.epoch = next_decode_epoch();
     const int nt = p.G > 8 ? 2 : 1;  // tiles of 8 columns
-    mp.warps = di.sms * decode_warps(kv_dtype, head_dim, nt);
-    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
-    if (e != cudaSuccess) return PQKV_ERR_CUDA;
-    e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
+    const cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
     if (e != cudaSuccess) return PQKV_ERR_CUDA;
   }
   return PQKV_OK;

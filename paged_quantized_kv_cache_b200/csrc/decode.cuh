@@ -14,9 +14,9 @@
 // The grid is persistent (one CTA per SM, NW warps each); the flat range is cut
 // into chunks of Q blocks and warp w takes chunks w, w + W, ... (W = all warps).
 // A chunk covers whole pairs (written straight to `out`) and at most two
-// partial pairs at its ends (written to a workspace slot). A second kernel,
-// launched as a programmatic dependent of the first, merges the pieces of each
-// split pair in chunk order, so results do not depend on timing.
+// partial pairs at its ends (written to a workspace slot). The warp that
+// writes the last piece of a split pair (counted in a per-pair arrival word)
+// merges its pieces in chunk order, so results do not depend on timing.
 //
 // Per warp: a private ring of NS shared-memory stages, each holding the K and V
 // tiles of one (block, head) pair fetched by one TMA tensor copy (128/64/32-byte
@@ -44,6 +44,7 @@ struct DecodeParams {
   const int32_t* seq_lens;      // [B]
   int32_t* err;
   float* partials;              // [2 * chunks][slot_floats]
+  unsigned long long* counters; // [chunks] arrival words of split pairs (tag << 24 | pieces)
   // G = MMA columns per KV head = Gh query heads x the query tokens q0,
   // q0 + 1, ... of this pass (column c = token q0 + c / Gh, head c % Gh); k > 1
   // is multi-query decode: token i of a sequence of length L sits at position
@@ -54,17 +55,7 @@ struct DecodeParams {
   int slot_floats;
   float scale_log2;             // softmax scale * log2(e)
   uint64_t timeout_ns;
-};
-
-struct MergeParams {
-  const int32_t* seq_lens;
-  const float* partials;
-  void* out;
-  int B, Hq, Hkv, G, maxblk;
-  int k, Gh, q0;             // as in DecodeParams
-  int warps;         // warps of the decode grid (its balanced chunk length depends on it)
-  int split_blocks;
-  int slot_floats;
+  unsigned long long epoch;     // tag of this launch (40 bits, never 0)
 };
 
 // Compile-time geometry of one format; NT = tiles of 8 MMA columns (query rows)

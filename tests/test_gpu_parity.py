@@ -190,6 +190,35 @@ def test_repeated_calls_are_deterministic_and_reuse_the_workspace():
         assert torch.equal(out, first) and int(e.item()) == 0
 
 
+def test_arrival_words_left_by_other_split_plans_do_not_matter():
+    """Split pairs are merged by the warp whose piece arrives last, counted in
+    per-chunk words of the workspace tagged with the launch. One workspace
+    serves calls with different split plans in turn (so words written under one
+    plan lie under the chunks of the next); every result equals the same call
+    on a fresh zeroed workspace, bit for bit."""
+    case = CASES[4]
+    lens = [1200, 17, 700, 5, 333]
+    g, o, bt, q = _scenario(case, lens, seed=510)
+    bt_d = torch.from_numpy(bt).cuda()
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    qd = q.cuda()
+    plans = (1, 5, 0, 3, 1, 0, 7, 1)
+    shared = torch.zeros(max(pq.decode_workspace_bytes(len(lens), case[3], case[4], case[2], bt.shape[1], s)
+                             for s in plans), dtype=torch.uint8, device="cuda")
+    for split in plans:
+        need = pq.decode_workspace_bytes(len(lens), case[3], case[4], case[2], bt.shape[1], split)
+        fresh = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        a, b = torch.empty_like(qd), torch.empty_like(qd)
+        e1, e2 = gh.err_flag(), gh.err_flag()
+        pq.paged_decode_attention(qd, g, bt_d, sl, 0.1, a, shared, e1, split_blocks=split)
+        pq.paged_decode_attention(qd, g, bt_d, sl, 0.1, b, fresh, e2, split_blocks=split)
+        torch.cuda.synchronize()
+        assert int(e1.item()) == int(e2.item()) == 0
+        assert torch.equal(a, b), "split %d" % split
+    ref, _ = oracle.paged_decode(o, q, bt, np.array(lens, np.int32), 0.1)
+    gh.assert_close(a, ref, case[0])
+
+
 def test_edge_lengths_and_error_bits():
     case = CASES[1]
     kv_dtype, qdt, D, Hq, Hkv = case
