@@ -561,7 +561,7 @@ def run_ours(args) -> None:
                 "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype]),
                 "kernel": "paged_decode_kernel", "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, "
                 "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms,
-                "timing": "CUDA events around each decode call (decode + merge kernels) over K further steps"}
+                "timing": "CUDA events around each decode call (per pass: decode kernel, merge kernel of long split pairs) over K further steps"}
 
     e2e = run_e2e(st, args, world) if not args.no_e2e else None
 
@@ -580,8 +580,9 @@ def run_ours(args) -> None:
             "decode_tok_s_per_layer": tok_s,
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            # per step: cache write, then one decode kernel per pass (split pairs merged inside it)
-            "gpu_launches": (1 + decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
+            # per step: cache write, then per decode pass the split decode and the merge kernel of
+            # long split pairs (short ones are merged inside the decode)
+            "gpu_launches": (1 + 2 * decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
             "clocks": clocks.summary(),
         }
         print(json.dumps(line), flush=True)

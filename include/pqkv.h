@@ -186,13 +186,16 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
  * GPU; > 0 = process the KV of all (sequence, head) pairs, laid end to end, in
  * chunks of exactly that many 16-token blocks. Results differ only by rounding.
  * workspace: device buffer of at least pqkv_decode_workspace_bytes(...) bytes,
- * scratch for the split pieces and one arrival word per chunk. One kernel runs
- * on `stream`; the warp that writes the last piece of a split pair merges the
- * pieces by log-sum-exp in chunk order. The arrival words carry a 40-bit tag
- * of the launch, so the buffer needs no clearing between calls; on a buffer's
- * first use its old bytes could match a tag with probability 2^-40 per split
- * pair, which pqkv_decode_workspace_init (zero fill) removes. Calls that share
- * a workspace must be ordered. batch <= PQKV_MAX_BATCH.
+ * scratch for the split pieces and one arrival word per chunk. Two kernels run
+ * on `stream`: the split decode, whose warp that writes the last piece of a
+ * pair split into at most 4 pieces merges the pieces by log-sum-exp in chunk
+ * order, then (as a programmatic dependent) the merge of pairs split into more
+ * pieces (few long sequences), whose warps exit at once when there are none.
+ * The arrival words carry a 40-bit tag of the launch, so the buffer needs no
+ * clearing between calls; on a buffer's first use its old bytes could match a
+ * tag with probability 2^-40 per split pair, which pqkv_decode_workspace_init
+ * (zero fill) removes. Calls that share a workspace must be ordered.
+ * batch <= PQKV_MAX_BATCH.
  */
 int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads,
                                 const void* cache, const void* scales,

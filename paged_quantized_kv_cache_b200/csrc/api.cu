@@ -15,6 +15,8 @@ namespace pqkv {
 cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st);
 size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt);
+int decode_warps(int kv_dtype, int D, int nt);
+cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
 }  // namespace pqkv
 
 using namespace pqkv;
@@ -306,14 +308,29 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   p.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
                                                      2 * chunks * (size_t)p.slot_floats * sizeof(float));
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MergeParams mp;
+  mp.seq_lens = seq_lens;
+  mp.partials = p.partials;
+  mp.out = out;
+  mp.B = batch;
+  mp.Hq = num_q_heads;
+  mp.Hkv = num_kv_heads;
+  mp.k = p.k;
+  mp.Gh = p.Gh;
+  mp.maxblk = max_blocks_per_seq;
+  mp.split_blocks = split_blocks;
+  mp.slot_floats = p.slot_floats;
   // passes run in stream order; each kernel waits for the previous one before
   // touching the workspace (programmatic dependents wait for the full grid)
   for (int q0 = 0; q0 < q_len; q0 += kp) {
-    p.q0 = q0;
-    p.G = Gh * std::min(kp, q_len - q0);
+    p.q0 = mp.q0 = q0;
+    p.G = mp.G = Gh * std::min(kp, q_len - q0);
     p.epoch = next_decode_epoch();
     const int nt = p.G > 8 ? 2 : 1;  // tiles of 8 columns
-    const cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
+    mp.warps = di.sms * decode_warps(kv_dtype, head_dim, nt);
+    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
+    if (e != cudaSuccess) return PQKV_ERR_CUDA;
+    e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
     if (e != cudaSuccess) return PQKV_ERR_CUDA;
   }
   return PQKV_OK;

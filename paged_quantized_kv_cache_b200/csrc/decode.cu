@@ -422,58 +422,80 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
 // Log-sum-exp merge of a split pair ("Flash-Decoding": the partial softmaxes of
 // the pieces are combined as M = max_j m_j, L = sum_j l_j 2^(m_j - M),
 // out = sum_j O_j 2^(m_j - M) / L, in fixed piece order) for all G columns of
-// the pair (b, h) whose np pieces start in chunk k0. Run by one warp: the warp
-// whose piece completed the pair (see arrive_split), so results do not depend
-// on which warp that is or on timing. It runs at the end of that warp's chunk,
-// so it is written for latency: 8 lanes per column, 4 columns at a time, and
-// the (m, l) of every piece are loaded together with the first two pieces'
-// outputs (one round trip to L2 per 4 columns for the usual np = 2).
+// the pair (b, h) whose np >= 2 pieces start in chunk k0. Run by one warp: the
+// warp whose piece completed the pair (see arrive_split), so results do not
+// depend on which warp that is or on timing. It runs at the end of that warp's
+// chunk, so it is written for latency: a group of 8 lanes per column, 4
+// columns at a time; lane j of a group holds the (m, l) of pieces j, j + 8, ...
+// (reduced over the group), and the outputs of kB pieces are loaded at once,
+// the first kB together with the (m, l). For the usual np <= kB that is one
+// round trip to L2 per 4 columns.
 // ---------------------------------------------------------------------------
 template <int D, bool QBF16>
 __device__ __forceinline__ void merge_pair(const DecodeParams& p, int b, int h, int k0, int np, int lane) {
   constexpr int DL = D / 8;   // head dims per lane
   constexpr int V4 = DL / 4;  // float4 per lane and piece
+  constexpr int kB = D == 128 ? 2 : 4;  // pieces whose outputs are loaded together
   const int G = p.G;
+  const int j = lane & 7, gbase = lane & ~7;
   auto slot_base = [&](int i) {  // piece i (0-based) of the pair
     const int kk = k0 + i;
     return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
   };
   for (int n0 = 0; n0 < G; n0 += 4) {
-    const int n = n0 + (lane >> 3), d0 = (lane & 7) * DL;
-    if (n < G) {
-      float4 v0[V4], v1[V4];
+    const int n = n0 + (lane >> 3), d0 = j * DL;
+    const bool act = n < G;  // the same on the 8 lanes of a group
+    float4 v[kB][V4];
+    auto load_batch = [&](int c0) {
 #pragma unroll
-      for (int u = 0; u < V4; ++u) {
-        v0[u] = __ldcg(reinterpret_cast<const float4*>(slot_base(0) + n * D + d0) + u);
-        v1[u] = __ldcg(reinterpret_cast<const float4*>(slot_base(1) + n * D + d0) + u);  // np >= 2
-      }
-      float M = kNegInf;
-      for (int i = 0; i < np; ++i) M = fmaxf(M, __ldcg(slot_base(i) + G * D + n));
-      auto weight = [&](int i) { return M == kNegInf ? 0.f : exp2f(__ldcg(slot_base(i) + G * D + n) - M); };
-      float L = 0.f;
-      for (int i = 0; i < np; ++i) L += weight(i) * __ldcg(slot_base(i) + G * D + G + n);
-      float acc[DL];
-      {
-        const float w0 = weight(0), w1 = weight(1);
+      for (int u = 0; u < kB; ++u)
 #pragma unroll
-        for (int u = 0; u < V4; ++u) {
-          acc[4 * u + 0] = w0 * v0[u].x + w1 * v1[u].x;
-          acc[4 * u + 1] = w0 * v0[u].y + w1 * v1[u].y;
-          acc[4 * u + 2] = w0 * v0[u].z + w1 * v1[u].z;
-          acc[4 * u + 3] = w0 * v0[u].w + w1 * v1[u].w;
+        for (int q = 0; q < V4; ++q)
+          v[u][q] = (act && c0 + u < np) ? __ldcg(reinterpret_cast<const float4*>(slot_base(c0 + u) + n * D + d0) + q)
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+    };
+    load_batch(0);
+    // weights: lane j of the group takes pieces j, j + 8, ...
+    float mA = kNegInf, lA = 0.f;
+    if (act && j < np) {
+      mA = __ldcg(slot_base(j) + G * D + n);
+      lA = __ldcg(slot_base(j) + G * D + G + n);
+    }
+    float M = mA;
+    if (act)
+      for (int i = j + 8; i < np; i += 8) M = fmaxf(M, __ldcg(slot_base(i) + G * D + n));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+    const float wA = (M == kNegInf || j >= np) ? 0.f : exp2f(mA - M);  // weight of piece j
+    float L = wA * lA;
+    if (act && M != kNegInf)
+      for (int i = j + 8; i < np; i += 8)
+        L += exp2f(__ldcg(slot_base(i) + G * D + n) - M) * __ldcg(slot_base(i) + G * D + G + n);
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) L += __shfl_xor_sync(kFull, L, o);
+    // outputs: pieces in order
+    float acc[DL];
+#pragma unroll
+    for (int e = 0; e < DL; ++e) acc[e] = 0.f;
+    for (int c0 = 0; c0 < np; c0 += kB) {
+      if (c0 > 0) load_batch(c0);
+#pragma unroll
+      for (int u = 0; u < kB; ++u) {
+        const int i = c0 + u;
+        float w = __shfl_sync(kFull, wA, gbase | (i & 7));  // piece i < 8: held by lane i of the group
+        if (i >= 8) w = (!act || M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + G * D + n) - M);
+        if (i < np) {
+#pragma unroll
+          for (int q = 0; q < V4; ++q) {
+            acc[4 * q + 0] += w * v[u][q].x;
+            acc[4 * q + 1] += w * v[u][q].y;
+            acc[4 * q + 2] += w * v[u][q].z;
+            acc[4 * q + 3] += w * v[u][q].w;
+          }
         }
       }
-      for (int i = 2; i < np; ++i) {
-        const float w = weight(i);
-#pragma unroll
-        for (int u = 0; u < V4; ++u) {
-          const float4 t = __ldcg(reinterpret_cast<const float4*>(slot_base(i) + n * D + d0) + u);
-          acc[4 * u + 0] += w * t.x;
-          acc[4 * u + 1] += w * t.y;
-          acc[4 * u + 2] += w * t.z;
-          acc[4 * u + 3] += w * t.w;
-        }
-      }
+    }
+    if (act) {
       const float inv = L > 0.f ? 1.f / L : 0.f;
       const size_t orow = col_row(b, h, n, p.k, p.q0, p.Gh, p.Hq, D) + d0;
 #pragma unroll
@@ -511,6 +533,124 @@ __device__ __forceinline__ bool arrive_split(const DecodeParams& p, int k0, int 
     if (last) __threadfence();  // order the reads of the other pieces after the count
   }
   return __shfl_sync(kFull, last, 0) != 0;
+}
+
+// ---------------------------------------------------------------------------
+// Log-sum-exp merge of the split pairs of more than kMergeInKernel pieces (same
+// formula as merge_pair). One warp per (sequence b, KV head h, column n).
+// Launched as a programmatic dependent of the decode kernel: it rebuilds the
+// decode's split plan from seq_lens while that grid is still running, and its
+// warps whose pair needs nothing from it exit before waiting for the decode,
+// so with no long split pair the whole grid is done before the decode is.
+// Long pairs (few long sequences spread over the whole GPU) get B x Hkv x G
+// warps here instead of one warp at the end of the decode.
+// ---------------------------------------------------------------------------
+template <int D, bool QBF16>
+__global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
+  extern __shared__ int P[];  // [B + 1]: blocks of the sequences before b, as in the decode
+  __shared__ int wsum[4];
+  constexpr int DPL = D / 32;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  {
+    const int B = p.B, per = (B + 127) / 128;
+    const int lo = min(B, tid * per), hi = min(B, lo + per);
+    const int lim = kBlock * p.maxblk;
+    int local = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      local += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(kFull, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) wsum[warp] = incl;
+    __syncthreads();
+    int run = incl - local;
+    for (int w = 0; w < warp; ++w) run += wsum[w];
+    if (tid == 0) P[0] = 0;
+    for (int i = lo; i < hi; ++i) {
+      const int L = p.seq_lens[i];
+      run += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
+      P[i + 1] = run;
+    }
+    __syncthreads();
+  }
+  const int T = p.Hkv * P[p.B];
+  const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + p.warps - 1) / p.warps);
+  const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (wid >= (long)p.B * p.Hkv * p.G) return;
+  const int b = (int)(wid / ((long)p.Hkv * p.G));
+  const int h = (int)((wid / p.G) % p.Hkv), n = (int)(wid % p.G);
+  const int nblk = P[b + 1] - P[b];
+  if (nblk == 0) return;
+  const int s0 = p.Hkv * P[b] + h * nblk;
+  const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
+  const int np = k1 - k0 + 1;
+  if (np <= kMergeInKernel) return;  // one chunk (no split), or merged inside the decode kernel
+  auto slot_base = [&](int i) {  // piece i (0-based) of the pair
+    const int kk = k0 + i;
+    return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
+  };
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // weights: lanes over pieces; lane i keeps piece i's (m, l) for the common np <= 32
+  float mi = kNegInf, li = 0.f;
+  if (lane < np) {
+    const float* bs = slot_base(lane);
+    mi = __ldcg(bs + p.G * D + n);
+    li = __ldcg(bs + p.G * D + p.G + n);
+  }
+  float M = mi;
+  for (int i = lane + 32; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  const float wi = (M == kNegInf || lane >= np) ? 0.f : exp2f(mi - M);
+  float L = wi * li;
+  for (int i = lane + 32; i < np; i += 32) {
+    const float* bs = slot_base(i);
+    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M) * __ldcg(bs + p.G * D + p.G + n);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+  // outputs: lanes over head dims, pieces in order; the loads of up to 16
+  // pieces are all issued before the first one is folded in
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  constexpr int kBatch = 16;
+  for (int i0 = 0; i0 < np; i0 += kBatch) {
+    float v[kBatch][DPL];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u;
+      if (i < np) {
+        const float* bs = slot_base(i) + n * D + lane * DPL;
+        if constexpr (DPL == 4) {
+          const float4 t = __ldcg(reinterpret_cast<const float4*>(bs));
+          v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < DPL; ++e) v[u][e] = __ldcg(bs + e);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int i = i0 + u;
+      float w = __shfl_sync(kFull, wi, i & 31);
+      if (i < np) {
+        if (i >= 32) w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + p.G * D + n) - M);
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) acc[e] += w * v[u][e];
+      }
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  const size_t orow = col_row(b, h, n, p.k, p.q0, p.Gh, p.Hq, D) + lane * DPL;
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
 }
 
 template <int KVF, int D, bool QBF16, int NT>
@@ -826,11 +966,12 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
           }
         }
       }
-      // the warp that brings the pair's last piece merges all of its pieces
+      // a pair of at most kMergeInKernel pieces is merged by the warp that
+      // brings its last piece; longer ones by paged_merge_kernel
       __syncwarp();
       const int s0 = Hkv * P[b] + h * nblk;  // flat index of the pair's first block
       const int k0 = s0 / Qc, np = (s0 + nblk - 1) / Qc - k0 + 1;
-      if (arrive_split(p, k0, np, lane)) merge_pair<D, QBF16>(p, b, h, k0, np, lane);
+      if (np <= kMergeInKernel && arrive_split(p, k0, np, lane)) merge_pair<D, QBF16>(p, b, h, k0, np, lane);
     };
 
     auto wait_stage = [&](int s) -> bool {
@@ -1067,7 +1208,49 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
   return cudaGetLastError();
 }
 
+// The merge kernel is launched right behind the decode kernel on the same
+// stream as a programmatic dependent (its launch overlaps the decode's tail;
+// griddepcontrol.wait inside it orders it after the decode grid).
+cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st) {
+  const long warps = (long)p.B * p.Hkv * p.G;  // one per (sequence, KV head, column)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = (size_t)(p.B + 1) * 4;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (D == 128)
+    return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, true>, p)
+                  : cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, false>, p);
+  return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, true>, p)
+                : cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, false>, p);
+}
+
 // nt = tiles of 8 MMA columns per warp (1, or 2 for up to 16 query rows per KV head)
+template <int NT>
+static int decode_warps_t(int kv_dtype, int D) {
+  switch (kv_dtype) {
+    case PQKV_DTYPE_FP16:
+    case PQKV_DTYPE_BF16:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_BF16, 128, NT>::kWarps : DecodeGeom<PQKV_DTYPE_BF16, 64, NT>::kWarps;
+    case PQKV_DTYPE_FP8_E4M3:
+    case PQKV_DTYPE_FP8_E5M2:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP8_E4M3, 128, NT>::kWarps
+                      : DecodeGeom<PQKV_DTYPE_FP8_E4M3, 64, NT>::kWarps;
+    default:
+      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP4_E2M1, 128, NT>::kWarps
+                      : DecodeGeom<PQKV_DTYPE_FP4_E2M1, 64, NT>::kWarps;
+  }
+}
+
+int decode_warps(int kv_dtype, int D, int nt) {
+  return nt == 2 ? decode_warps_t<2>(kv_dtype, D) : decode_warps_t<1>(kv_dtype, D);
+}
+
 template <int NT>
 static size_t decode_smem_bytes_t(int kv_dtype, int D, int B) {
   switch (kv_dtype) {

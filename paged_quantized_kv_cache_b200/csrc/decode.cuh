@@ -14,9 +14,12 @@
 // The grid is persistent (one CTA per SM, NW warps each); the flat range is cut
 // into chunks of Q blocks and warp w takes chunks w, w + W, ... (W = all warps).
 // A chunk covers whole pairs (written straight to `out`) and at most two
-// partial pairs at its ends (written to a workspace slot). The warp that
-// writes the last piece of a split pair (counted in a per-pair arrival word)
-// merges its pieces in chunk order, so results do not depend on timing.
+// partial pairs at its ends (written to a workspace slot). The pieces of a
+// split pair are merged in chunk order, so results do not depend on timing:
+// a pair of at most kMergeInKernel pieces (the usual case: many sequences)
+// by the warp that writes its last piece (counted in a per-pair arrival
+// word); a longer one (few long sequences spread over the GPU) by a second
+// kernel, launched as a programmatic dependent, with one warp per column.
 //
 // Per warp: a private ring of NS shared-memory stages, each holding the K and V
 // tiles of one (block, head) pair fetched by one TMA tensor copy (128/64/32-byte
@@ -33,6 +36,7 @@
 namespace pqkv {
 
 constexpr int kDecodeWarps = 12;  // upper bound of warps per CTA over all formats
+constexpr int kMergeInKernel = 4;  // split pairs of up to this many pieces are merged inside the decode
 
 struct DecodeParams {
   const void* q;
@@ -56,6 +60,17 @@ struct DecodeParams {
   float scale_log2;             // softmax scale * log2(e)
   uint64_t timeout_ns;
   unsigned long long epoch;     // tag of this launch (40 bits, never 0)
+};
+
+struct MergeParams {
+  const int32_t* seq_lens;
+  const float* partials;
+  void* out;
+  int B, Hq, Hkv, G, maxblk;
+  int k, Gh, q0;     // as in DecodeParams
+  int warps;         // warps of the decode grid (its balanced chunk length depends on it)
+  int split_blocks;
+  int slot_floats;
 };
 
 // Compile-time geometry of one format; NT = tiles of 8 MMA columns (query rows)
