@@ -89,12 +89,16 @@ struct DecodeGeom {
   static constexpr int kIdxBytes = kFp4 ? 16 : 0;
   static constexpr int kSide = kScaleBytes + kValBytes + kIdxBytes;  // multiple of 16
   static constexpr int kSideStride = kSide == 0 ? 0 : ((kSide + 127) / 128) * 128;
-  // Warps per CTA and shared-memory stages per warp (even: blocks are consumed
-  // in pairs while the next pair is in flight); about 192 KB of stages per SM.
-  // (two column tiles double the accumulators: quantized formats drop to 8 warps)
-  static constexpr int kWarps = k16 ? (D == 128 ? 6 : 8) : (NT == 1 ? 12 : 8);
+  // Warps per CTA and shared-memory stages per warp; about 192-200 KB of stages
+  // per SM. Blocks are consumed two at a time, so while a pair is computed NS - 2
+  // copies stay in flight: 16-bit D128 with one column tile takes 5 warps x 5
+  // stages (measured 1.2% faster per step than 6 x 4 on the llama8b workload);
+  // with two tiles the longer compute per block favours 6 x 4 (q_len 4: 4865
+  // against 4507 GB/s). Two tiles double the accumulators: quantized formats
+  // then drop to 8 warps.
+  static constexpr int kWarps = k16 ? (D == 128 ? (NT == 1 ? 5 : 6) : 8) : (NT == 1 ? 12 : 8);
   static constexpr int kCols = 8 * NT;                          // MMA columns per KV head
-  static constexpr int kStages = k16 ? (D == 128 ? 4 : 6) : (kFp8 ? (D == 128 ? 4 : 6) : (D == 128 ? 4 : 6));
+  static constexpr int kStages = k16 ? (D == 128 ? (NT == 1 ? 5 : 4) : 6) : (D == 128 ? 4 : 6);
   static constexpr uint32_t kTx = kTile + kSide;
   // FP4 per-warp shared rows, padded so that the 8 rows fall in different banks
   static constexpr int kQStride = D + 2;  // f16 query copy, halves per row
