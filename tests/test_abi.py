@@ -80,6 +80,18 @@ def test_invalid_arguments_are_rejected_before_any_launch():
                                                128, null, 4, null, f, 0, null, null, 0, null,
                                                null) == pq.ERR_ARG
     assert lib.pqkv_decode_workspace_init(null, 16, null) == pq.ERR_ARG
+    # workspace sizes: 0 for sizes no call accepts (checked before any device query)
+    # (batch, Hq, Hkv, D, max_blocks, split): Hq not a multiple of Hkv, 32 columns
+    # per KV head (at most 16 per pass), head_dim 96, no blocks, negative split, no batch
+    for args in [(2, 6, 4, 128, 8, 0), (2, 64, 2, 128, 8, 0), (2, 8, 8, 96, 8, 0), (2, 8, 8, 128, 0, 0),
+                 (2, 8, 8, 128, 8, -1), (0, 8, 8, 128, 8, 0)]:
+        assert lib.pqkv_decode_workspace_bytes(*args) == 0
+    # multi-query: q_len outside 1..64 or more than 8 query heads per KV head
+    for (k, Hq, Hkv) in [(0, 32, 8), (65, 32, 8), (4, 48, 4), (4, 6, 4)]:
+        assert lib.pqkv_multi_query_decode_workspace_bytes(2, k, Hq, Hkv, 128, 8, 0) == 0
+        assert lib.pqkv_paged_multi_query_decode_attention(null, pq.BF16, 2, k, Hq, null, null, null, null, pq.BF16,
+                                                           4, Hkv, 128, null, 4, null, f, 0, null, null, 0, null,
+                                                           null) == pq.ERR_ARG
     assert lib.pqkv_encode(null, 5, pq.FP8_E4M3, null, null) == pq.ERR_ARG
     assert lib.pqkv_encode(null, 0, pq.BF16, null, null) == pq.ERR_ARG
     for s in range(6):
