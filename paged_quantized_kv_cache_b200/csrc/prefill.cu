@@ -126,6 +126,34 @@ __device__ __forceinline__ bool wg_all(int wg, bool v) {
   return r != 0;
 }
 
+// Packed pairs of fp32 operations (two lanes of IEEE fp32 arithmetic, rounded to
+// nearest, in one instruction): (d0, d1) = (a0, a1) op (b0, b1) [+ (c0, c1)].
+__device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                     float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "sub.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+
 // E4M3 scale byte -> f16x2 (s, s).
 __device__ __forceinline__ __half2 scale2(uint32_t byte) {
   const uint32_t r = dec_fp8x2<PQKV_DTYPE_FP8_E4M3>(byte | (byte << 8));
@@ -561,7 +589,9 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       const float mu = (m == -INFINITY) ? 0.f : m;  // masked entries are -inf and give 0
       uint32_t pk[32], pl[32];
       {
-        float rp[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        // columns in pairs, two per packed fp32 instruction; running sums of
+        // the even (ra) and odd (rb) columns in 4 chains each
+        float ra[4] = {0.f, 0.f, 0.f, 0.f}, rb[4] = {0.f, 0.f, 0.f, 0.f};
         float vr[4] = {1.f, 1.f, 1.f, 1.f};
         if constexpr (Gm::kFp8) {
 #pragma unroll
@@ -569,25 +599,22 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         }
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
-          float pa, pb;
-          if constexpr (Gm::kFp8) {
-            pa = ex2(xs[c] - mu);
-            pb = ex2(xs[c + 1] - mu);
-          } else {
-            pa = ex2(fmaf(xs[c], p.scale_log2, -mu));
-            pb = ex2(fmaf(xs[c + 1], p.scale_log2, -mu));
-          }
-          rp[(c >> 1) & 7] += pa + pb;
+          float ya, yb;
+          if constexpr (Gm::kFp8) sub2(ya, yb, xs[c], xs[c + 1], mu, mu);
+          else fma2(ya, yb, xs[c], xs[c + 1], p.scale_log2, p.scale_log2, -mu, -mu);
+          const float pa = ex2(ya), pb = ex2(yb);
+          const int i = (c >> 1) & 3;
+          add2(ra[i], rb[i], ra[i], rb[i], pa, pb);
           float wa = pa, wb = pb;
-          if constexpr (Gm::kFp8) {
-            wa *= vr[c >> 4];
-            wb *= vr[c >> 4];
-          }
+          if constexpr (Gm::kFp8) mul2(wa, wb, pa, pb, vr[c >> 4], vr[c >> 4]);
           pk[c >> 1] = pack_f32x2(wa, wb, kBfMma);
-          if constexpr (Gm::kSplitP)
-            pl[c >> 1] = pack_f32x2(wa - unpack_lo(pk[c >> 1], kBfMma), wb - unpack_hi(pk[c >> 1], kBfMma), kBfMma);
+          if constexpr (Gm::kSplitP) {
+            float da, db;
+            sub2(da, db, wa, wb, unpack_lo(pk[c >> 1], kBfMma), unpack_hi(pk[c >> 1], kBfMma));
+            pl[c >> 1] = pack_f32x2(da, db, kBfMma);
+          }
         }
-        l += ((rp[0] + rp[1]) + (rp[2] + rp[3])) + ((rp[4] + rp[5]) + (rp[6] + rp[7]));
+        l += ((ra[0] + ra[1]) + (ra[2] + ra[3])) + ((rb[0] + rb[1]) + (rb[2] + rb[3]));
       }
 
       // PV(t-1) must be done before O is rescaled or P is overwritten
