@@ -578,6 +578,8 @@ def run_ours(args) -> None:
             "frac_of_hbm_peak": value / world / peaks["hbm_gbs"],
             "frac_of_8tbs_spec": value / world / 8000.0,
             "decode_tok_s_per_layer": tok_s,
+            # the decode call alone (no cache write): B x q_len / t(decode)
+            "decode_only_tok_s_per_layer": s.batch * args.q_len * world / (dec_ms * 1e-3),
             "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             # per step: cache write, then per decode pass the split decode and the merge kernel of
