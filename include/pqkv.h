@@ -225,6 +225,11 @@ int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q
  * q_len = 1 is pqkv_paged_decode_attention, bit for bit. Other arguments,
  * results and errors as there.
  */
+/* Device workspace needed by pqkv_paged_multi_query_decode_attention for these
+ * sizes, on the current device: pqkv_decode_workspace_bytes with the columns of
+ * one pass (num_q_heads x kp, kp as above). split_blocks as there. Returns 0 for
+ * sizes the call rejects (q_len outside 1..64, more than 8 query heads per KV
+ * head, the other checks of pqkv_decode_workspace_bytes) or without a device. */
 size_t pqkv_multi_query_decode_workspace_bytes(int batch, int q_len, int num_q_heads,
                                                int num_kv_heads, int head_dim,
                                                int max_blocks_per_seq, int split_blocks);
