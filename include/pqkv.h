@@ -102,7 +102,11 @@ enum {
                                 skipped and its output rows written as zeros */
   PQKV_DEVERR_RUN = 8,       /* write (FP8/FP4): two adjacent tokens map to the same block
                                 with non-consecutive offsets */
-  PQKV_DEVERR_TIMEOUT = 16   /* a bounded wait on an asynchronous copy gave up */
+  PQKV_DEVERR_TIMEOUT = 16,  /* a bounded wait on an asynchronous copy gave up; the kernel's
+                                remaining work for that warp is skipped (outputs it owns are
+                                left unwritten) after its copies in flight have landed */
+  PQKV_DEVERR_DRAIN = 32     /* after a TIMEOUT, a copy still in flight did not land within the
+                                full wait limit either */
 };
 
 #define PQKV_BLOCK_SIZE 16
@@ -117,6 +121,15 @@ int pqkv_version(void);
 
 /* Human-readable name of a PQKV_* return code. Never NULL. */
 const char* pqkv_status_string(int status);
+
+/* Limit, in nanoseconds, of each wait of the decode kernels
+ * (pqkv_paged_decode_attention and its variants) on one of their asynchronous
+ * copies, for the launches enqueued after this call (process-wide; 0 restores
+ * the default of 2 s). A wait that runs out sets PQKV_DEVERR_TIMEOUT and ends
+ * that warp's work, after its copies still in flight have landed (that wait
+ * keeps the 2 s limit). Meant for tests of the timeout path: a very short
+ * limit makes waits give up while their copies are still on the way. */
+void pqkv_set_decode_wait_limit_ns(uint64_t ns);
 
 /*
  * Byte sizes of the four cache arrays for `kv_dtype`: out_bytes[0] = cache,
@@ -255,11 +268,18 @@ int pqkv_paged_multi_query_decode_attention(const void* q, int q_dtype, int batc
  * launch nothing; with split_blocks = 0, head_dim <= 128 and up to 8 query heads
  * per KV head the need stays below 16 MiB on a 148-SM GPU. Nothing is
  * allocated. The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and should come before any stream capture. All calls
- * share the array: calls that overlap on the GPU (other streams, other host
- * threads) race on it and must be ordered by the caller. No part of the array
- * needs to start at zero; it keeps the last call's contents. Other arguments,
- * results and errors as pqkv_paged_decode_attention.
+ * (cudaGetSymbolAddress) and should come before any stream capture; the
+ * address is kept for the life of the process, so a device reset
+ * (cudaDeviceReset) leaves this entry point unusable, and devices numbered 64
+ * or higher get PQKV_ERR_CUDA. All calls share the array, which keeps the last
+ * call's contents: calls that overlap on the GPU (other streams, other host
+ * threads) race on it and must be ordered by the caller. When a call's sizes
+ * (batch, head counts, head_dim, max_blocks_per_seq, split_blocks) differ from
+ * the previous call's on the device, the part of the array it uses is zeroed
+ * first on `stream` (a memset, no allocation), so that nothing a call with
+ * another layout left there is taken for this call's split-pair bookkeeping.
+ * Other arguments, results and errors (checked in the same order, before the
+ * scratch limit) as pqkv_paged_decode_attention.
  */
 #define PQKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 int pqkv_paged_decode_attention_noalloc(const void* q, int q_dtype, int batch, int num_q_heads,
@@ -355,6 +375,23 @@ int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
  */
 int pqkv_encode(const float* x, int64_t n, int code_dtype, uint8_t* codes,
                 pqkv_stream_t stream);
+
+/*
+ * Read-bandwidth probe (a measurement helper, not a step of the method): the
+ * paged gather of pqkv_paged_decode_attention without its arithmetic. Every
+ * K|V tile of every (sequence, KV head, block) that a decode of the same batch
+ * reads through block_tables ([P3] "PagedAttention") is copied into shared
+ * memory; one word of each is XORed into *checksum (device uint32, which the
+ * caller zeroes) so that no copy can be skipped. The scales and outlier
+ * buffers are not read. With an identity table (sequence b's block j stored
+ * right after its block j - 1) it reads the cache front to back, the
+ * contiguous read ceiling. Arguments as in pqkv_paged_decode_attention;
+ * lengths outside [0, 16 * max_blocks_per_seq] count as empty and block ids
+ * outside [0, num_blocks) set PQKV_DEVERR_BLOCK_ID. One kernel on `stream`.
+ */
+int pqkv_read_probe(const void* cache, int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens,
+                    int batch, uint32_t* checksum, int32_t* err_flag, pqkv_stream_t stream);
 
 /* ---- block pool ([P3] PagedAttention / continuous batching; [P2] pool
  *      exhaustion) ------------------------------------------------------------

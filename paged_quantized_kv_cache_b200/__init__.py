@@ -25,7 +25,7 @@ FP16, BF16, FP8_E4M3, FP8_E5M2, FP4_E2M1 = 0, 1, 2, 3, 4
 DTYPE_NAMES = {FP16: "fp16", BF16: "bf16", FP8_E4M3: "fp8_e4m3", FP8_E5M2: "fp8_e5m2", FP4_E2M1: "fp4_e2m1"}
 OK, ERR_ARG, ERR_OOM, ERR_STATE, ERR_CUDA, ERR_SCRATCH = 0, 1, 2, 3, 4, 5
 NOALLOC_SCRATCH_BYTES = 16 << 20
-DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_RUN, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
+DEVERR_SLOT, DEVERR_BLOCK_ID, DEVERR_SEQ_LEN, DEVERR_RUN, DEVERR_TIMEOUT, DEVERR_DRAIN = 1, 2, 4, 8, 16, 32
 BLOCK_SIZE = 16
 MAX_BATCH = 4096
 
@@ -39,6 +39,7 @@ EXPORTS = (
     "pqkv_pool_prefix_lookup", "pqkv_pool_prefix_insert", "pqkv_pool_cow", "pqkv_copy_blocks",
     "pqkv_block_record_bytes", "pqkv_swap_out", "pqkv_swap_in", "pqkv_paged_prefill_attention",
     "pqkv_paged_multi_query_decode_attention", "pqkv_multi_query_decode_workspace_bytes",
+    "pqkv_read_probe", "pqkv_set_decode_wait_limit_ns",
 )
 
 
@@ -87,6 +88,8 @@ def _load() -> ctypes.CDLL:
                                              P, P, P]),
         "pqkv_paged_multi_query_decode_attention": (I, [P, I, I, I, I, P, P, P, P, I, I, I, I, P, I, P,
                                                         ctypes.c_float, I, P, P, Z, P, P]),
+        "pqkv_read_probe": (I, [P, I, I, I, I, P, I, P, I, P, P, P]),
+        "pqkv_set_decode_wait_limit_ns": (None, [ctypes.c_uint64]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -141,6 +144,12 @@ def _dt_of(t: torch.Tensor, name: str) -> int:
     if t.dtype == torch.bfloat16:
         return BF16
     raise ValueError("%s must be float16 or bfloat16" % name)
+
+
+def set_decode_wait_limit_ns(ns: int) -> None:
+    """pqkv_set_decode_wait_limit_ns: limit of the decode kernels' waits on their
+    copies for later launches (0 = the default 2 s); for tests of the timeout path."""
+    _lib.pqkv_set_decode_wait_limit_ns(int(ns))
 
 
 def version() -> int:
@@ -310,6 +319,24 @@ def encode(x: torch.Tensor, code_dtype: int, out: torch.Tensor, stream=None) -> 
         raise ValueError("x must be float32 and out uint8 of the same size")
     _check("pqkv_encode", _lib.pqkv_encode(_dev_ptr(x, "x"), x.numel(), code_dtype, _dev_ptr(out, "out"),
                                            _stream_handle(stream, x.device)))
+
+
+def read_probe(cache: KVCache, block_tables: torch.Tensor, seq_lens: torch.Tensor, checksum: torch.Tensor,
+               err_flag: torch.Tensor, stream=None) -> None:
+    """pqkv_read_probe: the decode's paged gather of K|V tiles without its math
+    (a bandwidth measurement); checksum: device int32 [1] that the caller zeroes."""
+    B = seq_lens.numel()
+    if block_tables.dtype != torch.int32 or block_tables.dim() != 2 or block_tables.shape[0] != B:
+        raise ValueError("block_tables must be int32 [B][max_blocks_per_seq]")
+    if seq_lens.dtype != torch.int32:
+        raise ValueError("seq_lens must be int32 [B]")
+    if checksum.dtype != torch.int32 or checksum.numel() < 1:
+        raise ValueError("checksum must be int32 [1]")
+    _check("pqkv_read_probe", _lib.pqkv_read_probe(
+        _dev_ptr(cache.cache, "cache"), cache.kv_dtype, cache.num_blocks, cache.num_kv_heads, cache.head_dim,
+        _dev_ptr(block_tables, "block_tables"), block_tables.shape[1], _dev_ptr(seq_lens, "seq_lens"), B,
+        _dev_ptr(checksum, "checksum"), _dev_ptr(err_flag, "err_flag"),
+        _stream_handle(stream, cache.cache.device)))
 
 
 def copy_blocks(cache: KVCache, pairs: torch.Tensor, err_flag: torch.Tensor, stream=None) -> None:

@@ -17,6 +17,10 @@ cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtens
 size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt);
 int decode_warps(int kv_dtype, int D, int nt);
 cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
+size_t read_probe_smem_bytes(int B);
+cudaError_t launch_read_probe(const uint8_t* cache, int kv_dtype, int nb, int H, int D, const int32_t* block_tables,
+                              int maxblk, const int32_t* seq_lens, int B, uint32_t* checksum, int32_t* err,
+                              uint64_t timeout_ns, int sms, cudaStream_t st);
 }  // namespace pqkv
 
 using namespace pqkv;
@@ -24,6 +28,9 @@ using namespace pqkv;
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // bounded wait on one asynchronous copy
+
+// Limit of the decode kernels' waits on their copies (pqkv_set_decode_wait_limit_ns).
+std::atomic<uint64_t> g_decode_wait_ns{kWaitLimitNs};
 
 bool is_kv_dtype(int t) { return t >= PQKV_DTYPE_FP16 && t <= PQKV_DTYPE_FP4_E2M1; }
 bool is_16(int t) { return t == PQKV_DTYPE_FP16 || t == PQKV_DTYPE_BF16; }
@@ -131,9 +138,27 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace
 
+namespace pqkv {
+// The size and type checks of a decode call, shared by every decode entry point
+// (the pointer and workspace checks follow in decode_impl).
+int decode_check_sizes(int q_dtype, int batch, int q_len, int num_q_heads, int kv_dtype, int num_blocks,
+                       int num_kv_heads, int head_dim, int max_blocks_per_seq, int split_blocks) {
+  if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
+  if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
+  if (batch < 0 || batch > PQKV_MAX_BATCH || num_kv_heads < 1 || num_q_heads < 1 ||
+      num_q_heads % num_kv_heads != 0 || q_len < 1 || q_len > 64 || num_q_heads / num_kv_heads > 8 ||
+      (head_dim != 64 && head_dim != 128) ||
+      num_blocks < 1 || max_blocks_per_seq < 1 || split_blocks < 0)
+    return PQKV_ERR_ARG;
+  return PQKV_OK;
+}
+}  // namespace pqkv
+
 extern "C" {
 
 int pqkv_version(void) { return 10000; }
+
+void pqkv_set_decode_wait_limit_ns(uint64_t ns) { g_decode_wait_ns.store(ns ? ns : kWaitLimitNs); }
 
 const char* pqkv_status_string(int status) {
   switch (status) {
@@ -245,17 +270,14 @@ size_t pqkv_multi_query_decode_workspace_bytes(int batch, int q_len, int num_q_h
                                      split_blocks);
 }
 
+
 static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num_q_heads, const void* cache,
                        const void* scales, const void* outliers_idx, const void* outliers_val, int kv_dtype,
                        int num_blocks, int num_kv_heads, int head_dim, const int32_t* block_tables,
                        int max_blocks_per_seq, const int32_t* seq_lens, float scale, int split_blocks, void* out,
                        void* workspace, size_t workspace_bytes, int32_t* err_flag, pqkv_stream_t stream) {
-  if (!is_kv_dtype(kv_dtype) || (q_dtype != PQKV_DTYPE_FP16 && q_dtype != PQKV_DTYPE_BF16)) return PQKV_ERR_ARG;
-  if (is_16(kv_dtype) && q_dtype != kv_dtype) return PQKV_ERR_ARG;
-  if (batch < 0 || batch > PQKV_MAX_BATCH || num_kv_heads < 1 || num_q_heads < 1 ||
-      num_q_heads % num_kv_heads != 0 || q_len < 1 || q_len > 64 || num_q_heads / num_kv_heads > 8 ||
-      (head_dim != 64 && head_dim != 128) ||
-      num_blocks < 1 || max_blocks_per_seq < 1 || split_blocks < 0)
+  if (decode_check_sizes(q_dtype, batch, q_len, num_q_heads, kv_dtype, num_blocks, num_kv_heads, head_dim,
+                         max_blocks_per_seq, split_blocks) != PQKV_OK)
     return PQKV_ERR_ARG;
   if (batch == 0) return PQKV_OK;
   if (!q || !cache || !block_tables || !seq_lens || !out || !workspace || !err_flag) return PQKV_ERR_ARG;
@@ -302,7 +324,8 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   p.split_blocks = split_blocks;
   p.slot_floats = (int)round_up((size_t)Gh * kp * head_dim + 2 * Gh * kp, 4);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = kWaitLimitNs;
+  p.timeout_ns = g_decode_wait_ns.load();
+  p.drain_ns = kWaitLimitNs;
   // the arrival words follow the partial slots (16-byte aligned: slot_floats is a multiple of 4)
   const size_t chunks = decode_chunks(batch, num_kv_heads, max_blocks_per_seq, split_blocks, di.sms);
   p.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
@@ -465,8 +488,27 @@ int pqkv_paged_prefill_attention(const void* q, int q_dtype, int batch, int max_
   p.tiles_per_seq = (int)tiles;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.timeout_ns = kWaitLimitNs;
+  p.drain_ns = kWaitLimitNs;
   const cudaError_t e = launch_prefill(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p,
                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
+}
+
+int pqkv_read_probe(const void* cache, int kv_dtype, int num_blocks, int num_kv_heads, int head_dim,
+                    const int32_t* block_tables, int max_blocks_per_seq, const int32_t* seq_lens, int batch,
+                    uint32_t* checksum, int32_t* err_flag, pqkv_stream_t stream) {
+  if (!is_kv_dtype(kv_dtype) || num_blocks < 1 || num_kv_heads < 1 || (head_dim != 64 && head_dim != 128) ||
+      max_blocks_per_seq < 1 || batch < 0 || batch > PQKV_MAX_BATCH)
+    return PQKV_ERR_ARG;
+  if ((int64_t)batch * num_kv_heads * max_blocks_per_seq >= INT32_MAX) return PQKV_ERR_ARG;
+  if (batch == 0) return PQKV_OK;
+  if (!cache || !block_tables || !seq_lens || !checksum || !err_flag || !aligned16(cache)) return PQKV_ERR_ARG;
+  DeviceInfo di;
+  if (!device_info(di)) return PQKV_ERR_CUDA;
+  if (read_probe_smem_bytes(batch) > (size_t)di.max_smem) return PQKV_ERR_ARG;
+  const cudaError_t e = launch_read_probe(static_cast<const uint8_t*>(cache), kv_dtype, num_blocks, num_kv_heads,
+                                          head_dim, block_tables, max_blocks_per_seq, seq_lens, batch, checksum,
+                                          err_flag, kWaitLimitNs, di.sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
 }
 

@@ -767,66 +767,78 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     j = rel - h * n;
   };
 
-  for (int k = warp * gridDim.x + blockIdx.x; k < K && !aborted; k += W) {
-    const int f0 = k * Qc;
-    const int f1 = min(T, f0 + Qc);
-
-    // Per-lane window of (physical id, head) for flat blocks wbase + lane and,
-    // loaded ahead, wbase + 32 + lane. Values are only inspected when issued.
-    auto load_entry = [&](int f, int& id, int& hh) {
-      id = -1;
-      hh = 0;
-      if (f < f1) {
-        int b, h, j;
-        locate(f, b, h, j);
-        id = __ldg(p.block_tables + (size_t)b * p.maxblk + j);
-        hh = h;
-      }
-    };
-    int wbase = f0, wid, wh, nid, nh;
-    load_entry(f0 + lane, wid, wh);
-    load_entry(f0 + 32 + lane, nid, nh);
-    uint32_t skip = 0;
-    auto issue = [&](int s, int f) {
-      while (f - wbase >= 32) {
-        wbase += 32;
-        wid = nid;
-        wh = nh;
-        load_entry(wbase + 32 + lane, nid, nh);
-      }
-      const int id = __shfl_sync(kFull, wid, f - wbase);
-      const int hh = __shfl_sync(kFull, wh, f - wbase);
-      const bool bad = (id < 0 || id >= p.nb);
-      inflight |= 1u << s;
-      if (bad) skip |= 1u << s; else skip &= ~(1u << s);
-      if (lane == 0) {
-        uint64_t* bar = &wbar[s];
-        if (bad) {
-          raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
-          mbar_arrive(bar);
-        } else {
-          const int coord = (id * Hkv + hh) * 32;
-          mbar_arrive_expect_tx(bar, Gm::kTx);
-          uint8_t* dst = wtile + s * Gm::kTile;
-          constexpr int kElem = Gm::k16 ? 2 : 1;
+  // This warp's chunks are k0, k0 + W, k0 + 2W, ... Its blocks, chunk after
+  // chunk, are numbered v = 0 .. Vtot - 1; the copy ring runs over v without a
+  // break at chunk boundaries, so the next chunk's first blocks are already on
+  // the way while a chunk drains.
+  const int k0 = warp * gridDim.x + blockIdx.x;
+  const int nck = k0 < K ? (K - 1 - k0) / W + 1 : 0;
+  const int Vtot = nck == 0 ? 0 : (nck - 1) * Qc + (min(T, (k0 + (nck - 1) * W + 1) * Qc) - (k0 + (nck - 1) * W) * Qc);
+  auto vflat = [&](int v) {  // virtual block index -> flat block index
+    const int i = v / Qc;
+    return (k0 + i * W) * Qc + (v - i * Qc);
+  };
+  // Per-lane window of (physical id, head) for blocks wbase + lane and, loaded
+  // ahead, wbase + 32 + lane. Values are only inspected when issued.
+  auto load_entry = [&](int v, int& id, int& hh) {
+    id = -1;
+    hh = 0;
+    if (v < Vtot) {
+      int b, h, j;
+      locate(vflat(v), b, h, j);
+      id = __ldg(p.block_tables + (size_t)b * p.maxblk + j);
+      hh = h;
+    }
+  };
+  int wbase = 0, wid, wh, nid, nh;
+  load_entry(lane, wid, wh);
+  load_entry(32 + lane, nid, nh);
+  uint32_t skip = 0;
+  auto issue = [&](int s, int v) {
+    while (v - wbase >= 32) {
+      wbase += 32;
+      wid = nid;
+      wh = nh;
+      load_entry(wbase + 32 + lane, nid, nh);
+    }
+    const int id = __shfl_sync(kFull, wid, v - wbase);
+    const int hh = __shfl_sync(kFull, wh, v - wbase);
+    const bool bad = (id < 0 || id >= p.nb);
+    inflight |= 1u << s;
+    if (bad) skip |= 1u << s; else skip &= ~(1u << s);
+    if (lane == 0) {
+      uint64_t* bar = &wbar[s];
+      if (bad) {
+        raise_flag(p.err, PQKV_DEVERR_BLOCK_ID);
+        mbar_arrive(bar);
+      } else {
+        const int coord = (id * Hkv + hh) * 32;
+        mbar_arrive_expect_tx(bar, Gm::kTx);
+        uint8_t* dst = wtile + s * Gm::kTile;
+        constexpr int kElem = Gm::k16 ? 2 : 1;
 #pragma unroll
-          for (int bx = 0; bx < Gm::kBoxes; ++bx)
-            tma_load_2d(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar);
-          const size_t pair = (size_t)id * Hkv + hh;
-          uint8_t* side = wside + s * Gm::kSideStride;
-          if constexpr (Gm::kFp8) {
-            bulk_load(side, p.scales + pair * 16, 16, bar);
-          } else if constexpr (Gm::kFp4) {
-            bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, bar);
-            bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, bar);
-            bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, bar);
-          }
+        for (int bx = 0; bx < Gm::kBoxes; ++bx)
+          tma_load_2d(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar);
+        const size_t pair = (size_t)id * Hkv + hh;
+        uint8_t* side = wside + s * Gm::kSideStride;
+        if constexpr (Gm::kFp8) {
+          bulk_load(side, p.scales + pair * 16, 16, bar);
+        } else if constexpr (Gm::kFp4) {
+          bulk_load(side, p.scales + pair * Gm::kScaleBytes, Gm::kScaleBytes, bar);
+          bulk_load(side + Gm::kScaleBytes, p.oval + pair * Gm::kValBytes, Gm::kValBytes, bar);
+          bulk_load(side + Gm::kScaleBytes + Gm::kValBytes, p.oidx + pair * 16, 16, bar);
         }
       }
-    };
+    }
+  };
+  for (int i = 0; i < min(NS, Vtot); ++i) issue(i, i);
+  int s = 0;  // stage of the next block to consume
 
-    const int npre = min(NS, f1 - f0);
-    for (int i = 0; i < npre; ++i) issue(i, f0 + i);
+  for (int ci = 0; ci < nck && !aborted; ++ci) {
+    const int k = k0 + ci * W;
+    const int f0 = k * Qc;
+    const int f1 = min(T, f0 + Qc);
+    const int vb = ci * Qc - f0;  // v = f + vb inside this chunk
 
     // ---- consumer state of the current (sequence, head) piece ----
     int b, h, j;
@@ -837,6 +849,10 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     uint32_t qf[NT][KT][2];
     float acc[NT][KT][4];
     float mm[NT][2], ll[NT][2], vref;  // running max and sum of each of the lane's columns
+    // softmax scale (log2 units) of each of the lane's columns, times the power
+    // of two its query row was scaled down by before narrowing to f16
+    // (quantized caches; 16-bit caches keep the query in its own type)
+    float csc[NT][2];
     OutlierState<NT> ost;  // FP4 only
 
     auto begin_piece = [&]() {
@@ -849,10 +865,33 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
       }
       vref = 0.f;
       ost.reset();  // the query changes with the piece
+      float rowmul[NT];  // quantized caches: 2^-e applied to this lane's query row 8nt + g
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
       const bool has = 8 * nt + g < G;
       const size_t qrow = has ? col_row(b, h, 8 * nt + g, p.k, p.q0, p.Gh, Hq, D) : 0;
+      // k-slot order of the dequantized K fragments: FP8 k-step kk holds
+      // d = 16kk + 4qd + {0,1 | 2,3}; FP4 k-step (c, s) = (kk/2, kk%2) holds
+      // d = 32c + 8qd + 4s + {0,1 | 2,3}.
+      auto d0_of = [&](int kk) { return Gm::kFp8 ? 16 * kk + 4 * qd : 32 * (kk >> 1) + 8 * qd + 4 * (kk & 1); };
+      rowmul[nt] = 1.f;
+      if constexpr (!Gm::k16 && QBF16) {
+        // A bf16 row is narrowed to f16 for the MMA: scale it by the power of two
+        // 2^-e that brings its largest |q| into [2^13, 2^14) (exact, and far
+        // from both ends of the f16 range); the logits of its column are
+        // multiplied back by 2^e in the softmax.
+        float mx = 0.f;
+        if (has) {
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) mx = fmaxf(mx, fabsf(q_at<QBF16>(p.q, qrow + d0_of(kk) + i)));
+        }
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+        const int ex = (mx > 0.f && mx <= FLT_MAX) ? ilogbf(mx) - 13 : 0;
+        rowmul[nt] = ldexpf(1.f, -ex);
+      }
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
         if constexpr (Gm::k16) {
@@ -860,28 +899,33 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
           qf[nt][kk][0] = has ? __ldg(q32 + (qrow + 16 * kk + 2 * qd) / 2) : 0u;
           qf[nt][kk][1] = has ? __ldg(q32 + (qrow + 16 * kk + 8 + 2 * qd) / 2) : 0u;
         } else {
-          // k-slot order of the dequantized K fragments: FP8 k-step kk holds
-          // d = 16kk + 4qd + {0,1 | 2,3}; FP4 k-step (c, s) = (kk/2, kk%2) holds
-          // d = 32c + 8qd + 4s + {0,1 | 2,3}.
-          const int d0 = Gm::kFp8 ? 16 * kk + 4 * qd : 32 * (kk >> 1) + 8 * qd + 4 * (kk & 1);
+          const int d0 = d0_of(kk);
           float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
           if (has) {
-            v0 = q_at<QBF16>(p.q, qrow + d0);
-            v1 = q_at<QBF16>(p.q, qrow + d0 + 1);
-            v2 = q_at<QBF16>(p.q, qrow + d0 + 2);
-            v3 = q_at<QBF16>(p.q, qrow + d0 + 3);
+            v0 = q_at<QBF16>(p.q, qrow + d0) * rowmul[nt];
+            v1 = q_at<QBF16>(p.q, qrow + d0 + 1) * rowmul[nt];
+            v2 = q_at<QBF16>(p.q, qrow + d0 + 2) * rowmul[nt];
+            v3 = q_at<QBF16>(p.q, qrow + d0 + 3) * rowmul[nt];
           }
           qf[nt][kk][0] = f16x2_from(v0, v1);
           qf[nt][kk][1] = f16x2_from(v2, v3);
         }
       }
+      // column c of this lane is query row 2qd + c of the tile, held by lanes g = 2qd + c
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float m = __shfl_sync(kFull, rowmul[nt], (2 * qd + c) << 2);
+        csc[nt][c] = (Gm::k16 || !QBF16) ? p.scale_log2 : p.scale_log2 / m;  // 1 / m = 2^e: exact
+      }
       }
       if constexpr (Gm::kFp4) {
-        // f16 copy of this warp's query rows for the outlier channels
+        // f16 copy of this warp's query rows for the outlier channels, scaled
+        // like the fragments (the row of element i is the same on all lanes)
         __syncwarp();
         for (int i = lane; i < NC * D; i += 32) {
           const int n = i / D;
-          const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.q0, p.Gh, Hq, D) + (i % D)) : 0.f;
+          const float m = __shfl_sync(kFull, rowmul[n >> 3 < NT ? n >> 3 : 0], (n & 7) << 2);
+          const float v = (n < G) ? q_at<QBF16>(p.q, col_row(b, h, n, p.k, p.q0, p.Gh, Hq, D) + (i % D)) * m : 0.f;
           wq[n * Gm::kQStride + i % D] = __half_as_ushort(__float2half_rn(v));
         }
         __syncwarp();
@@ -974,15 +1018,18 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
       if (np <= kMergeInKernel && arrive_split(p, k0, np, lane)) merge_pair<D, QBF16>(p, b, h, k0, np, lane);
     };
 
+    // A stage whose wait gives up keeps its phase and its in-flight bit, so
+    // that the drain below waits for that very copy.
     auto wait_stage = [&](int s) -> bool {
       const bool ok = __all_sync(kFull, mbar_wait_bounded(&wbar[s], (phase >> s) & 1u, p.timeout_ns));
-      phase ^= 1u << s;
-      inflight &= ~(1u << s);
+      if (ok) {
+        phase ^= 1u << s;
+        inflight &= ~(1u << s);
+      }
       return ok;
     };
 
     begin_piece();
-    int s = 0;
     int f = f0;
     while (f < f1) {
       // two consecutive blocks of the same piece when available, else one
@@ -1019,18 +1066,19 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 
       // ---- online softmax over up to 32 tokens (log2 domain) ----
       // x[nt][e]: row (token) g + 8 (e >> 1), column 8nt + 2qd + (e & 1)
-      const float mA = p.scale_log2 * skA, mB = p.scale_log2 * skB;
       float xA[NT][4], xB[NT][4], bm[NT][2];
       bool need_any = false;
       constexpr float kLazy = lazy_of<KVF>();
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
+        const float mA0 = csc[nt][0] * skA, mA1 = csc[nt][1] * skA;
+        const float mB0 = csc[nt][0] * skB, mB1 = csc[nt][1] * skB;
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int r = g + 8 * (e >> 1), hd = hid[nt][e & 1];
           // column n sees the tokens before the last hid ones (0 for one query token)
-          xA[nt][e] = (!useA || r >= remA - hd) ? kNegInf : scA[nt][e] * mA;
-          xB[nt][e] = (!useB || r >= remB - hd) ? kNegInf : scB[nt][e] * mB;
+          xA[nt][e] = (!useA || r >= remA - hd) ? kNegInf : scA[nt][e] * ((e & 1) ? mA1 : mA0);
+          xB[nt][e] = (!useB || r >= remB - hd) ? kNegInf : scB[nt][e] * ((e & 1) ? mB1 : mB0);
         }
         bm[nt][0] = fmaxf(fmaxf(xA[nt][0], xA[nt][2]), fmaxf(xB[nt][0], xB[nt][2]));
         bm[nt][1] = fmaxf(fmaxf(xA[nt][1], xA[nt][3]), fmaxf(xB[nt][1], xB[nt][3]));
@@ -1139,8 +1187,9 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
       if (useB && (!Gm::kFp8 || prB > 0.f)) pv(tbB, sdB, validB, pB, prB);
 
       __syncwarp();
-      if (f + NS < f1) issue(sA, f + NS);
-      if (n2 == 2 && f + 1 + NS < f1) issue(sB, f + 1 + NS);
+      const int v = f + vb;
+      if (v + NS < Vtot) issue(sA, v + NS);
+      if (n2 == 2 && v + 1 + NS < Vtot) issue(sB, v + 1 + NS);
       s = (sB + 1 == NS) ? 0 : sB + 1;
       if (n2 == 1) s = sB;
 
@@ -1166,10 +1215,13 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     }
   }
 
-  // after a timeout: let copies still in flight land before the CTA exits
+  // after a timeout: let copies still in flight land before the warp exits
+  // (with the full limit, whatever the limit that gave up)
   if (aborted) {
+    bool drained = true;
     for (int s2 = 0; s2 < NS; ++s2)
-      if ((inflight >> s2) & 1u) (void)mbar_wait_bounded(&wbar[s2], (phase >> s2) & 1u, p.timeout_ns);
+      if ((inflight >> s2) & 1u) drained = mbar_wait_bounded(&wbar[s2], (phase >> s2) & 1u, p.drain_ns) && drained;
+    if (!drained && lane == 0) raise_flag(p.err, PQKV_DEVERR_DRAIN);
   }
 }
 

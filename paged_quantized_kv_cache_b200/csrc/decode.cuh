@@ -58,7 +58,8 @@ struct DecodeParams {
   int split_blocks;
   int slot_floats;
   float scale_log2;             // softmax scale * log2(e)
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;          // limit of a wait on a copy before the warp gives up
+  uint64_t drain_ns;            // after giving up: limit of the wait for copies still in flight
   unsigned long long epoch;     // tag of this launch (40 bits, never 0)
 };
 

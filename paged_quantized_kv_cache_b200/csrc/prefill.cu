@@ -30,6 +30,7 @@
 // scale seen so far (O is kept in units of it). FP4 operands are exact in f16
 // (E2M1 x E4M3 and the fp16 outlier values).
 #include <atomic>
+#include <cfloat>
 
 #include "prefill.cuh"
 #include "tcgen05.cuh"
@@ -240,18 +241,41 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   }
   if constexpr (Gm::k16)
     if (tid == NWG * kWG) prefetch_tensormap(&tmap);
+  // softmax scale in log2 units of this thread's row, times 2^e when the row's
+  // bf16 query was scaled by 2^-e before narrowing to f16 (quantized caches)
+  float sl2 = p.scale_log2;
   if (is_compute) {
     // row r of the warpgroup's Q tile, converted to the operand type, 16-byte chunks swizzled
     uint8_t* sQ = smem + Gm::oQ + wg * Gm::kQBytes;
     const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(p.q) + orow * 2);
+    float qmul = 1.f;
+    if constexpr (!Gm::k16 && QBF16) {
+      // the power of two 2^-e that brings the row's largest |q| into
+      // [2^13, 2^14): exact, and far from both ends of the f16 range
+      float mx = 0.f;
+      if (row_ok) {
+#pragma unroll 4
+        for (int c = 0; c < D / 8; ++c) {
+          const uint4 v = __ldg(src + c);
+          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            mx = fmaxf(mx, fmaxf(fabsf(__uint_as_float(w[i] << 16)), fabsf(__uint_as_float(w[i] & 0xFFFF0000u))));
+        }
+      }
+      const int ex = (mx > 0.f && mx <= FLT_MAX) ? ilogbf(mx) - 13 : 0;
+      qmul = ldexpf(1.f, -ex);
+      sl2 = p.scale_log2 * ldexpf(1.f, ex);
+    }
 #pragma unroll 4
     for (int c = 0; c < D / 8; ++c) {
       uint4 v = make_uint4(0, 0, 0, 0);
       if (row_ok) v = __ldg(src + c);
-      if constexpr (!Gm::k16 && QBF16) {  // bf16 query -> f16 operand
+      if constexpr (!Gm::k16 && QBF16) {  // bf16 query -> f16 operand, scaled by 2^-e
         uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 4; ++i) w[i] = to_f16x2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xFFFF0000u));
+        for (int i = 0; i < 4; ++i)
+          w[i] = to_f16x2(__uint_as_float(w[i] << 16) * qmul, __uint_as_float(w[i] & 0xFFFF0000u) * qmul);
         v = make_uint4(w[0], w[1], w[2], w[3]);
       }
       const int bx = c >> 3, ch = c & 7;
@@ -544,7 +568,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       if constexpr (Gm::kFp8) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float cj = p.scale_log2 * tile_sk[(t & 1) * 4 + j];
+          const float cj = sl2 * tile_sk[(t & 1) * 4 + j];
           vs[j] = tile_sv[(t & 1) * 4 + j];
 #pragma unroll
           for (int c = 16 * j; c < 16 * j + 16; ++c) xs[c] = __uint_as_float(sv[c]) * cj;
@@ -566,7 +590,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
 #pragma unroll
         for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], xs[c]);
         mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-        if constexpr (!Gm::kFp8) mx *= p.scale_log2;  // -inf stays -inf (the scale is positive)
+        if constexpr (!Gm::kFp8) mx *= sl2;  // -inf stays -inf (the scale is positive)
       }
       float fm = 1.f;  // rescale of l and O for a larger row max
       if (mx > m + kLazy) {
@@ -601,7 +625,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         for (int c = 0; c < 64; c += 2) {
           float ya, yb;
           if constexpr (Gm::kFp8) sub2(ya, yb, xs[c], xs[c + 1], mu, mu);
-          else fma2(ya, yb, xs[c], xs[c + 1], p.scale_log2, p.scale_log2, -mu, -mu);
+          else fma2(ya, yb, xs[c], xs[c + 1], sl2, sl2, -mu, -mu);
           const float pa = ex2(ya), pb = ex2(yb);
           const int i = (c >> 1) & 3;
           add2(ra[i], rb[i], ra[i], rb[i], pa, pb);
@@ -672,11 +696,13 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         *abort_flag = 1;
         raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
       }
-      // let products still in flight finish (each wait bounded)
+      // let products still in flight finish (each wait bounded by the full limit)
+      bool drained = true;
       for (int k = n_s_waited; k < n_s; ++k)
-        (void)mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.timeout_ns);
+        drained = mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.drain_ns) && drained;
       for (int k = n_pv_waited; k < pv_done; ++k)
-        (void)mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.timeout_ns);
+        drained = mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.drain_ns) && drained;
+      if (!drained) raise_flag(p.err, PQKV_DEVERR_DRAIN);
     } else {
       tc::fence_after_sync();
       const float inv = l > 0.f ? (Gm::kFp8 ? vref : 1.f) / l : 0.f;
@@ -704,8 +730,10 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   if (tid == 0) {
     // tiles issued but never consumed (only after a timeout) land before the CTA exits
     const int issued = *n_issued_slot;
+    bool drained = true;
     for (int k = n_prepared; k < issued; ++k)
-      (void)mbar_wait_bounded(&bar_full[k % kStages], (uint32_t)(k / kStages) & 1u, p.timeout_ns);
+      drained = mbar_wait_bounded(&bar_full[k % kStages], (uint32_t)(k / kStages) & 1u, p.drain_ns) && drained;
+    if (!drained) raise_flag(p.err, PQKV_DEVERR_DRAIN);
   }
   if (warp == 0) {
     tc::fence_after_sync();

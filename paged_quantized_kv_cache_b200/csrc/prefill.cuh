@@ -21,7 +21,8 @@ struct PrefillParams {
   int B, Hq, Hkv, G, nb, maxblk;
   int tiles_per_seq;            // 128-row query tiles per sequence (from the longest chunk)
   float scale_log2;             // softmax scale * log2(e)
-  uint64_t timeout_ns;
+  uint64_t timeout_ns;          // limit of a wait before the CTA gives up
+  uint64_t drain_ns;            // after giving up: limit of the wait for work still in flight
 };
 
 cudaError_t launch_prefill(int kv_dtype, int D, bool q_bf16, const CUtensorMap& tmap16, const PrefillParams& p,

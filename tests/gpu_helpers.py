@@ -1,5 +1,8 @@
 """Helpers for the GPU parity tests: drive the CUDA path (through the C ABI
 binding) and the CPU oracle on the same seeded inputs and compare them."""
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -66,9 +69,25 @@ def decode_gpu(g, q, block_tables, seq_lens, scale, split_blocks=0):
     return out, int(e.item())
 
 
+def _log_errors(tag, kv_dtype, d, ref, atol, rtol):
+    """With PQKV_PARITY_LOG set, append the achieved error of one comparison to
+    that file (JSON lines), so that the margin left under the tolerance is
+    on record, not only pass / fail."""
+    path = os.environ.get("PQKV_PARITY_LOG")
+    if not path or d.size == 0:
+        return
+    rec = {"test": os.environ.get("PYTEST_CURRENT_TEST", "").split(" ")[0], "tag": tag,
+           "kv_dtype": pq.DTYPE_NAMES.get(kv_dtype, str(kv_dtype)), "n": int(d.size),
+           "max_abs_err": float(d.max()), "tol_used": float((d / (atol + rtol * np.abs(ref))).max()),
+           "atol": atol, "rtol": rtol}
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
+
+
 def assert_close(out, ref, kv_dtype, tag=""):
     atol, rtol = TOL[kv_dtype]
     o = out.double().cpu().numpy()
+    _log_errors(tag, kv_dtype, np.abs(o - ref), ref, atol, rtol)
     bad = ~(np.abs(o - ref) <= atol + rtol * np.abs(ref))
     if bad.any():
         i = tuple(np.argwhere(bad)[0])

@@ -79,6 +79,21 @@ def test_invalid_arguments_are_rejected_before_any_launch():
         assert lib.pqkv_paged_decode_attention(null, pq.BF16, B, Hq, null, null, null, null, pq.BF16, 4, Hkv,
                                                128, null, 4, null, f, 0, null, null, 0, null,
                                                null) == pq.ERR_ARG
+        # the entry point without a workspace checks the same sizes first
+        assert lib.pqkv_paged_decode_attention_noalloc(null, pq.BF16, B, Hq, null, null, null, null, pq.BF16, 4,
+                                                       Hkv, 128, null, 4, null, f, 0, null, null,
+                                                       null) == pq.ERR_ARG
+    # 12 query heads per KV head (a workspace size exists for 16 columns, but a
+    # single-query decode takes at most 8): an argument error, not a scratch one
+    assert lib.pqkv_paged_decode_attention_noalloc(null, pq.BF16, 2, 96, null, null, null, null, pq.BF16, 4, 8,
+                                                   128, null, 4, null, f, 0, null, null, null) == pq.ERR_ARG
+    # no sequences: nothing to do, but only for arguments the call accepts
+    assert lib.pqkv_paged_decode_attention_noalloc(null, pq.BF16, 0, 32, null, null, null, null, pq.BF16, 4, 8,
+                                                   128, null, 4, null, f, 0, null, null, null) == pq.OK
+    assert lib.pqkv_paged_decode_attention_noalloc(null, pq.BF16, 0, 32, null, null, null, null, 9, 4, 8,
+                                                   128, null, 4, null, f, 0, null, null, null) == pq.ERR_ARG
+    assert lib.pqkv_paged_decode_attention_noalloc(null, pq.BF16, 0, 32, null, null, null, null, pq.BF16, 4, 8,
+                                                   96, null, 4, null, f, 0, null, null, null) == pq.ERR_ARG
     assert lib.pqkv_decode_workspace_init(null, 16, null) == pq.ERR_ARG
     # workspace sizes: 0 for sizes no call accepts (checked before any device query)
     # (batch, Hq, Hkv, D, max_blocks, split): Hq not a multiple of Hkv, 32 columns

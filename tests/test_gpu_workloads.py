@@ -28,6 +28,7 @@ CASES = [
     ("llama70b", None, 32),
     ("llama70b", "fp8_e4m3", 32),
     ("llama70b", None, 0),
+    ("llama70b", "fp8_e4m3", 0),
     ("fp4", None, 0),
 ]
 

@@ -74,12 +74,13 @@ def _oracle_cache(s, st, sample, q_len):
     return o, obt
 
 
-MQ = [("llama8b", None), ("fp8", "fp8_e4m3"), ("fp4", None)]
+# q_len 2: one 8-column tile; 4: two tiles (G = 4); 8: two passes of two tiles
+MQ = [("llama8b", None, 2), ("fp8", "fp8_e4m3", 2), ("fp4", None, 2),
+      ("llama8b", None, 4), ("llama8b", None, 8), ("fp8", "fp8_e4m3", 4), ("fp4", None, 4)]
 
 
-@pytest.mark.parametrize("name,kv", MQ, ids=["%s-%s" % (n, k or "default") for n, k in MQ])
-def test_full_size_multi_query_decode(name, kv):
-    q_len = 2
+@pytest.mark.parametrize("name,kv,q_len", MQ, ids=["%s-%s-q%d" % (n, k or "default", q) for n, k, q in MQ])
+def test_full_size_multi_query_decode(name, kv, q_len):
     s = bench.bench_spec(name, kv, q_len=q_len)
     st = bench.Setup(s, torch.device("cuda", 0), 0, q_len=q_len)
     st.write()

@@ -63,3 +63,5 @@ def test_reference_arm_under_torchrun_prints_once():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+    # the same config keys as our arm's line
+    assert {"context_tokens", "kv_bytes_per_step", "l2", "split_blocks"} <= set(d["config"])

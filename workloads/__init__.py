@@ -93,12 +93,12 @@ def spec(name: str, kv_dtype: Optional[int] = None, batch: Optional[int] = None)
 
 def _streams(s: Spec) -> List[np.random.SeedSequence]:
     # children 0..B-1: per-sequence K/V; B: lengths; B+1: physical ids; B+2: q;
-    # B+3: shared prefix K/V; B+4: outlier channel choice; B+5: multi-token q.
-    # The number of children depends only on the full batch of the named
-    # workload so that a batch cut keeps every sequence's stream (a child's
-    # stream depends on its index only).
+    # B+3: shared prefix K/V; B+4: outlier channel choice; B+5: multi-token q;
+    # B+6: stand-alone write-call inputs (write_kv). The number of children
+    # depends only on the full batch of the named workload so that a batch cut
+    # keeps every sequence's stream (a child's stream depends on its index only).
     full = spec(s.name).batch
-    return np.random.SeedSequence(s.seed).spawn(full + 6)
+    return np.random.SeedSequence(s.seed).spawn(full + 7)
 
 
 def seq_lens(s: Spec) -> np.ndarray:
@@ -212,6 +212,27 @@ def seq_kv(s: Spec, b: int, with_append: bool = True) -> Tuple[torch.Tensor, tor
             v[:, h, ch[h, 1]] *= s.outlier_gain
     in_dt = torch.float16 if s.kv_dtype == DT_FP16 else (
         torch.float16 if s.q_dtype == DT_FP16 else torch.bfloat16)
+    return torch.from_numpy(k).to(in_dt), torch.from_numpy(v).to(in_dt)
+
+
+def write_kv(s: Spec, b: int, start: int, n: int) -> Tuple[torch.Tensor, torch.Tensor]:
+    """K and V [n][Hkv][D] for positions start..start+n-1 of sequence b, for
+    timing a write call on its own: N(0,1) with the workload's planted outlier
+    channels, rounded to the input dtype, like seq_kv, but drawn from a stream
+    of their own (per sequence and start) so that no sequence's full stream is
+    needed. Not the values seq_kv gives for those positions."""
+    full = spec(s.name).batch
+    ss = np.random.SeedSequence(entropy=s.seed, spawn_key=_streams(s)[full + 6].spawn_key + (b, start))
+    rng = np.random.Generator(np.random.PCG64(ss))
+    H, D = s.num_kv_heads, s.head_dim
+    k = _normal(rng, (n, H, D))
+    v = _normal(rng, (n, H, D))
+    if s.outlier_channels:
+        ch = outlier_channels(s)
+        for h in range(H):
+            k[:, h, ch[h, 0]] *= s.outlier_gain
+            v[:, h, ch[h, 1]] *= s.outlier_gain
+    in_dt = TORCH_DTYPE[input_dtype(s)]
     return torch.from_numpy(k).to(in_dt), torch.from_numpy(v).to(in_dt)
 
 
