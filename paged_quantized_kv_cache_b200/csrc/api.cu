@@ -343,6 +343,7 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   mp.maxblk = max_blocks_per_seq;
   mp.split_blocks = split_blocks;
   mp.slot_floats = p.slot_floats;
+  mp.wpc = split_blocks > 0 ? 4 : 1;
   // passes run in stream order; each kernel waits for the previous one before
   // touching the workspace (programmatic dependents wait for the full grid)
   for (int q0 = 0; q0 < q_len; q0 += kp) {

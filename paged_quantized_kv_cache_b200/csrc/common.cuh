@@ -139,34 +139,31 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// mbarrier.try_wait with a suspend-time hint: the thread is suspended for at
-// most about hint_ns nanoseconds (instead of the system-dependent limit) when
-// the phase is not complete yet.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+// mbarrier.test_wait: whether the phase with `parity` has completed, without
+// waiting at all.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
 
-// Limits below this use the hinted try_wait, so that a wait can give up that
-// soon (a plain try_wait may stay suspended until the copy lands).
+// Limits below this poll with test_wait, so that a wait can give up that soon
+// (try_wait may keep the thread suspended until the copy lands).
 constexpr uint64_t kShortWaitNs = 1000000;
 
 // Wait until the phase with `parity` of `bar` completes, giving up after
 // `limit_ns` nanoseconds. Returns false on timeout.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
   if (limit_ns < kShortWaitNs) {
-    const uint32_t hint = (uint32_t)limit_ns;
-    if (mbar_try_wait_hint(bar, parity, hint)) return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-      if (mbar_try_wait_hint(bar, parity, hint)) return true;
+      if (mbar_test_wait(bar, parity)) return true;
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }

@@ -59,14 +59,39 @@ __device__ __forceinline__ void store_out(void* out, size_t i, float v) {
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
+// Four E4M3 codes -> f16x2 of bytes (0,1) and (2,3) by the hardware conversion
+// (true values; the FP4 group scales).
+__device__ __forceinline__ void dec4_e4m3_cvt(uint32_t r, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(r));
+}
+
+// E4M3 codes of the cache are decoded by placing their bits (true) or by the
+// hardware conversion (false); see dec4.
+constexpr bool kE4m3Place = true;
+// The placed f16 of an E4M3 code is its value times 2^-8 (bias 15 against 7).
+template <int KVF>
+constexpr float fp8_unit() { return (KVF == PQKV_DTYPE_FP8_E4M3 && kE4m3Place) ? 256.f : 1.f; }
+
 // Four FP8 codes of a word -> f16x2 of bytes (0,1) and of bytes (2,3), exact.
 // E5M2 codes are the high byte of the binary16 of the same value, so they are
-// placed, not converted.
+// placed, not converted. An E4M3 code s.eeee.mmm placed as the binary16
+// s.0eeee.mmm0000000 is its value times 2^-8 exactly (normals and subnormals:
+// the exponent biases are 15 and 7); the factor 2^8 (fp8_unit) is folded into
+// the logit scale of K and the output scale of V. In one word: a byte permute
+// puts code c0 in bits 15..8, its sign replicated in bits 23..16 and code c1 in
+// bits 31..24; an arithmetic shift by one then leaves each half as
+// s.s.eeee.mmm0000000 and a mask clears the second sign bit.
 template <int KVF>
 __device__ __forceinline__ void dec4(uint32_t r, uint32_t& lo, uint32_t& hi) {
   if constexpr (KVF == PQKV_DTYPE_FP8_E5M2) {
     lo = prmt(r, 0u, 0x1404u);
     hi = prmt(r, 0u, 0x3424u);
+  } else if constexpr (kE4m3Place) {
+    lo = (uint32_t)((int32_t)prmt(r, 0u, 0x1804u) >> 1) & 0xBF80BF80u;
+    hi = (uint32_t)((int32_t)prmt(r, 0u, 0x3A24u) >> 1) & 0xBF80BF80u;
   } else {
     asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
         "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
@@ -222,8 +247,8 @@ __device__ __forceinline__ void block_scores(uint32_t tb, const uint8_t* side,
       const uint32_t* rb = reinterpret_cast<const uint32_t*>(side + (g + 8) * SPR);
 #pragma unroll
       for (int w = 0; w < SPR / 4; ++w) {  // word w = groups 4w..4w+3 = chunks 2w, 2w+1
-        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(ra[w], 0u, sel), sa2[2 * w], sa2[2 * w + 1]);
-        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(rb[w], 0u, sel), sb2[2 * w], sb2[2 * w + 1]);
+        dec4_e4m3_cvt(prmt(ra[w], 0u, sel), sa2[2 * w], sa2[2 * w + 1]);
+        dec4_e4m3_cvt(prmt(rb[w], 0u, sel), sb2[2 * w], sb2[2 * w + 1]);
       }
     }
 #pragma unroll
@@ -360,8 +385,8 @@ __device__ __forceinline__ void block_pv(uint32_t tb, const uint8_t* side, const
       const uint32_t* w1 = reinterpret_cast<const uint32_t*>(vs + (ta + 1) * SPR);
 #pragma unroll
       for (int w = 0; w < SPR / 4; ++w) {
-        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], 0x5140u), sp[hh][4 * w], sp[hh][4 * w + 1]);
-        dec4<PQKV_DTYPE_FP8_E4M3>(prmt(w0[w], w1[w], 0x7362u), sp[hh][4 * w + 2], sp[hh][4 * w + 3]);
+        dec4_e4m3_cvt(prmt(w0[w], w1[w], 0x5140u), sp[hh][4 * w], sp[hh][4 * w + 1]);
+        dec4_e4m3_cvt(prmt(w0[w], w1[w], 0x7362u), sp[hh][4 * w + 2], sp[hh][4 * w + 3]);
       }
       if (valid < kBlock) {  // scales past the end may be NaN codes
 #pragma unroll
@@ -537,19 +562,26 @@ __device__ __forceinline__ bool arrive_split(const DecodeParams& p, int k0, int 
 
 // ---------------------------------------------------------------------------
 // Log-sum-exp merge of the split pairs of more than kMergeInKernel pieces (same
-// formula as merge_pair). One warp per (sequence b, KV head h, column n).
-// Launched as a programmatic dependent of the decode kernel: it rebuilds the
-// decode's split plan from seq_lens while that grid is still running, and its
-// warps whose pair needs nothing from it exit before waiting for the decode,
-// so with no long split pair the whole grid is done before the decode is.
-// Long pairs (few long sequences spread over the whole GPU) get B x Hkv x G
-// warps here instead of one warp at the end of the decode.
+// formula as merge_pair). CTAs of 4 warps; each output column (sequence b, KV
+// head h, column n) gets p.wpc warps: 1 with the balanced split (pairs have
+// few pieces; 4 columns per CTA keep the grid small) or 4 with a fixed split
+// (tens of pieces per pair). Launched as a programmatic dependent of the decode
+// kernel: it rebuilds the decode's split plan from seq_lens while that grid is
+// still running, and its warps whose pair needs nothing from it exit before
+// waiting for the decode, so with no long split pair the whole grid is done
+// before the decode is. Warp q of a column takes a contiguous share of the
+// pair's pieces and issues the loads of all of them (up to kBatch at a time)
+// together with the (m, l) of every piece, so that a merge costs about one
+// round trip to L2; the shares' weighted sums are added in order, so results
+// do not depend on timing.
 // ---------------------------------------------------------------------------
 template <int D, bool QBF16>
-__global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
+__global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p) {
   extern __shared__ int P[];  // [B + 1]: blocks of the sequences before b, as in the decode
   __shared__ int wsum[4];
-  constexpr int DPL = D / 32;
+  __shared__ float part[4][D];  // each warp's weighted sum of its pieces
+  constexpr int DPL = D / 32;   // head dims per lane
+  constexpr int kBatch = 16;    // pieces whose outputs a warp loads at once
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   {
     const int B = p.B, per = (B + 127) / 128;
@@ -580,10 +612,11 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
   }
   const int T = p.Hkv * P[p.B];
   const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + p.warps - 1) / p.warps);
-  const long wid = ((long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (wid >= (long)p.B * p.Hkv * p.G) return;
-  const int b = (int)(wid / ((long)p.Hkv * p.G));
-  const int h = (int)((wid / p.G) % p.Hkv), n = (int)(wid % p.G);
+  const int wpc = p.wpc, sh = warp % wpc;                // this warp's share of its column
+  const long cid = ((long)blockIdx.x * 4 + warp) / wpc;  // column
+  if (cid >= (long)p.B * p.Hkv * p.G) return;           // (the same for the warps of a column)
+  const int b = (int)(cid / ((long)p.Hkv * p.G));
+  const int h = (int)((cid / p.G) % p.Hkv), n = (int)(cid % p.G);
   const int nblk = P[b + 1] - P[b];
   if (nblk == 0) return;
   const int s0 = p.Hkv * P[b] + h * nblk;
@@ -594,54 +627,76 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
     const int kk = k0 + i;
     return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
   };
+  const int q0 = (int)((long)np * sh / wpc), q1 = (int)((long)np * (sh + 1) / wpc);  // this warp's pieces
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  // weights: lanes over pieces; lane i keeps piece i's (m, l) for the common np <= 32
-  float mi = kNegInf, li = 0.f;
-  if (lane < np) {
-    const float* bs = slot_base(lane);
-    mi = __ldcg(bs + p.G * D + n);
-    li = __ldcg(bs + p.G * D + p.G + n);
-  }
-  float M = mi;
-  for (int i = lane + 32; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
-  const float wi = (M == kNegInf || lane >= np) ? 0.f : exp2f(mi - M);
-  float L = wi * li;
-  for (int i = lane + 32; i < np; i += 32) {
-    const float* bs = slot_base(i);
-    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M) * __ldcg(bs + p.G * D + p.G + n);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
-  // outputs: lanes over head dims, pieces in order; the loads of up to 16
-  // pieces are all issued before the first one is folded in
-  float acc[DPL];
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  constexpr int kBatch = 16;
-  for (int i0 = 0; i0 < np; i0 += kBatch) {
-    float v[kBatch][DPL];
+  // the first batch of this warp's outputs, in flight with the (m, l) loads below
+  float v[kBatch][DPL];
+  auto load_batch = [&](int i0) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = i0 + u;
-      if (i < np) {
+      if (i < q1) {
         const float* bs = slot_base(i) + n * D + lane * DPL;
         if constexpr (DPL == 4) {
           const float4 t = __ldcg(reinterpret_cast<const float4*>(bs));
           v[u][0] = t.x; v[u][1] = t.y; v[u][2] = t.z; v[u][3] = t.w;
         } else {
-#pragma unroll
-          for (int e = 0; e < DPL; ++e) v[u][e] = __ldcg(bs + e);
+          const float2 t = __ldcg(reinterpret_cast<const float2*>(bs));
+          v[u][0] = t.x; v[u][1] = t.y;
         }
       }
     }
+  };
+  load_batch(q0);
+  // weights over all pieces: lanes over pieces (every warp computes the same M, L)
+  float mi[4], li[4];  // pieces lane, lane + 32, lane + 64, lane + 96
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int i = lane + 32 * r;
+    mi[r] = kNegInf;
+    li[r] = 0.f;
+    if (i < np) {
+      const float* bs = slot_base(i);
+      mi[r] = __ldcg(bs + p.G * D + n);
+      li[r] = __ldcg(bs + p.G * D + p.G + n);
+    }
+  }
+  float M = fmaxf(fmaxf(mi[0], mi[1]), fmaxf(mi[2], mi[3]));
+  for (int i = lane + 128; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
+  float wr[4];
+  float L = 0.f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    wr[r] = (M == kNegInf || mi[r] == kNegInf) ? 0.f : exp2f(mi[r] - M);
+    L += wr[r] * li[r];
+  }
+  for (int i = lane + 128; i < np; i += 32) {
+    const float* bs = slot_base(i);
+    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M) * __ldcg(bs + p.G * D + p.G + n);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
+  // this warp's weighted sum, pieces in order
+  float acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+  for (int i0 = q0; i0 < q1; i0 += kBatch) {
+    if (i0 > q0) load_batch(i0);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = i0 + u;
-      float w = __shfl_sync(kFull, wi, i & 31);
-      if (i < np) {
-        if (i >= 32) w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + p.G * D + n) - M);
+      if (i < q1) {  // the same on every lane
+        float w;
+        if (i < 128) {
+          const float wv = __shfl_sync(kFull, (i >> 5) == 0 ? wr[0] : (i >> 5) == 1 ? wr[1] : (i >> 5) == 2 ? wr[2]
+                                                                                                       : wr[3],
+                                       i & 31);
+          w = wv;
+        } else {
+          w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + p.G * D + n) - M);
+        }
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[e] += w * v[u][e];
       }
@@ -649,8 +704,22 @@ __global__ void __launch_bounds__(128) paged_merge_kernel(const MergeParams p) {
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const size_t orow = col_row(b, h, n, p.k, p.q0, p.Gh, p.Hq, D) + lane * DPL;
+  if (wpc == 1) {
 #pragma unroll
-  for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
+    for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
+    return;
+  }
+  // four shares of one column (all warps of the CTA are here): add them in order
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) part[warp][lane * DPL + e] = acc[e];
+  __syncthreads();
+  if (warp == 0) {
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) {
+      const int d = lane * DPL + e;
+      store_out<QBF16>(p.out, orow + e, (((part[0][d] + part[1][d]) + part[2][d]) + part[3][d]) * inv);
+    }
+  }
 }
 
 template <int KVF, int D, bool QBF16, int NT>
@@ -767,17 +836,20 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     j = rel - h * n;
   };
 
-  // This warp's chunks are k0, k0 + W, k0 + 2W, ... Its blocks, chunk after
-  // chunk, are numbered v = 0 .. Vtot - 1; the copy ring runs over v without a
-  // break at chunk boundaries, so the next chunk's first blocks are already on
-  // the way while a chunk drains.
+  // With a fixed split (split_blocks > 0) the K chunks go to Wa = ceil(K /
+  // rounds) warps, rounds = ceil(K / W), each taking `rounds` consecutive
+  // chunks (the last one fewer): every working warp has the same number of
+  // chunks, and a warp's chunks are mostly pieces of one (sequence, head)
+  // pair, so its query stays loaded from one chunk to the next. The balanced
+  // split has K <= W chunks, one per warp. A warp's blocks, chunk after chunk,
+  // are the flat blocks kbase * Qc + v, v = 0 .. Vtot - 1; the copy ring runs
+  // over v without a break at chunk boundaries.
   const int k0 = warp * gridDim.x + blockIdx.x;
-  const int nck = k0 < K ? (K - 1 - k0) / W + 1 : 0;
-  const int Vtot = nck == 0 ? 0 : (nck - 1) * Qc + (min(T, (k0 + (nck - 1) * W + 1) * Qc) - (k0 + (nck - 1) * W) * Qc);
-  auto vflat = [&](int v) {  // virtual block index -> flat block index
-    const int i = v / Qc;
-    return (k0 + i * W) * Qc + (v - i * Qc);
-  };
+  const int rounds = K > 0 ? (K + W - 1) / W : 1;
+  const int kbase = k0 * rounds;
+  const int nck = kbase < K ? min(K, kbase + rounds) - kbase : 0;
+  const int Vtot = nck == 0 ? 0 : min(T, (kbase + nck) * Qc) - kbase * Qc;
+  auto vflat = [&](int v) { return kbase * Qc + v; };  // virtual block index -> flat block index
   // Per-lane window of (physical id, head) for blocks wbase + lane and, loaded
   // ahead, wbase + 32 + lane. Values are only inspected when issued.
   auto load_entry = [&](int v, int& id, int& hh) {
@@ -834,27 +906,33 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
   for (int i = 0; i < min(NS, Vtot); ++i) issue(i, i);
   int s = 0;  // stage of the next block to consume
 
+  // ---- consumer state of the current (sequence, head) piece ----
+  int b = 0, h = 0, j = 0;
+  int nblk = 0, Lb = 0;
+  bool started_before = false;
+  uint32_t qf[NT][KT][2];
+  float acc[NT][KT][4];
+  float mm[NT][2], ll[NT][2], vref;  // running max and sum of each of the lane's columns
+  // softmax scale (log2 units) of each of the lane's columns, times the power
+  // of two its query row was scaled down by before narrowing to f16
+  // (quantized caches; 16-bit caches keep the query in its own type)
+  float csc[NT][2];
+  OutlierState<NT> ost;  // FP4 only
+  int qb = -1, qh = -1;  // the pair whose query is loaded
+
   for (int ci = 0; ci < nck && !aborted; ++ci) {
-    const int k = k0 + ci * W;
+    const int k = kbase + ci;
     const int f0 = k * Qc;
     const int f1 = min(T, f0 + Qc);
     const int vb = ci * Qc - f0;  // v = f + vb inside this chunk
 
-    // ---- consumer state of the current (sequence, head) piece ----
-    int b, h, j;
     locate(f0, b, h, j);
-    int nblk = P[b + 1] - P[b];
-    int Lb = p.seq_lens[b];
-    bool started_before = j > 0;
-    uint32_t qf[NT][KT][2];
-    float acc[NT][KT][4];
-    float mm[NT][2], ll[NT][2], vref;  // running max and sum of each of the lane's columns
-    // softmax scale (log2 units) of each of the lane's columns, times the power
-    // of two its query row was scaled down by before narrowing to f16
-    // (quantized caches; 16-bit caches keep the query in its own type)
-    float csc[NT][2];
-    OutlierState<NT> ost;  // FP4 only
+    nblk = P[b + 1] - P[b];
+    Lb = p.seq_lens[b];
+    started_before = j > 0;
 
+    // a new piece: zero the softmax state; load the pair's query unless the
+    // previous piece of this warp was of the same pair
     auto begin_piece = [&]() {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -864,7 +942,10 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
         for (int mt = 0; mt < KT; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
       }
       vref = 0.f;
-      ost.reset();  // the query changes with the piece
+      if (b == qb && h == qh) return;
+      qb = b;
+      qh = h;
+      ost.reset();  // the query changes
       float rowmul[NT];  // quantized caches: 2^-e applied to this lane's query row 8nt + g
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
@@ -915,7 +996,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const float m = __shfl_sync(kFull, rowmul[nt], (2 * qd + c) << 2);
-        csc[nt][c] = (Gm::k16 || !QBF16) ? p.scale_log2 : p.scale_log2 / m;  // 1 / m = 2^e: exact
+        csc[nt][c] = ((Gm::k16 || !QBF16) ? p.scale_log2 : p.scale_log2 / m) * fp8_unit<KVF>();  // exact
       }
       }
       if constexpr (Gm::kFp4) {
@@ -944,7 +1025,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
           lt[nt][1] += __shfl_xor_sync(kFull, lt[nt][1], o);
         }
       }
-      const float vs = Gm::kFp8 ? vref : 1.f;
+      const float vs = Gm::kFp8 ? vref * fp8_unit<KVF>() : 1.f;
       if constexpr (Gm::kFp4) {  // fold the outlier channels' O in and clear it
         ost.template flush<Gm::kOStride>(woext, lane, D);
 #pragma unroll
@@ -1264,7 +1345,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
 // stream as a programmatic dependent (its launch overlaps the decode's tail;
 // griddepcontrol.wait inside it orders it after the decode grid).
 cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st) {
-  const long warps = (long)p.B * p.Hkv * p.G;  // one per (sequence, KV head, column)
+  const long warps = (long)p.B * p.Hkv * p.G * p.wpc;  // wpc per (sequence, KV head, column)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
   cfg.blockDim = dim3(128);

@@ -72,6 +72,7 @@ struct MergeParams {
   int warps;         // warps of the decode grid (its balanced chunk length depends on it)
   int split_blocks;
   int slot_floats;
+  int wpc;           // warps per output column: 1 (4 columns per CTA) or 4 (one column per CTA)
 };
 
 // Compile-time geometry of one format; NT = tiles of 8 MMA columns (query rows)

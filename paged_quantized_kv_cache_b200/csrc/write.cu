@@ -14,6 +14,7 @@
 // hardware cvt with round-to-nearest-even and saturation; the FP4 outlier
 // statistics are summed in fp64 in channel order on one lane.
 #include <algorithm>
+#include <cfloat>
 
 #include "write.cuh"
 
@@ -177,48 +178,148 @@ __global__ void __launch_bounds__(128) write_fp8_kernel(const WriteParams p) {
 }
 
 // ---- FP4 E2M1 + FP16 outlier channels ----
+
+// x / d rounded to nearest even, for d a positive E4M3 value and r = 1 / d
+// rounded to nearest (__frcp_rn): the product x r is corrected once by its
+// residual x - d (x r), which an FMA computes exactly (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000 processor",
+// IBM J. Res. Develop. 34(1), 1990). The sign of a zero result is not kept;
+// the encoder takes signs from x. The write's codes built on it are checked
+// bit for bit against the oracle's IEEE division for every bf16 and fp16 input
+// value and every E4M3 group scale that can occur together (tests).
+__device__ __forceinline__ float div_by_scale(float x, float d, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q0, d, x);
+  return __fmaf_rn(e, r, q0);
+}
+
+// 16 quotients -> 16 E2M1 codes (channel 2i in the low nibble of byte i), the
+// sign bit of each code taken from its input x (so that -0 and negative values
+// rounding to zero keep their sign).
+__device__ __forceinline__ uint2 e2m1_codes16(const float (&x)[16], float d, float r) {
+  uint32_t w[2];
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t c = 0, sg = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float a = x[8 * h + 2 * k], b = x[8 * h + 2 * k + 1];
+      uint32_t byte;
+      asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+          : "=r"(byte)
+          : "f"(fabsf(div_by_scale(b, d, r))), "f"(fabsf(div_by_scale(a, d, r))));
+      c |= byte << (8 * k);
+      sg |= ((__float_as_uint(a) >> 31) << (8 * k + 3)) | ((__float_as_uint(b) >> 31) << (8 * k + 7));
+    }
+    w[h] = c | sg;
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// Lane layout: lane l takes the 16 channels of group g = l % GPL (GPL = D / 16
+// groups per token) for block rows tl, tl + TL, ... (tl = l / GPL, TL = 32 /
+// GPL): a token-group's absmax, scale and codes stay in one lane, and the two
+// rows of a V token pair (r, r ^ 1) sit in lanes l and l ^ GPL.
 template <int D, bool INBF16>
 __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
   // inputs may come from the previous kernel; let the next one start launching
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  constexpr int CPL = D / 32;          // channels per lane
-  constexpr int LPG = kGroup / CPL;    // lanes per 16-channel group
+  constexpr int GPL = D / kGroup;    // groups per token: 8 or 4
+  constexpr int TL = 32 / GPL;       // lanes per group: 4 or 8
+  constexpr int TPL = kBlock / TL;   // block rows per lane: 4 or 2
+  constexpr int PREC = INBF16 ? 8 : 11;  // significant bits of an input value
   __shared__ float s_norm[4][D];
+  __shared__ int s_oc[4][kOutSlots];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane % GPL, tl = lane / GPL;
   const int win = blockIdx.x * 4 + warp;
   const int h = blockIdx.y, kv = blockIdx.z;
   const int t = win * p.tpw + lane;
   uint32_t starts = run_starts(p, t, lane < p.tpw, h == 0 && kv == 0);
   while (starts) {
-    const int i = __ffs(starts) - 1;
+    const int i0 = __ffs(starts) - 1;
     starts &= starts - 1;
-    const int ts = win * p.tpw + i;
+    const int ts = win * p.tpw + i0;
     const int s0 = p.slots[ts];
     const int n = run_length(p, ts, s0, lane);
     const int blk = s0 >> 4, off0 = s0 & 15;
-    const size_t pair = (size_t)blk * p.Hkv + h;
-    {
-      const void* x = kv ? p.v : p.k;
-      const size_t tile = pair * 2 + kv;  // (block, head, K|V) index
-      float xs[kBlock][CPL];
-      float nrm[CPL];
+    const size_t tile = ((size_t)blk * p.Hkv + h) * 2 + kv;  // (block, head, K|V) index
+    const auto* x = reinterpret_cast<const uint16_t*>(kv ? p.v : p.k);
+    // this lane's rows of the run (rows outside it read as zeros)
+    float xs[TPL][16];
 #pragma unroll
-      for (int e = 0; e < CPL; ++e) nrm[e] = 0.f;
+    for (int i = 0; i < TPL; ++i) {
+      const int r = tl + TL * i, j = r - off0;
+      uint4 u0 = make_uint4(0, 0, 0, 0), u1 = u0;
+      if (j >= 0 && j < n) {
+        const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)(ts + j) * p.Hkv + h) * D + kGroup * g);
+        u0 = __ldg(src);
+        u1 = __ldg(src + 1);
+      }
+      const uint32_t w[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
 #pragma unroll
-      for (int j = 0; j < kBlock; ++j) {
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) {
-          xs[j][e] = (j < n) ? in_at<INBF16>(x, ((size_t)(ts + j) * p.Hkv + h) * D + lane * CPL + e) : 0.f;
-          nrm[e] = fmaxf(nrm[e], fabsf(xs[j][e]));
+      for (int k = 0; k < 8; ++k) {
+        if constexpr (INBF16) {
+          xs[i][2 * k] = __uint_as_float(w[k] << 16);
+          xs[i][2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        } else {
+          xs[i][2 * k] = __half2float(__ushort_as_half((unsigned short)(w[k] & 0xFFFFu)));
+          xs[i][2 * k + 1] = __half2float(__ushort_as_half((unsigned short)(w[k] >> 16)));
         }
       }
-      uint8_t* idxp = p.oidx + tile * kIdxStride;
-      int oc[kOutSlots];  // outlier channels (>= D: empty)
-      if (off0 == 0) {
-        // step 1: channel norms; step 2: mu + 3.2 sigma over the D norms (fp64, channel order)
+    }
+    uint8_t* idxp = p.oidx + tile * kIdxStride;
+    int oc[kOutSlots];  // outlier channels, ascending (>= D: empty)
+    if (off0 == 0) {
+      // step 1: channel norms (L-inf over the run's tokens), the same on every
+      // lane of a group
+      float nrm[16];
 #pragma unroll
-        for (int e = 0; e < CPL; ++e) s_norm[warp][lane * CPL + e] = nrm[e];
+      for (int c = 0; c < 16; ++c) {
+        nrm[c] = fabsf(xs[0][c]);
+#pragma unroll
+        for (int i = 1; i < TPL; ++i) nrm[c] = fmaxf(nrm[c], fabsf(xs[i][c]));
+      }
+#pragma unroll
+      for (int o = GPL; o < 32; o <<= 1)
+#pragma unroll
+        for (int c = 0; c < 16; ++c) nrm[c] = fmaxf(nrm[c], __shfl_xor_sync(kFull, nrm[c], o));
+      // step 2: mu + 3.2 sigma of the D norms, in fp64 as the channel-order sums
+      // S1 = sum n, S2 = sum n^2. Norms are input values (PREC significant
+      // bits); when the nonzero ones span at most 23 - PREC binades, every
+      // partial sum of n and of n^2 is exact in fp64 (< 2^53 units of the
+      // smallest term), so any order of summation gives the channel-order
+      // result and the lanes add theirs in a tree. Otherwise: channel order.
+      float mx = 0.f, mn = FLT_MAX;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        mx = fmaxf(mx, nrm[c]);
+        mn = fminf(mn, nrm[c] > 0.f ? nrm[c] : FLT_MAX);
+      }
+#pragma unroll
+      for (int o = 1; o < GPL; o <<= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, o));
+        mn = fminf(mn, __shfl_xor_sync(kFull, mn, o));
+      }
+      const bool exact = (mx == 0.f) || (mn >= FLT_MIN && ilogbf(mx) - ilogbf(mn) <= 23 - PREC);
+      double s1 = 0.0, s2 = 0.0;
+      if (exact) {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const double v = (double)nrm[c];
+          s1 = __dadd_rn(s1, v);
+          s2 = __dadd_rn(s2, __dmul_rn(v, v));
+        }
+#pragma unroll
+        for (int o = 1; o < GPL; o <<= 1) {
+          s1 = __dadd_rn(s1, __shfl_xor_sync(kFull, s1, o));
+          s2 = __dadd_rn(s2, __shfl_xor_sync(kFull, s2, o));
+        }
+      } else {
+        if (tl == 0)
+#pragma unroll
+          for (int c = 0; c < 16; ++c) s_norm[warp][kGroup * g + c] = nrm[c];
         __syncwarp();
         double acc = 0.0;
         if (lane == 0) {
@@ -229,138 +330,172 @@ __global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
             acc = __dadd_rn(acc, __dmul_rn(v, v));
           }
         }
-        const double s2 = __shfl_sync(kFull, acc, 1);
-        double thr = 0.0;
-        if (lane == 0) {
-          const double mu = __ddiv_rn(acc, (double)D);
-          double var = __dsub_rn(__ddiv_rn(s2, (double)D), __dmul_rn(mu, mu));
-          if (var < 0.0) var = 0.0;
-          thr = __dadd_rn(mu, __dmul_rn(3.2, __dsqrt_rn(var)));
-        }
-        thr = __shfl_sync(kFull, thr, 0);
+        s1 = __shfl_sync(kFull, acc, 0);
+        s2 = __shfl_sync(kFull, acc, 1);
         __syncwarp();
-        // keep at most 4: largest norm first, ties to the lower channel
-        uint32_t cand = 0;
+      }
+      const double mu = __ddiv_rn(s1, (double)D);
+      double var = __dsub_rn(__ddiv_rn(s2, (double)D), __dmul_rn(mu, mu));
+      if (var < 0.0) var = 0.0;
+      const double thr = __dadd_rn(mu, __dmul_rn(3.2, __dsqrt_rn(var)));
+      uint32_t cand = 0;
 #pragma unroll
-        for (int e = 0; e < CPL; ++e)
-          if ((double)nrm[e] >= thr) cand |= 1u << e;
-        int nsel = 0;
+      for (int c = 0; c < 16; ++c)
+        if ((double)nrm[c] >= thr) cand |= 1u << c;
+      // candidates of the groups before this lane's (a scan within the GPL lanes of a row)
+      int incl = __popc(cand);
 #pragma unroll
-        for (int r = 0; r < kOutSlots; ++r) oc[r] = 0xFF;
+      for (int o = 1; o < GPL; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (g >= o) incl += v;
+      }
+      const int before = incl - __popc(cand);
+      int total = __popc(cand);
+#pragma unroll
+      for (int o = 1; o < GPL; o <<= 1) total += __shfl_xor_sync(kFull, total, o);
+      if (total <= kOutSlots) {
+        // all candidates, in channel order
+        if (tl == 0) {
+          int k = before;
+          uint32_t m = cand;
+          while (m) {
+            const int c = __ffs(m) - 1;
+            m &= m - 1;
+            s_oc[warp][k++] = kGroup * g + c;
+          }
+        }
+        if (lane == 0)
+          for (int k = total; k < kOutSlots; ++k) s_oc[warp][k] = 0xFF;
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < kOutSlots; ++r) oc[r] = s_oc[warp][r];
+        __syncwarp();
+      } else {
+        // keep 4: largest norm first, ties to the lower channel; then ascending
+#pragma unroll
         for (int r = 0; r < kOutSlots; ++r) {
           float bv = -1.f;
           int bc = 0x7FFFFFFF;
 #pragma unroll
-          for (int e = 0; e < CPL; ++e)
-            if ((cand >> e) & 1u) {
-              if (nrm[e] > bv) { bv = nrm[e]; bc = lane * CPL + e; }
+          for (int c = 0; c < 16; ++c)
+            if (((cand >> c) & 1u) && nrm[c] > bv) {
+              bv = nrm[c];
+              bc = kGroup * g + c;
             }
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
+          for (int o = 1; o < GPL; o <<= 1) {
             const float ov = __shfl_xor_sync(kFull, bv, o);
             const int occ = __shfl_xor_sync(kFull, bc, o);
-            if (ov > bv || (ov == bv && occ < bc)) { bv = ov; bc = occ; }
+            if (ov > bv || (ov == bv && occ < bc)) {
+              bv = ov;
+              bc = occ;
+            }
           }
-          if (bc == 0x7FFFFFFF) break;
-          oc[nsel++] = bc;
-          if (bc / CPL == lane) cand &= ~(1u << (bc % CPL));
+          oc[r] = bc;  // a candidate exists in every round (more than 4 of them)
+          if ((bc >> 4) == g) cand &= ~(1u << (bc & 15));
         }
-        // ascending order
 #pragma unroll
         for (int a2 = 1; a2 < kOutSlots; ++a2)
 #pragma unroll
           for (int b2 = kOutSlots - 1; b2 >= a2; --b2)
-            if (oc[b2 - 1] > oc[b2]) { const int tmp = oc[b2]; oc[b2] = oc[b2 - 1]; oc[b2 - 1] = tmp; }
-        if (lane == 0) {
-          const uint32_t lo = (uint32_t)oc[0] | ((uint32_t)oc[1] << 8) | ((uint32_t)oc[2] << 16) | ((uint32_t)oc[3] << 24);
-          reinterpret_cast<uint32_t*>(idxp)[0] = lo;
-          reinterpret_cast<uint32_t*>(idxp)[1] = 0xFFFFFFFFu;
-        }
-      } else {
-        const uint32_t lo = *reinterpret_cast<const uint32_t*>(idxp);
-#pragma unroll
-        for (int r = 0; r < kOutSlots; ++r) oc[r] = (lo >> (8 * r)) & 0xFF;
-      }
-      bool is_out[CPL];
-#pragma unroll
-      for (int e = 0; e < CPL; ++e) {
-        const int c = lane * CPL + e;
-        is_out[e] = (c == oc[0]) || (c == oc[1]) || (c == oc[2]) || (c == oc[3]);
-      }
-      // step 3: per token, fp16 outlier values, E4M3 group scales, E2M1 codes
-      uint32_t vpend = 0;  // V codes of the even token of a pair, stored with its partner
-#pragma unroll
-      for (int j = 0; j < kBlock; ++j) {
-        if (j >= n) break;
-        const int row = off0 + j;
-        // outlier buffer: lane r (< 4) stores slot r of this token
-        {
-          float ov = 0.f;
-          int owner = 0, el = 0;
-          const int r = lane & 3;
-          const int c = oc[r];
-          if (c < D) { owner = c / CPL; el = c % CPL; }
-          float mine[CPL];
-#pragma unroll
-          for (int e = 0; e < CPL; ++e) mine[e] = xs[j][e];
-          float got = 0.f;
-#pragma unroll
-          for (int e = 0; e < CPL; ++e) {
-            const float v = __shfl_sync(kFull, mine[e], owner);
-            if (e == el) got = v;
-          }
-          ov = (c < D) ? got : 0.f;
-          if (lane < kOutSlots) {
-            __half hv = (c < D) ? __float2half_rn(ov) : __ushort_as_half((unsigned short)0);
-            reinterpret_cast<__half*>(p.oval)[(tile * kBlock + row) * kOutSlots + lane] = hv;
-          }
-        }
-        float a = 0.f;
-#pragma unroll
-        for (int e = 0; e < CPL; ++e)
-          if (!is_out[e]) a = fmaxf(a, fabsf(xs[j][e]));
-#pragma unroll
-        for (int o = 1; o < LPG; o <<= 1) a = fmaxf(a, __shfl_xor_sync(kFull, a, o));
-        const uint32_t sc = enc_fp8x2<PQKV_DTYPE_FP8_E4M3>(__fdiv_rn(a, 6.0f), 0.f) & 0xFFu;
-        const float sd = e4m3_value(sc);
-        float y[CPL];
-#pragma unroll
-        for (int e = 0; e < CPL; ++e) y[e] = (is_out[e] || sd == 0.f) ? 0.f : __fdiv_rn(xs[j][e], sd);
-        const uint32_t c01 = enc_e2m1x2(y[0], y[1]);
-        const uint32_t c23 = (CPL == 4) ? enc_e2m1x2(y[2], y[3]) : 0u;
-        if (kv == 0) {
-          // K: one row per token, channel 2i in the low nibble of byte i
-          uint8_t* crow = p.cache + (tile * kBlock + row) * (D / 2) + lane * (CPL / 2);
-          if constexpr (CPL == 4)
-            *reinterpret_cast<uint16_t*>(crow) = (uint16_t)(c01 | (c23 << 8));
-          else
-            *crow = (uint8_t)c01;
-        } else {
-          // V: a byte holds one channel of a token pair (even token in the low
-          // nibble). Pairs inside the run are stored whole; a pair split by the
-          // run's ends keeps the other token's nibbles.
-          const uint32_t cw = (c01 & 0xFu) | ((c01 >> 4) << 8) | ((c23 & 0xFu) << 16) | ((c23 >> 4) << 24);
-          const int pr = (row < 8) ? (row & ~1) : (((row - 8) & ~1) + 1);
-          const int cb = lane * CPL;
-          uint8_t* vb = p.cache + (tile * kBlock + 8 * (cb / (D / 2)) + pr) * (D / 2) + cb % (D / 2);
-          const bool odd = row & 1;
-          if (!odd && j + 1 < n) {
-            vpend = cw;
-          } else {
-            const int sh = odd ? 4 : 0;
-            uint32_t keep = odd ? 0x0F0F0F0Fu : 0xF0F0F0F0u, put = cw << sh;
-            if (odd && j > 0) { keep = 0u; put |= vpend; }
-            if constexpr (CPL == 4) {
-              uint32_t* w = reinterpret_cast<uint32_t*>(vb);
-              *w = (keep ? (*w & keep) : 0u) | put;
-            } else {
-              uint16_t* w = reinterpret_cast<uint16_t*>(vb);
-              *w = (uint16_t)((keep ? (*w & keep) : 0u) | put);
+            if (oc[b2 - 1] > oc[b2]) {
+              const int tmp = oc[b2];
+              oc[b2] = oc[b2 - 1];
+              oc[b2 - 1] = tmp;
             }
-          }
+      }
+      if (lane == 0) {
+        reinterpret_cast<uint32_t*>(idxp)[0] =
+            (uint32_t)oc[0] | ((uint32_t)oc[1] << 8) | ((uint32_t)oc[2] << 16) | ((uint32_t)oc[3] << 24);
+        reinterpret_cast<uint32_t*>(idxp)[1] = 0xFFFFFFFFu;
+      }
+    } else {
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(idxp);
+#pragma unroll
+      for (int r = 0; r < kOutSlots; ++r) oc[r] = (lo >> (8 * r)) & 0xFF;
+    }
+    // step 3a: the fp16 outlier buffer, lane (row, slot) for 8 rows at a time,
+    // read again from the input (the values are in L1/L2)
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int r = (lane >> 2) + 8 * half, slot = lane & 3, j = r - off0;
+      if (j >= 0 && j < n) {
+        int c = 0xFF;
+#pragma unroll
+        for (int k = 0; k < kOutSlots; ++k)
+          if (k == slot) c = oc[k];
+        unsigned short hv = 0;
+        if (c < D) {
+          const uint16_t raw = x[((size_t)(ts + j) * p.Hkv + h) * D + c];
+          hv = INBF16 ? __half_as_ushort(__float2half_rn(__uint_as_float((uint32_t)raw << 16))) : raw;
         }
-        if ((lane % LPG) == 0)
-          p.scales[(tile * kBlock + row) * (D / kGroup) + (lane * CPL) / kGroup] = (uint8_t)sc;
+        reinterpret_cast<unsigned short*>(p.oval)[(tile * kBlock + r) * kOutSlots + slot] = hv;
+      }
+    }
+    // outlier channels of this lane's group get code 0 and stay out of the
+    // group absmax: zero them
+    uint32_t om = 0;
+#pragma unroll
+    for (int r = 0; r < kOutSlots; ++r)
+      if (oc[r] < D && (oc[r] >> 4) == g) om |= 1u << (oc[r] & 15);
+    if (om) {
+#pragma unroll
+      for (int i = 0; i < TPL; ++i)
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          if ((om >> c) & 1u) xs[i][c] = 0.f;
+    }
+    // step 3b: per row, E4M3 group scale and E2M1 codes
+#pragma unroll
+    for (int i = 0; i < TPL; ++i) {
+      const int r = tl + TL * i, j = r - off0;
+      const bool act = j >= 0 && j < n;
+      float a = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) a = fmaxf(a, fabsf(xs[i][c]));
+      const uint32_t sc = enc_fp8x2<PQKV_DTYPE_FP8_E4M3>(__fdiv_rn(a, 6.0f), 0.f) & 0xFFu;
+      const float sd = e4m3_value(sc);
+      uint2 codes = make_uint2(0u, 0u);
+      if (sd > 0.f) codes = e2m1_codes16(xs[i], sd, __frcp_rn(sd));
+      if (act) p.scales[(tile * kBlock + r) * GPL + g] = (uint8_t)sc;
+      if (kv == 0) {
+        // K: one row per token
+        if (act) *reinterpret_cast<uint2*>(p.cache + (tile * kBlock + r) * (D / 2) + 8 * g) = codes;
+      } else {
+        // V: a byte holds one channel of a token pair (even row in the low
+        // nibble); the partner row sits in lane ^ GPL. A pair split by the
+        // run's ends keeps the other row's nibbles.
+        const uint32_t o0 = __shfl_xor_sync(kFull, codes.x, GPL);
+        const uint32_t o1 = __shfl_xor_sync(kFull, codes.y, GPL);
+        const bool pact = (r ^ 1) - off0 >= 0 && (r ^ 1) - off0 < n;
+        const bool even = (r & 1) == 0;
+        if (act && (even || !pact)) {
+          const uint32_t e0 = even ? codes.x : o0, e1 = even ? codes.y : o1;  // even row's codes
+          const uint32_t d0 = even ? o0 : codes.x, d1 = even ? o1 : codes.y;  // odd row's codes
+          // channel 2k of the even row -> low nibble, of the odd row -> high nibble
+          auto spread = [](uint32_t ev, uint32_t od) -> uint4 {
+            const uint32_t lo_e = ev & 0x0F0F0F0Fu, hi_e = (ev >> 4) & 0x0F0F0F0Fu;
+            const uint32_t lo_o = (od & 0x0F0F0F0Fu) << 4, hi_o = od & 0xF0F0F0F0u;
+            const uint32_t ce = lo_e | lo_o;  // channels 0, 2, 4, 6 (bytes)
+            const uint32_t co = hi_e | hi_o;  // channels 1, 3, 5, 7
+            return make_uint4(prmt(ce, co, 0x5140u), prmt(ce, co, 0x7362u), 0u, 0u);
+          };
+          const uint4 lo8 = spread(e0, d0), hi8 = spread(e1, d1);
+          uint4 out = make_uint4(lo8.x, lo8.y, hi8.x, hi8.y);
+          const int pr = (r < 8) ? (r & ~1) : (((r - 8) & ~1) + 1);
+          const int cb = kGroup * g;
+          uint4* dst = reinterpret_cast<uint4*>(p.cache + (tile * kBlock + 8 * (cb / (D / 2)) + pr) * (D / 2) +
+                                                cb % (D / 2));
+          if (!pact) {  // only this row: keep the partner's nibbles
+            const uint4 cur = *dst;
+            const uint32_t keep = even ? 0xF0F0F0F0u : 0x0F0F0F0Fu;
+            out.x = (cur.x & keep) | (out.x & ~keep);
+            out.y = (cur.y & keep) | (out.y & ~keep);
+            out.z = (cur.z & keep) | (out.z & ~keep);
+            out.w = (cur.w & keep) | (out.w & ~keep);
+          }
+          *dst = out;
+        }
       }
     }
   }
