@@ -615,8 +615,8 @@ def measure_decode(args, s: W.Spec, device, world: int, kv_list=None, keep_kv: b
                 "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype], args.split_blocks),
                 "kernel": "paged_decode_kernel", "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, "
                 "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms,
-                "timing": "CUDA events around each decode call (per pass: decode kernel, merge kernel of long split "
-                          "pairs) over K further steps"}
+                "timing": "CUDA events around each decode call (one decode kernel per pass, which also merges the "
+                          "split pairs) over K further steps"}
     e2e = run_e2e(st, args, world) if not args.no_e2e else None
     value = b["kv"] * world / (ms_step * 1e-3) / 1e9
     m = {"value": value, "ms_per_step": ms_step,
@@ -626,9 +626,8 @@ def measure_decode(args, s: W.Spec, device, world: int, kv_list=None, keep_kv: b
          # the decode call alone (no cache write): B x q_len / t(decode)
          "decode_only_tok_s_per_layer": s.batch * args.q_len * world / (dec_ms * 1e-3),
          "decode_kernel_ms": dec_ms, "write_kernel_ms": wr_ms, "roofline": roofline, "e2e": e2e,
-         # per step: cache write, then per decode pass the split decode and the merge kernel of
-         # long split pairs (short ones are merged inside the decode)
-         "gpu_launches": (1 + 2 * decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
+         # per step: cache write, then one decode kernel per pass (it merges the split pairs itself)
+         "gpu_launches": (1 + decode_passes(args.q_len, s.num_q_heads // s.num_kv_heads)) * K,
          "clocks": clocks.summary()}
     return m, st
 

@@ -15,8 +15,6 @@ namespace pqkv {
 cudaError_t launch_decode(int kv_dtype, int D, bool q_bf16, int nt, const CUtensorMap& tmap, const DecodeParams& p,
                           int grid, cudaStream_t st);
 size_t decode_smem_bytes(int kv_dtype, int D, int B, int nt);
-int decode_warps(int kv_dtype, int D, int nt);
-cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st);
 size_t read_probe_smem_bytes(int B);
 cudaError_t launch_read_probe(const uint8_t* cache, int kv_dtype, int nb, int H, int D, const int32_t* block_tables,
                               int maxblk, const int32_t* seq_lens, int B, uint32_t* checksum, int32_t* err,
@@ -217,11 +215,13 @@ int pqkv_kv_cache_write(const void* k, const void* v, int in_dtype, int num_toke
   return e == cudaSuccess ? PQKV_OK : PQKV_ERR_CUDA;
 }
 
-// Upper bound of the decode's chunks (each has two partial slots and one
-// arrival word in the workspace).
+// Upper bound of the decode's units (each has two partial slots and one
+// arrival word in the workspace): one per warp with the balanced split; with
+// a fixed split, the split's chunks plus the warps' share boundaries inside them.
 static size_t decode_chunks(int batch, int num_kv_heads, int max_blocks_per_seq, int split_blocks, int sms) {
   const size_t total_blocks = (size_t)batch * num_kv_heads * max_blocks_per_seq;
-  return split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks : (size_t)sms * kDecodeWarps;
+  const size_t warps = (size_t)sms * kDecodeWarps;
+  return split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks + warps : warps;
 }
 
 // Launch tags of the decode's arrival words: 40 bits, never 0, so a zeroed
@@ -331,30 +331,14 @@ static int decode_impl(const void* q, int q_dtype, int batch, int q_len, int num
   p.counters = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) +
                                                      2 * chunks * (size_t)p.slot_floats * sizeof(float));
   const cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  MergeParams mp;
-  mp.seq_lens = seq_lens;
-  mp.partials = p.partials;
-  mp.out = out;
-  mp.B = batch;
-  mp.Hq = num_q_heads;
-  mp.Hkv = num_kv_heads;
-  mp.k = p.k;
-  mp.Gh = p.Gh;
-  mp.maxblk = max_blocks_per_seq;
-  mp.split_blocks = split_blocks;
-  mp.slot_floats = p.slot_floats;
-  mp.wpc = split_blocks > 0 ? 4 : 1;
   // passes run in stream order; each kernel waits for the previous one before
   // touching the workspace (programmatic dependents wait for the full grid)
   for (int q0 = 0; q0 < q_len; q0 += kp) {
-    p.q0 = mp.q0 = q0;
-    p.G = mp.G = Gh * std::min(kp, q_len - q0);
+    p.q0 = q0;
+    p.G = Gh * std::min(kp, q_len - q0);
     p.epoch = next_decode_epoch();
     const int nt = p.G > 8 ? 2 : 1;  // tiles of 8 columns
-    mp.warps = di.sms * decode_warps(kv_dtype, head_dim, nt);
-    cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
-    if (e != cudaSuccess) return PQKV_ERR_CUDA;
-    e = launch_merge(head_dim, q_dtype == PQKV_DTYPE_BF16, mp, st);
+    const cudaError_t e = launch_decode(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, nt, tmap, p, di.sms, st);
     if (e != cudaSuccess) return PQKV_ERR_CUDA;
   }
   return PQKV_OK;
@@ -488,7 +472,7 @@ int pqkv_paged_prefill_attention(const void* q, int q_dtype, int batch, int max_
   p.maxblk = max_blocks_per_seq;
   p.tiles_per_seq = (int)tiles;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.timeout_ns = kWaitLimitNs;
+  p.timeout_ns = g_decode_wait_ns.load();
   p.drain_ns = kWaitLimitNs;
   const cudaError_t e = launch_prefill(kv_dtype, head_dim, q_dtype == PQKV_DTYPE_BF16, tmap, p,
                                        reinterpret_cast<cudaStream_t>(stream));

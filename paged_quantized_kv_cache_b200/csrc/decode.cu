@@ -59,8 +59,7 @@ __device__ __forceinline__ void store_out(void* out, size_t i, float v) {
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
-// Four E4M3 codes -> f16x2 of bytes (0,1) and (2,3) by the hardware conversion
-// (true values; the FP4 group scales).
+// Four E4M3 codes -> f16x2 of bytes (0,1) and (2,3) by the hardware conversion.
 __device__ __forceinline__ void dec4_e4m3_cvt(uint32_t r, uint32_t& lo, uint32_t& hi) {
   asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
       "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
@@ -68,35 +67,19 @@ __device__ __forceinline__ void dec4_e4m3_cvt(uint32_t r, uint32_t& lo, uint32_t
       : "r"(r));
 }
 
-// E4M3 codes of the cache are decoded by placing their bits (true) or by the
-// hardware conversion (false); see dec4.
-constexpr bool kE4m3Place = true;
-// The placed f16 of an E4M3 code is its value times 2^-8 (bias 15 against 7).
-template <int KVF>
-constexpr float fp8_unit() { return (KVF == PQKV_DTYPE_FP8_E4M3 && kE4m3Place) ? 256.f : 1.f; }
-
 // Four FP8 codes of a word -> f16x2 of bytes (0,1) and of bytes (2,3), exact.
 // E5M2 codes are the high byte of the binary16 of the same value, so they are
-// placed, not converted. An E4M3 code s.eeee.mmm placed as the binary16
-// s.0eeee.mmm0000000 is its value times 2^-8 exactly (normals and subnormals:
-// the exponent biases are 15 and 7); the factor 2^8 (fp8_unit) is folded into
-// the logit scale of K and the output scale of V. In one word: a byte permute
-// puts code c0 in bits 15..8, its sign replicated in bits 23..16 and code c1 in
-// bits 31..24; an arithmetic shift by one then leaves each half as
-// s.s.eeee.mmm0000000 and a mask clears the second sign bit.
+// placed, not converted; E4M3 codes go through the hardware conversion (placing
+// their bits too, as the binary16 of value x 2^-8 with three integer
+// operations per pair, measured 20% slower per decode: the kernel is bound by
+// instruction issue, not by the conversions).
 template <int KVF>
 __device__ __forceinline__ void dec4(uint32_t r, uint32_t& lo, uint32_t& hi) {
   if constexpr (KVF == PQKV_DTYPE_FP8_E5M2) {
     lo = prmt(r, 0u, 0x1404u);
     hi = prmt(r, 0u, 0x3424u);
-  } else if constexpr (kE4m3Place) {
-    lo = (uint32_t)((int32_t)prmt(r, 0u, 0x1804u) >> 1) & 0xBF80BF80u;
-    hi = (uint32_t)((int32_t)prmt(r, 0u, 0x3A24u) >> 1) & 0xBF80BF80u;
   } else {
-    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
-        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
-        : "=r"(lo), "=r"(hi)
-        : "r"(r));
+    dec4_e4m3_cvt(r, lo, hi);
   }
 }
 
@@ -529,113 +512,69 @@ __device__ __forceinline__ void merge_pair(const DecodeParams& p, int b, int h, 
   }
 }
 
-// A warp has written its piece of a split pair (all lanes' stores done):
-// count it in the pair's arrival word and tell whether it was the last one.
-// The word (counters[k0], k0 = the chunk where the pair starts) holds the
-// launch's tag in its high 40 bits and the pieces seen in its low 24, so a
-// word left by an earlier launch (or an aborted one) reads as zero pieces and
-// the workspace needs no clearing between launches. Pieces of one pair come
-// from different chunks and never wait on one another; the bounded loop only
-// retries when another piece's update got in between.
+// Arrival words. counters[k0] (k0 = the chunk where a split pair starts) holds
+// the launch's tag in its high 40 bits and the pieces of the pair counted so
+// far in its low 24. A word whose tag is not this launch's (left by an earlier
+// or aborted launch, or whatever the workspace held) reads as zero pieces, so
+// the workspace needs no clearing. Adds n pieces (lane 0 only; the warp's
+// partials are made visible first) and returns the count after the add. Pieces
+// of one pair never wait on one another; the bounded loop only retries when
+// another update got in between.
+__device__ __forceinline__ unsigned long long count_pieces(const DecodeParams& p, int k0, int n) {
+  __threadfence();  // this warp's partials are visible before the arrivals count
+  unsigned long long* w = p.counters + k0;
+  const unsigned long long tag = (unsigned long long)p.epoch << 24;
+  unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(w);
+  for (int it = 0; it < 4096; ++it) {
+    const unsigned long long have = ((cur >> 24) == p.epoch) ? (cur & 0xFFFFFFull) : 0ull;
+    const unsigned long long prev = atomicCAS(w, cur, tag | (have + (unsigned long long)n));
+    if (prev == cur) return have + (unsigned long long)n;
+    cur = prev;
+  }
+  raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+  return 0;
+}
+
+// A warp has written its piece of a short pair (all lanes' stores done): count
+// it and tell whether it was the last one (its warp then merges the pair).
 __device__ __forceinline__ bool arrive_split(const DecodeParams& p, int k0, int np, int lane) {
   int last = 0;
   if (lane == 0) {
-    __threadfence();  // this warp's partials are visible before the arrival counts
-    unsigned long long* w = p.counters + k0;
-    const unsigned long long tag = (unsigned long long)p.epoch << 24;
-    unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(w);
-    int it = 0;
-    for (; it < 4096; ++it) {
-      const unsigned long long have = ((cur >> 24) == p.epoch) ? (cur & 0xFFFFFFull) : 0ull;
-      const unsigned long long prev = atomicCAS(w, cur, tag | (have + 1));
-      if (prev == cur) {
-        last = (have + 1 == (unsigned long long)np);
-        break;
-      }
-      cur = prev;
-    }
-    if (it == 4096) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+    last = count_pieces(p, k0, 1) == (unsigned long long)np;
     if (last) __threadfence();  // order the reads of the other pieces after the count
   }
   return __shfl_sync(kFull, last, 0) != 0;
 }
 
+// Count n pieces of a long pair that this warp has written (all lanes' stores
+// done). The pair is merged by the warps that own its output columns, which
+// poll the word (wait_pieces).
+__device__ __forceinline__ void publish_pieces(const DecodeParams& p, int k0, int n, int lane) {
+  if (lane == 0 && n > 0) count_pieces(p, k0, n);
+}
+
 // ---------------------------------------------------------------------------
-// Log-sum-exp merge of the split pairs of more than kMergeInKernel pieces (same
-// formula as merge_pair). CTAs of 4 warps; each output column (sequence b, KV
-// head h, column n) gets p.wpc warps: 1 with the balanced split (pairs have
-// few pieces; 4 columns per CTA keep the grid small) or 4 with a fixed split
-// (tens of pieces per pair). Launched as a programmatic dependent of the decode
-// kernel: it rebuilds the decode's split plan from seq_lens while that grid is
-// still running, and its warps whose pair needs nothing from it exit before
-// waiting for the decode, so with no long split pair the whole grid is done
-// before the decode is. Warp q of a column takes a contiguous share of the
-// pair's pieces and issues the loads of all of them (up to kBatch at a time)
-// together with the (m, l) of every piece, so that a merge costs about one
-// round trip to L2; the shares' weighted sums are added in order, so results
-// do not depend on timing.
+// Log-sum-exp merge of one output column (query row n of the pair (b, h)) over
+// the np > kMergeInKernel pieces of a long split pair (same formula as
+// merge_pair), by one warp: the (m, l) of every piece with lanes over pieces,
+// then the outputs with lanes over head dims, pieces in order, the loads of up
+// to kBatch pieces issued before they are folded in (the first batch together
+// with the (m, l) loads).
 // ---------------------------------------------------------------------------
-template <int D, bool QBF16>
-__global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p) {
-  extern __shared__ int P[];  // [B + 1]: blocks of the sequences before b, as in the decode
-  __shared__ int wsum[4];
-  __shared__ float part[4][D];  // each warp's weighted sum of its pieces
-  constexpr int DPL = D / 32;   // head dims per lane
-  constexpr int kBatch = 16;    // pieces whose outputs a warp loads at once
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  {
-    const int B = p.B, per = (B + 127) / 128;
-    const int lo = min(B, tid * per), hi = min(B, lo + per);
-    const int lim = kBlock * p.maxblk;
-    int local = 0;
-    for (int i = lo; i < hi; ++i) {
-      const int L = p.seq_lens[i];
-      local += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(kFull, incl, o);
-      if (lane >= o) incl += v;
-    }
-    if (lane == 31) wsum[warp] = incl;
-    __syncthreads();
-    int run = incl - local;
-    for (int w = 0; w < warp; ++w) run += wsum[w];
-    if (tid == 0) P[0] = 0;
-    for (int i = lo; i < hi; ++i) {
-      const int L = p.seq_lens[i];
-      run += (L < 0 || L > lim || (L > 0 && L < p.k)) ? 0 : (L + kBlock - 1) / kBlock;
-      P[i + 1] = run;
-    }
-    __syncthreads();
-  }
-  const int T = p.Hkv * P[p.B];
-  const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + p.warps - 1) / p.warps);
-  const int wpc = p.wpc, sh = warp % wpc;                // this warp's share of its column
-  const long cid = ((long)blockIdx.x * 4 + warp) / wpc;  // column
-  if (cid >= (long)p.B * p.Hkv * p.G) return;           // (the same for the warps of a column)
-  const int b = (int)(cid / ((long)p.Hkv * p.G));
-  const int h = (int)((cid / p.G) % p.Hkv), n = (int)(cid % p.G);
-  const int nblk = P[b + 1] - P[b];
-  if (nblk == 0) return;
-  const int s0 = p.Hkv * P[b] + h * nblk;
-  const int k0 = s0 / Qc, k1 = (s0 + nblk - 1) / Qc;
-  const int np = k1 - k0 + 1;
-  if (np <= kMergeInKernel) return;  // one chunk (no split), or merged inside the decode kernel
+template <int D, bool QBF16, int kBatch>
+__device__ __forceinline__ void merge_column(const DecodeParams& p, int b, int h, int n, int k0, int np, int lane) {
+  constexpr int DPL = D / 32;  // head dims per lane
+  const int G = p.G;
   auto slot_base = [&](int i) {  // piece i (0-based) of the pair
     const int kk = k0 + i;
     return p.partials + (size_t)(i == 0 ? 2 * kk + 1 : 2 * kk) * p.slot_floats;
   };
-  const int q0 = (int)((long)np * sh / wpc), q1 = (int)((long)np * (sh + 1) / wpc);  // this warp's pieces
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  // the first batch of this warp's outputs, in flight with the (m, l) loads below
   float v[kBatch][DPL];
   auto load_batch = [&](int i0) {
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = i0 + u;
-      if (i < q1) {
+      if (i < np) {
         const float* bs = slot_base(i) + n * D + lane * DPL;
         if constexpr (DPL == 4) {
           const float4 t = __ldcg(reinterpret_cast<const float4*>(bs));
@@ -647,8 +586,7 @@ __global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p
       }
     }
   };
-  load_batch(q0);
-  // weights over all pieces: lanes over pieces (every warp computes the same M, L)
+  load_batch(0);
   float mi[4], li[4];  // pieces lane, lane + 32, lane + 64, lane + 96
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
@@ -657,12 +595,12 @@ __global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p
     li[r] = 0.f;
     if (i < np) {
       const float* bs = slot_base(i);
-      mi[r] = __ldcg(bs + p.G * D + n);
-      li[r] = __ldcg(bs + p.G * D + p.G + n);
+      mi[r] = __ldcg(bs + G * D + n);
+      li[r] = __ldcg(bs + G * D + G + n);
     }
   }
   float M = fmaxf(fmaxf(mi[0], mi[1]), fmaxf(mi[2], mi[3]));
-  for (int i = lane + 128; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + p.G * D + n));
+  for (int i = lane + 128; i < np; i += 32) M = fmaxf(M, __ldcg(slot_base(i) + G * D + n));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, o));
   float wr[4];
@@ -674,28 +612,25 @@ __global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p
   }
   for (int i = lane + 128; i < np; i += 32) {
     const float* bs = slot_base(i);
-    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + p.G * D + n) - M) * __ldcg(bs + p.G * D + p.G + n);
+    L += (M == kNegInf) ? 0.f : exp2f(__ldcg(bs + G * D + n) - M) * __ldcg(bs + G * D + G + n);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(kFull, L, o);
-  // this warp's weighted sum, pieces in order
   float acc[DPL];
 #pragma unroll
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-  for (int i0 = q0; i0 < q1; i0 += kBatch) {
-    if (i0 > q0) load_batch(i0);
+  for (int i0 = 0; i0 < np; i0 += kBatch) {
+    if (i0 > 0) load_batch(i0);
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
       const int i = i0 + u;
-      if (i < q1) {  // the same on every lane
+      if (i < np) {  // the same on every lane
         float w;
         if (i < 128) {
-          const float wv = __shfl_sync(kFull, (i >> 5) == 0 ? wr[0] : (i >> 5) == 1 ? wr[1] : (i >> 5) == 2 ? wr[2]
-                                                                                                       : wr[3],
-                                       i & 31);
-          w = wv;
+          const int r = i >> 5;
+          w = __shfl_sync(kFull, r == 0 ? wr[0] : r == 1 ? wr[1] : r == 2 ? wr[2] : wr[3], i & 31);
         } else {
-          w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + p.G * D + n) - M);
+          w = (M == kNegInf) ? 0.f : exp2f(__ldcg(slot_base(i) + G * D + n) - M);
         }
 #pragma unroll
         for (int e = 0; e < DPL; ++e) acc[e] += w * v[u][e];
@@ -704,22 +639,32 @@ __global__ void __launch_bounds__(128, 1) paged_merge_kernel(const MergeParams p
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   const size_t orow = col_row(b, h, n, p.k, p.q0, p.Gh, p.Hq, D) + lane * DPL;
-  if (wpc == 1) {
 #pragma unroll
-    for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
-    return;
-  }
-  // four shares of one column (all warps of the CTA are here): add them in order
-#pragma unroll
-  for (int e = 0; e < DPL; ++e) part[warp][lane * DPL + e] = acc[e];
-  __syncthreads();
-  if (warp == 0) {
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) {
-      const int d = lane * DPL + e;
-      store_out<QBF16>(p.out, orow + e, (((part[0][d] + part[1][d]) + part[2][d]) + part[3][d]) * inv);
+  for (int e = 0; e < DPL; ++e) store_out<QBF16>(p.out, orow + e, acc[e] * inv);
+}
+
+// Wait until the arrival word of the pair whose first unit is k0 shows all its
+// np pieces (lane 0 polls it, sleeping between polls), giving up after the
+// wait limit. The pieces come from other warps of the same persistent grid,
+// all resident, which never wait for this one, so the wait ends unless one of
+// them gave up itself.
+__device__ __forceinline__ bool wait_pieces(const DecodeParams& p, int k0, int np, int lane) {
+  int ok = 0;
+  if (lane == 0) {
+    const volatile unsigned long long* w = p.counters + k0;
+    const unsigned long long want = ((unsigned long long)p.epoch << 24) | (unsigned long long)np;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      if (*w == want) {
+        ok = 1;
+        break;
+      }
+      if (globaltimer_ns() - t0 > p.timeout_ns) break;
+      __nanosleep(128);
     }
+    __threadfence();  // order the reads of the pieces after the count
   }
+  return __shfl_sync(kFull, ok, 0) != 0;
 }
 
 template <int KVF, int D, bool QBF16, int NT>
@@ -814,8 +759,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 
   const int T = Hkv * P[B];
   const int W = gridDim.x * NW;
-  const int Qc = p.split_blocks > 0 ? p.split_blocks : max(1, (T + W - 1) / W);
-  const int K = T > 0 ? (T + Qc - 1) / Qc : 0;
+  const SplitPlan plan = make_split_plan(T, W, p.split_blocks);
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   uint32_t phase = 0;     // parity bit per stage
@@ -836,20 +780,16 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     j = rel - h * n;
   };
 
-  // With a fixed split (split_blocks > 0) the K chunks go to Wa = ceil(K /
-  // rounds) warps, rounds = ceil(K / W), each taking `rounds` consecutive
-  // chunks (the last one fewer): every working warp has the same number of
-  // chunks, and a warp's chunks are mostly pieces of one (sequence, head)
-  // pair, so its query stays loaded from one chunk to the next. The balanced
-  // split has K <= W chunks, one per warp. A warp's blocks, chunk after chunk,
-  // are the flat blocks kbase * Qc + v, v = 0 .. Vtot - 1; the copy ring runs
-  // over v without a break at chunk boundaries.
-  const int k0 = warp * gridDim.x + blockIdx.x;
-  const int rounds = K > 0 ? (K + W - 1) / W : 1;
-  const int kbase = k0 * rounds;
-  const int nck = kbase < K ? min(K, kbase + rounds) - kbase : 0;
-  const int Vtot = nck == 0 ? 0 : min(T, (kbase + nck) * Qc) - kbase * Qc;
-  auto vflat = [&](int v) { return kbase * Qc + v; };  // virtual block index -> flat block index
+  // This warp's share of the flat range (see SplitPlan), cut into units at the
+  // multiples of C inside it. Its blocks are numbered v = 0 .. Vtot - 1 from
+  // f0w; the copy ring runs over v without a break at unit boundaries, and a
+  // warp's units are mostly pieces of one (sequence, head) pair, so its query
+  // stays loaded from one unit to the next.
+  const int wr = warp * gridDim.x + blockIdx.x;
+  const int f0w = (int)min((long long)T, (long long)wr * plan.Qw);
+  const int f1w = min(T, f0w + plan.Qw);
+  const int Vtot = f1w - f0w;
+  auto vflat = [&](int v) { return f0w + v; };  // virtual block index -> flat block index
   // Per-lane window of (physical id, head) for blocks wbase + lane and, loaded
   // ahead, wbase + 32 + lane. Values are only inspected when issued.
   auto load_entry = [&](int v, int& id, int& hh) {
@@ -919,12 +859,12 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
   float csc[NT][2];
   OutlierState<NT> ost;  // FP4 only
   int qb = -1, qh = -1;  // the pair whose query is loaded
+  int owed_k0 = -1, owed_n = 0;  // pieces of a long pair written but not yet published
 
-  for (int ci = 0; ci < nck && !aborted; ++ci) {
-    const int k = kbase + ci;
-    const int f0 = k * Qc;
-    const int f1 = min(T, f0 + Qc);
-    const int vb = ci * Qc - f0;  // v = f + vb inside this chunk
+  const int vb = -f0w;  // v = f + vb
+  for (int f0 = f0w, f1 = f0w; f0 < f1w && !aborted; f0 = f1) {
+    f1 = min(f1w, (f0 / plan.C + 1) * plan.C);  // this unit: [f0, f1)
+    const int k = plan.unit(f0);
 
     locate(f0, b, h, j);
     nblk = P[b + 1] - P[b];
@@ -996,7 +936,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
         const float m = __shfl_sync(kFull, rowmul[nt], (2 * qd + c) << 2);
-        csc[nt][c] = ((Gm::k16 || !QBF16) ? p.scale_log2 : p.scale_log2 / m) * fp8_unit<KVF>();  // exact
+        csc[nt][c] = (Gm::k16 || !QBF16) ? p.scale_log2 : p.scale_log2 / m;  // 1 / m = 2^e: exact
       }
       }
       if constexpr (Gm::kFp4) {
@@ -1025,7 +965,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
           lt[nt][1] += __shfl_xor_sync(kFull, lt[nt][1], o);
         }
       }
-      const float vs = Gm::kFp8 ? vref * fp8_unit<KVF>() : 1.f;
+      const float vs = Gm::kFp8 ? vref : 1.f;
       if constexpr (Gm::kFp4) {  // fold the outlier channels' O in and clear it
         ost.template flush<Gm::kOStride>(woext, lane, D);
 #pragma unroll
@@ -1091,12 +1031,24 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
           }
         }
       }
-      // a pair of at most kMergeInKernel pieces is merged by the warp that
-      // brings its last piece; longer ones by paged_merge_kernel
+      // every piece is counted in its pair's arrival word. A pair of at most
+      // kMergeInKernel pieces is merged at once by the warp that brings its
+      // last piece. A longer one is merged column by column after the warps'
+      // shares, so its pieces are only counted here and published together
+      // when the warp moves on to another pair (one fence for all of them).
       __syncwarp();
       const int s0 = Hkv * P[b] + h * nblk;  // flat index of the pair's first block
-      const int k0 = s0 / Qc, np = (s0 + nblk - 1) / Qc - k0 + 1;
-      if (np <= kMergeInKernel && arrive_split(p, k0, np, lane)) merge_pair<D, QBF16>(p, b, h, k0, np, lane);
+      const int k0 = plan.unit(s0), np = plan.unit(s0 + nblk - 1) - k0 + 1;
+      if (np <= kMergeInKernel) {
+        if (arrive_split(p, k0, np, lane)) merge_pair<D, QBF16>(p, b, h, k0, np, lane);
+      } else {
+        if (k0 != owed_k0) {
+          publish_pieces(p, owed_k0, owed_n, lane);
+          owed_n = 0;
+        }
+        owed_k0 = k0;
+        ++owed_n;
+      }
     };
 
     // A stage whose wait gives up keeps its phase and its in-flight bit, so
@@ -1296,6 +1248,30 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
     }
   }
 
+  publish_pieces(p, owed_k0, owed_n, lane);
+
+  // ---- long split pairs (more than kMergeInKernel pieces): output column c
+  // of all (sequence, head, query row) columns is merged by warp c mod W, once
+  // its pair's pieces are all written ----
+  if (!aborted) {
+    const long ncols = (long)B * Hkv * G;
+    for (long c = wr; c < ncols; c += W) {
+      const int cb = (int)(c / ((long)Hkv * G));
+      const int ch = (int)((c / G) % Hkv), cn = (int)(c % G);
+      const int cnb = P[cb + 1] - P[cb];
+      if (cnb == 0) continue;
+      const int s0 = Hkv * P[cb] + ch * cnb;
+      const int k0 = plan.unit(s0), np = plan.unit(s0 + cnb - 1) - k0 + 1;
+      if (np <= kMergeInKernel) continue;
+      if (!wait_pieces(p, k0, np, lane)) {
+        if (lane == 0) raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+        continue;
+      }
+      // pieces loaded at once: as many as the registers the main loop leaves allow
+      merge_column<D, QBF16, Gm::k16 ? 32 : 16>(p, cb, ch, cn, k0, np, lane);
+    }
+  }
+
   // after a timeout: let copies still in flight land before the warp exits
   // (with the full limit, whatever the limit that gave up)
   if (aborted) {
@@ -1341,49 +1317,7 @@ static cudaError_t launch_decode_t(const CUtensorMap& tmap, const DecodeParams& 
   return cudaGetLastError();
 }
 
-// The merge kernel is launched right behind the decode kernel on the same
-// stream as a programmatic dependent (its launch overlaps the decode's tail;
-// griddepcontrol.wait inside it orders it after the decode grid).
-cudaError_t launch_merge(int D, bool q_bf16, const MergeParams& p, cudaStream_t st) {
-  const long warps = (long)p.B * p.Hkv * p.G * p.wpc;  // wpc per (sequence, KV head, column)
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
-  cfg.blockDim = dim3(128);
-  cfg.dynamicSmemBytes = (size_t)(p.B + 1) * 4;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (D == 128)
-    return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, true>, p)
-                  : cudaLaunchKernelEx(&cfg, paged_merge_kernel<128, false>, p);
-  return q_bf16 ? cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, true>, p)
-                : cudaLaunchKernelEx(&cfg, paged_merge_kernel<64, false>, p);
-}
-
 // nt = tiles of 8 MMA columns per warp (1, or 2 for up to 16 query rows per KV head)
-template <int NT>
-static int decode_warps_t(int kv_dtype, int D) {
-  switch (kv_dtype) {
-    case PQKV_DTYPE_FP16:
-    case PQKV_DTYPE_BF16:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_BF16, 128, NT>::kWarps : DecodeGeom<PQKV_DTYPE_BF16, 64, NT>::kWarps;
-    case PQKV_DTYPE_FP8_E4M3:
-    case PQKV_DTYPE_FP8_E5M2:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP8_E4M3, 128, NT>::kWarps
-                      : DecodeGeom<PQKV_DTYPE_FP8_E4M3, 64, NT>::kWarps;
-    default:
-      return D == 128 ? DecodeGeom<PQKV_DTYPE_FP4_E2M1, 128, NT>::kWarps
-                      : DecodeGeom<PQKV_DTYPE_FP4_E2M1, 64, NT>::kWarps;
-  }
-}
-
-int decode_warps(int kv_dtype, int D, int nt) {
-  return nt == 2 ? decode_warps_t<2>(kv_dtype, D) : decode_warps_t<1>(kv_dtype, D);
-}
-
 template <int NT>
 static size_t decode_smem_bytes_t(int kv_dtype, int D, int B) {
   switch (kv_dtype) {

@@ -12,14 +12,16 @@
 // Work decomposition. The blocks of all (sequence b, KV head h) pairs are laid
 // end to end (b-major, then h, then block j) into one flat range of T blocks.
 // The grid is persistent (one CTA per SM, NW warps each); the flat range is cut
-// into chunks of Q blocks and warp w takes chunks w, w + W, ... (W = all warps).
-// A chunk covers whole pairs (written straight to `out`) and at most two
+// into W equal shares, one per warp (W = all warps), and a fixed split also cuts
+// it at every multiple of split_blocks (SplitPlan); the cells are the units.
+// A unit covers whole pairs (written straight to `out`) and at most two
 // partial pairs at its ends (written to a workspace slot). The pieces of a
-// split pair are merged in chunk order, so results do not depend on timing:
+// split pair are merged in unit order, so results do not depend on timing:
 // a pair of at most kMergeInKernel pieces (the usual case: many sequences)
 // by the warp that writes its last piece (counted in a per-pair arrival
-// word); a longer one (few long sequences spread over the GPU) by a second
-// kernel, launched as a programmatic dependent, with one warp per column.
+// word); a longer one (few long sequences spread over the GPU) column by
+// column, each column by one warp of the same grid once its own share is
+// done, when the arrival word shows all pieces.
 //
 // Per warp: a private ring of NS shared-memory stages, each holding the K and V
 // tiles of one (block, head) pair fetched by one TMA tensor copy (128/64/32-byte
@@ -63,17 +65,36 @@ struct DecodeParams {
   unsigned long long epoch;     // tag of this launch (40 bits, never 0)
 };
 
-struct MergeParams {
-  const int32_t* seq_lens;
-  const float* partials;
-  void* out;
-  int B, Hq, Hkv, G, maxblk;
-  int k, Gh, q0;     // as in DecodeParams
-  int warps;         // warps of the decode grid (its balanced chunk length depends on it)
-  int split_blocks;
-  int slot_floats;
-  int wpc;           // warps per output column: 1 (4 columns per CTA) or 4 (one column per CTA)
+// The split of the flat block range (T blocks of all (sequence, head) pairs,
+// laid end to end) over the W warps of the decode grid: warp w takes blocks
+// [w Qw, (w + 1) Qw), Qw = ceil(T / W), so every warp has the same share. With
+// a fixed split (split_blocks = C > 0) a piece of a pair also ends at every
+// multiple of C, so that each partial result lies inside one C-block chunk of
+// the split; the balanced split has C = Qw. The cells between consecutive
+// boundaries (multiples of Qw or of C) are the units; a pair's pieces are the
+// units its blocks cross, in order, and a piece's workspace slot is indexed by
+// its unit (there are at most ceil(T / C) + W of them).
+struct SplitPlan {
+  int Qw, C;
+  long long lcm;  // of Qw and C: boundaries that are both count once
+  __device__ __forceinline__ int unit(int f) const {  // the unit holding flat block f
+    return f / C + f / Qw - (int)((long long)f / lcm);
+  }
 };
+
+__device__ __forceinline__ SplitPlan make_split_plan(int T, int W, int split_blocks) {
+  SplitPlan s;
+  s.Qw = max(1, (T + W - 1) / W);
+  s.C = split_blocks > 0 ? split_blocks : s.Qw;
+  int a = s.Qw, b = s.C;
+  while (b != 0) {
+    const int t = a % b;
+    a = b;
+    b = t;
+  }
+  s.lcm = (long long)(s.Qw / a) * s.C;
+  return s;
+}
 
 // Compile-time geometry of one format; NT = tiles of 8 MMA columns (query rows)
 // per KV head: 1, or 2 for multi-query decode with up to 16 rows.
