@@ -122,13 +122,15 @@ int pqkv_version(void);
 /* Human-readable name of a PQKV_* return code. Never NULL. */
 const char* pqkv_status_string(int status);
 
-/* Limit, in nanoseconds, of each wait of the decode kernels
- * (pqkv_paged_decode_attention and its variants) on one of their asynchronous
- * copies, for the launches enqueued after this call (process-wide; 0 restores
- * the default of 2 s). A wait that runs out sets PQKV_DEVERR_TIMEOUT and ends
- * that warp's work, after its copies still in flight have landed (that wait
- * keeps the 2 s limit). Meant for tests of the timeout path: a very short
- * limit makes waits give up while their copies are still on the way. */
+/* Limit, in nanoseconds, of each wait of the attention kernels
+ * (pqkv_paged_decode_attention and its variants, pqkv_paged_prefill_attention)
+ * on an asynchronous copy, on a tensor-core product or on another warp of the
+ * same CTA, for the launches enqueued after this call (process-wide; 0
+ * restores the default of 2 s). A wait that runs out sets PQKV_DEVERR_TIMEOUT
+ * and ends that warp's work, after its copies and products still in flight
+ * have completed (that wait keeps the 2 s limit; PQKV_DEVERR_DRAIN if it runs
+ * out too). Meant for tests of the timeout path: a very short limit makes
+ * waits give up while the work they wait for is still on the way. */
 void pqkv_set_decode_wait_limit_ns(uint64_t ns);
 
 /*

@@ -147,8 +147,8 @@ def _dt_of(t: torch.Tensor, name: str) -> int:
 
 
 def set_decode_wait_limit_ns(ns: int) -> None:
-    """pqkv_set_decode_wait_limit_ns: limit of the decode kernels' waits on their
-    copies for later launches (0 = the default 2 s); for tests of the timeout path."""
+    """pqkv_set_decode_wait_limit_ns: limit of the decode and prefill kernels'
+    waits for later launches (0 = the default 2 s); for tests of the timeout path."""
     _lib.pqkv_set_decode_wait_limit_ns(int(ns))
 
 

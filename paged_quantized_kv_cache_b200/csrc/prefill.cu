@@ -9,26 +9,33 @@
 // q_len cached positions (the chunk is written to the cache first); query token
 // i at position p attends to positions 0..p.
 //
-// Work decomposition. One CTA per (sequence, KV head, tile of 128 rows); a row
-// is (query token, query head of the GQA group), so a tile holds 128 / G query
-// tokens. Four compute warps own one row each per thread (its S and O rows live
-// in tensor-memory lane r); a fifth warp only fetches: it refills each stage of
-// a 4-deep ring as soon as the stage is released (by a tcgen05 commit after
-// the last product reading it, or once its raw codes are dequantized). The
-// compute warps walk the KV positions the tile needs in tiles of 64 tokens (4
-// cache blocks):
-//   S(t) = Q K(t)^T            tcgen05.mma M=128 N=64, two S buffers in TMEM
-//   online softmax of S(t)     one row per thread, no shuffles, lazy rescale
-//   O += P(t) V(t)             tcgen05.mma M=128 N=D, P from shared memory
-//                              (P = P_hi + P_lo in two products for bf16)
-// S(t+1) is issued before the softmax of tile t, so the tensor cores compute
-// while the threads exponentiate. Operands are 128-byte-swizzled shared-memory
-// tiles: 16-bit K/V land there directly by TMA; FP8 / FP4 tiles are fetched raw
-// (one bulk copy per block plus its scales and outlier buffers) and the threads
-// dequantize them into f16 operands. FP8 scales stay out of the operands: the
-// K scale multiplies S, the V scale multiplies P relative to the largest V
-// scale seen so far (O is kept in units of it). FP4 operands are exact in f16
-// (E2M1 x E4M3 and the fp16 outlier values).
+// Work decomposition. One CTA per (sequence, KV head, pair of 128-row tiles); a
+// row is (query token, query head of the GQA group), so a tile holds 128 / G
+// query tokens. Warps have one role each:
+//   two compute warpgroups, one row per thread (its S, P and O rows live in
+//     tensor-memory lane r of the warpgroup's 256 columns): online softmax,
+//     and for quantized caches the dequantization of each tile (both together);
+//   a producer warp: refills each stage of a 4-deep ring as soon as it is
+//     released (by the MMA warp's commit after the last product reading it, or
+//     once its raw codes are dequantized);
+//   an MMA warp: issues every tensor-core product and commits each to an
+//     mbarrier, so no compute warp waits on a barrier with the others.
+// Per KV tile t of 64 tokens (4 cache blocks) and warpgroup:
+//   S(t) = Q K(t)^T        tcgen05.mma M=128 N=64 (A, B in shared memory),
+//                          into one of two S buffers in tensor memory
+//   softmax of S(t)        one row per thread, no shuffles, lazy rescale of O
+//   P(t) -> tensor memory  over the S(t) columns (16-bit, two per column;
+//                          P = P_hi + P_lo for bf16), then one arrival per warp
+//   O += P(t) V(t)         tcgen05.mma M=128 N=D, A = P from tensor memory
+// The MMA warp issues S(t + 2) into a buffer as soon as PV(t) has read the P
+// it held, so the scores of a warpgroup's next tile are always computed while
+// it exponentiates the current one. Operands in shared memory are
+// 128-byte-swizzled tiles: 16-bit K/V land there directly by TMA; FP8 / FP4
+// tiles are fetched raw (one bulk copy per block plus its scales and outlier
+// buffers) and dequantized into f16 operands. FP8 scales stay out of the
+// operands: the K scale multiplies S, the V scale multiplies P relative to
+// the largest V scale seen so far (O is kept in units of it). FP4 operands are
+// exact in f16 (E2M1 x E4M3 and the fp16 outlier values).
 #include <atomic>
 #include <cfloat>
 
@@ -54,16 +61,16 @@ struct PrefillGeom {
   // the K/V stages (one issues while the other stalls; a K/V tile serves 256
   // rows). Quantized tiles are dequantized by both together.
   static constexpr int NWG = 2;
-  static constexpr int kStages = (kFp8 && D == 128) ? 2 : 3;  // KV tiles in flight (shared memory)
-  static constexpr int kThreads = NWG * kWG + 32; // + one producer warp
+  static constexpr int kStages = 4;                // KV tiles in flight (shared memory)
+  static constexpr int kThreads = NWG * kWG + 64; // + one producer warp + one MMA warp
   static constexpr int NB = D / 64;                // 128-byte boxes per operand row
   static constexpr int kQBytes = NB * kM * 128;    // Q operand of one warpgroup [box][128 rows][128 B]
   static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
-  static constexpr int kPBytes = kM * 128;         // P operand: 64 tokens (2 B) per row
   // bf16 operands: P = P_hi + P_lo, both rounded to bf16, keeps ~16 significant
   // bits of the probabilities (a bf16 P alone errs by up to |v| 2^-9, too much
   // for the 2e-3 tolerance); f16 operands (fp16, FP8, FP4 caches) take a single
-  // f16 P (|v| 2^-11 at most)
+  // f16 P (|v| 2^-11 at most). P lives in tensor memory, over the columns of
+  // the S tile it came from (32 columns per part).
   static constexpr bool kSplitP = (KVF == PQKV_DTYPE_BF16);
   static constexpr int kRawTile = 32 * row_bytes(KVF, D);  // one block's K|V codes
   static constexpr int kScaleBytes = kFp8 ? 16 : (kFp4 ? 2 * 16 * (D / 16) : 0);
@@ -74,15 +81,14 @@ struct PrefillGeom {
   static constexpr int kStageBytes = (kRawStage + 1023) / 1024 * 1024;
   static constexpr int kKops = k16 ? 0 : 2;        // dequantized K tiles (S of tile t-1 may still read one)
   static constexpr int kVops = k16 ? 0 : 3;        // dequantized V tiles (PV of tile t-2 may still read one)
-  static constexpr int kPSet = (kSplitP ? 2 : 1) * kPBytes;  // P operands of one warpgroup
   static constexpr int oQ = 0;
   static constexpr int oStage = oQ + NWG * kQBytes;
   static constexpr int oKop = oStage + kStages * kStageBytes;
   static constexpr int oVop = oKop + kKops * kOpBytes;
-  static constexpr int oP = oVop + kVops * kOpBytes;
-  static constexpr int oMisc = oP + NWG * kPSet;
-  static constexpr int kMiscBytes = 256;
+  static constexpr int oMisc = oVop + kVops * kOpBytes;
+  static constexpr int kMiscBytes = 512;
   static constexpr int kSmem = oMisc + kMiscBytes + 1024;  // + alignment slack
+  static_assert(kSmem <= 227 * 1024, "shared memory of one CTA");
   // per warpgroup 256 columns: O at [0, D), S buffers at D and D + 64
   static constexpr uint32_t kTmemCols = 256 * NWG;
 };
@@ -98,9 +104,6 @@ __device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Barrier of the 128 threads of one compute warpgroup (named barrier 1 + wg;
-// the other warpgroup and the producer warp run on their own).
-__device__ __forceinline__ void wg_sync(int wg) { asm volatile("bar.sync %0, 128;" ::"r"(1 + wg) : "memory"); }
 // Barrier of all compute threads (named barrier 3), and its and-reduction.
 template <int NWG>
 __device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 3, %0;" ::"n"(NWG * 128) : "memory"); }
@@ -115,18 +118,6 @@ __device__ __forceinline__ bool cta_all(bool v) {
       : "memory");
   return r != 0;
 }
-// The warpgroup barrier, returning whether v held on every thread of the warpgroup.
-__device__ __forceinline__ bool wg_all(int wg, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, %2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(1 + wg)
-      : "memory");
-  return r != 0;
-}
-
 // Packed pairs of fp32 operations (two lanes of IEEE fp32 arithmetic, rounded to
 // nearest, in one instruction): (d0, d1) = (a0, a1) op (b0, b1) [+ (c0, c1)].
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
@@ -184,10 +175,13 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   uint8_t* sVop = smem + Gm::oVop;
   uint64_t* bar_full = reinterpret_cast<uint64_t*>(smem + Gm::oMisc);  // [kStages] tile landed
   uint64_t* bar_empty = bar_full + kStages;                             // [kStages] stage free again
-  uint64_t* bar_s_all = bar_empty + kStages;                            // [NWG][2] S(t) computed
-  uint64_t* bar_pv_all = bar_s_all + 2 * NWG;                           // [NWG] PV(t) computed
-  float* tile_sk = reinterpret_cast<float*>(bar_pv_all + NWG);          // [2][4] FP8 K scales
-  float* tile_sv = tile_sk + 8;                                         // [2][4] FP8 V scales
+  uint64_t* bar_s = bar_empty + kStages;     // [NWG][2] S(t) computed (buffer t % 2)
+  uint64_t* bar_p = bar_s + 2 * NWG;         // [NWG][2] P(t) in tensor memory (one arrival per warp)
+  uint64_t* bar_pv = bar_p + 2 * NWG;        // [NWG][2] PV(t) computed
+  uint64_t* bar_op = bar_pv + 2 * NWG;       // [2] quantized: operands of tile t dequantized
+  uint64_t* bar_drain = bar_op + 2;          // every product issued has completed
+  float* tile_sk = reinterpret_cast<float*>(bar_drain + 1);  // [2][4] FP8 K scales
+  float* tile_sv = tile_sk + 8;                              // [2][4] FP8 V scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* n_issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
@@ -205,6 +199,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
   if (qn <= 0 || mt0 * TOK >= qn) return;
   const bool is_compute = tid < NWG * kWG;
+  const bool is_producer = warp == NWG * 4, is_mma = warp == NWG * 4 + 1;
   const int wg = is_compute ? tid / kWG : 0;
   const int r = tid % kWG;                           // row of this thread in its warpgroup's tile
   const int i0 = (mt0 + wg) * TOK;                   // first query token of the warpgroup's tile
@@ -231,10 +226,16 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], Gm::k16 ? NWG : 1);  // 16-bit: each warpgroup's commit; else one arrival
+      mbar_init(&bar_empty[s], 1);  // 16-bit: the MMA warp's commit; else one arrival once dequantized
     }
-    for (int i = 0; i < 2 * NWG; ++i) mbar_init(&bar_s_all[i], 1);
-    for (int i = 0; i < NWG; ++i) mbar_init(&bar_pv_all[i], 1);
+    for (int i = 0; i < 2 * NWG; ++i) {
+      mbar_init(&bar_s[i], 1);
+      mbar_init(&bar_p[i], 4);
+      mbar_init(&bar_pv[i], 1);
+    }
+    mbar_init(&bar_op[0], 1);
+    mbar_init(&bar_op[1], 1);
+    mbar_init(bar_drain, 1);
     *abort_flag = 0;
     *n_issued_slot = 0;
     fence_mbar_init();
@@ -287,9 +288,9 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  int n_prepared = 0;  // KV tiles consumed by this thread's warpgroup
+  int n_prepared = 0;  // KV tiles waited for by this thread (compute threads)
 
-  if (!is_compute) {
+  if (is_producer) {
     // ================= producer warp: KV tiles into the stage ring =================
     if (lane == 0) {
       int t = 0;
@@ -346,27 +347,90 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       }
       *n_issued_slot = t;
     }
-  } else {
+  } else if (is_mma) {
+    // ================= MMA warp: every tensor-core product of both warpgroups =================
+    // Order per KV tile t: PV(t) of each warpgroup once its P(t) is in tensor
+    // memory, then S(t + 2) of each warpgroup into the buffer P(t) occupied,
+    // once PV(t) has read it. S(0) and S(1) are issued up front, so a
+    // warpgroup always finds the scores of its next tile computed.
+    if (lane == 0) {
+      bool good = true;
+      // operands of tile t ready: 16-bit K/V landed; quantized tiles dequantized
+      auto ready = [&](int t) -> bool {
+        if constexpr (Gm::k16)
+          return mbar_wait_bounded(&bar_full[t % kStages], (uint32_t)(t / kStages) & 1u, p.timeout_ns);
+        else
+          return mbar_wait_bounded(&bar_op[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
+      };
+      auto issue_s = [&](int t, int w) {
+        tc::fence_after_sync();
+        const uint32_t d = tmem + 256u * w + D + 64 * (t & 1);
+        const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
+        const uint32_t qa = smem_u32(smem + Gm::oQ + w * Gm::kQBytes), ka = smem_u32(kop);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = tc::sw128_desc(ka + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
+          tc::mma_ss(d, a, bd, kIdescS, kk > 0);
+        }
+        tc::commit(&bar_s[2 * w + (t & 1)]);
+      };
+      auto issue_pv = [&](int t, int w) {
+        tc::fence_after_sync();
+        const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
+                                     : sVop + (t % 3) * Gm::kOpBytes;
+        const uint32_t o = tmem + 256u * w, pa = o + D + 64 * (t & 1), va = smem_u32(vop);
+#pragma unroll
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
+          tc::mma_ts(o, pa + kk * 8, bd, kIdescPV, !(t == 0 && kk == 0));
+          if constexpr (Gm::kSplitP) tc::mma_ts(o, pa + 32 + kk * 8, bd, kIdescPV, true);
+        }
+        tc::commit(&bar_pv[2 * w + (t & 1)]);
+      };
+      for (int t = 0; t < min(2, T) && good; ++t) {
+        good = ready(t);
+        if (good)
+          for (int w = 0; w < NWG; ++w) issue_s(t, w);
+      }
+      for (int t = 0; t < T && good; ++t) {
+        for (int w = 0; w < NWG && good; ++w) {
+          good = mbar_wait_bounded(&bar_p[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
+          if (good) issue_pv(t, w);
+        }
+        if (!good) break;
+        // a 16-bit stage holds the operands themselves: free once S(t) and PV(t) are done
+        if constexpr (Gm::k16) tc::commit(&bar_empty[t % kStages]);
+        if (t + 2 < T) {
+          good = ready(t + 2);
+          for (int w = 0; w < NWG && good; ++w) {
+            good = mbar_wait_bounded(&bar_pv[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
+            if (good) issue_s(t + 2, w);
+          }
+        }
+      }
+      if (!good) {
+        *abort_flag = 1;
+        raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+      }
+      // every product issued completes before tensor memory is released
+      tc::commit(bar_drain);
+      if (!mbar_wait_bounded(bar_drain, 0, p.drain_ns)) raise_flag(p.err, PQKV_DEVERR_DRAIN);
+    }
+  } else if (is_compute) {
     // ================= compute warpgroup wg: one row per thread =================
     const uint32_t t_row = tmem + 256u * wg + ((uint32_t)(32 * (warp & 3)) << 16);
-    const uint32_t t_base = tmem + 256u * wg;
-    uint64_t* bar_s = bar_s_all + 2 * wg;
-    uint64_t* bar_pv = bar_pv_all + wg;
-    uint8_t* sQ = smem + Gm::oQ + wg * Gm::kQBytes;
-    uint8_t* sP = smem + Gm::oP + wg * Gm::kPSet;
-    uint32_t ph_full = 0, ph_s = 0, ph_pv = 0;  // parity bits per barrier
-    bool ok = true;                             // no wait of this thread has timed out
+    uint64_t* my_s = bar_s + 2 * wg;
+    uint64_t* my_p = bar_p + 2 * wg;
+    uint64_t* my_pv = bar_pv + 2 * wg;
+    bool ok = true;  // no wait of this thread has timed out
     bool aborted = false;
-    // operations issued and waited for (the same on every thread of the
-    // warpgroup), so that a timeout can let the ones in flight finish
-    int n_s = 0, n_s_waited = 0, n_pv_waited = 0;
     int mask_cur = 0, mask_next = 0;  // blocks of tile t / t + 1 holding data
 
     // ---- make KV tile t's operands ready; returns its block mask ----
     auto prepare = [&](int t) -> int {
       const int s = t % kStages;
-      ok = mbar_wait_bounded(&bar_full[s], (ph_full >> s) & 1u, p.timeout_ns) && ok;
-      ph_full ^= 1u << s;
+      ok = mbar_wait_bounded(&bar_full[s], (uint32_t)(t / kStages) & 1u, p.timeout_ns) && ok;
       ++n_prepared;
       // blocks of the tile that were fetched (as the producer decided), from the
       // block table itself so that every thread agrees even after a timeout
@@ -384,7 +448,8 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       if constexpr (Gm::k16) {
         // V rows without valid data (past the sequence, or a block not loaded)
         // are zeroed: P is 0 there, and 0 x NaN would poison O. Each warpgroup
-        // zeroes before its own products (the same zeros).
+        // zeroes before its own P(t) is handed over (the same zeros), so the
+        // product PV(t) of each warpgroup follows its own zeroing.
         if (mask != 0xF || base + kN > L) {
           for (int u = r; u < kN * Gm::NB * 8; u += kWG) {
             const int rr = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
@@ -393,11 +458,11 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
                 make_uint4(0, 0, 0, 0);
           }
           tc::fence_smem_to_async();
-          wg_sync(wg);
         }
       } else {
-        // both warpgroups are past the previous tile (its products read the
-        // operand buffers written below), then dequantize half of the tile each
+        // both warpgroups are past the products that read the operand buffers
+        // written below (S(t - 2) and PV(t - 3), waited for by each before
+        // this barrier), then dequantize half of the tile each
         cta_sync<NWG>();
         const int gt = wg * kWG + r;
         uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
@@ -477,81 +542,53 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           }
         }
         tc::fence_smem_to_async();
-        tc::fence_before_sync();
         // the products may read the operands once every thread wrote its part;
         // the consensus over both warpgroups also carries timeouts (quantized
         // caches abort only here, so that neither warpgroup is left waiting)
         ok = cta_all<NWG>(ok);
-        // a raw stage is free as soon as it is dequantized
-        if (gt == 0) mbar_arrive(&bar_empty[s]);
+        if (gt == 0 && ok) {
+          mbar_arrive(&bar_empty[s]);  // a raw stage is free as soon as it is dequantized
+          mbar_arrive(&bar_op[t & 1]);
+        }
       }
       return mask;
     };
 
-    // ---- MMA issue (thread 0 of the warpgroup) ----
-    auto issue_s = [&](int t) {
-      tc::fence_after_sync();
-      const uint32_t d = t_base + D + 64 * (t & 1);
-      const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
-      const uint32_t qa = smem_u32(sQ), ka = smem_u32(kop);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t a = tc::sw128_desc(qa + (kk >> 2) * (kM * 128) + (kk & 3) * 32, 16, 1024);
-        const uint64_t bd = tc::sw128_desc(ka + (kk >> 2) * (kN * 128) + (kk & 3) * 32, 16, 1024);
-        tc::mma_ss(d, a, bd, kIdescS, kk > 0);
-      }
-      tc::commit(&bar_s[t & 1]);
-    };
-    auto issue_pv = [&](int t, bool first) {
-      tc::fence_after_sync();
-      const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
-                                   : sVop + (t % 3) * Gm::kOpBytes;
-      const uint32_t pa = smem_u32(sP), va = smem_u32(vop);
-#pragma unroll
-      for (int kk = 0; kk < kN / 16; ++kk) {
-        const uint64_t bd = tc::sw128_desc(va + kk * 2048, kN * 128, 1024);
-        tc::mma_ss(t_base, tc::sw128_desc(pa + kk * 32, 16, 1024), bd, kIdescPV, !(first && kk == 0));
-        if constexpr (Gm::kSplitP)
-          tc::mma_ss(t_base, tc::sw128_desc(pa + Gm::kPBytes + kk * 32, 16, 1024), bd, kIdescPV, true);
-      }
-      tc::commit(bar_pv);
-      // a 16-bit stage holds the operands themselves: free once S(t) and PV(t) are done
-      if constexpr (Gm::k16) tc::commit(&bar_empty[t % kStages]);
-    };
-
     // ---- main loop ----
+    // A warp leaves when one of its threads' waits gave up (tensor-memory loads
+    // and stores are collective over the warp, so the decision is too). 16-bit
+    // caches: at any wait, no barrier spans warps inside the loop. Quantized
+    // caches: at the consensus of a dequantization, which the whole CTA takes
+    // together (or after the last tile, where no barrier follows).
+    auto leave = [&]() -> bool { return !__all_sync(kFull, ok); };
     float m = -INFINITY, l = 0.f, vref = 0.f;
-    int pv_done = 0;  // PV products issued so far
     mask_next = prepare(0);
-    if (!(Gm::k16 ? wg_all(wg, ok) : ok)) aborted = true;
-    else {
-      if (r == 0) issue_s(0);
-      n_s = 1;
-    }
+    if (leave()) aborted = true;
 
     for (int t = 0; t < T && !aborted; ++t) {
       mask_cur = mask_next;
-      if (t + 1 < T) {
-        mask_next = prepare(t + 1);
-        if (Gm::k16 ? true : ok) {
-          if (r == 0) issue_s(t + 1);
-          ++n_s;
-        } else {
-          aborted = true;
-          break;
-        }
+      // PV(t - 2) is done: its P (in the S buffer S(t) now holds) has been read,
+      // and, for quantized caches, the V operand buffer that tile t + 1 takes
+      if (t >= 2) ok = mbar_wait_bounded(&my_pv[t & 1], (uint32_t)((t - 2) >> 1) & 1u, p.timeout_ns) && ok;
+      if (t + 1 < T) mask_next = prepare(t + 1);
+      if (leave()) {
+        aborted = true;
+        break;
       }
-      ok = mbar_wait_bounded(&bar_s[t & 1], (ph_s >> (t & 1)) & 1u, p.timeout_ns) && ok;
-      ph_s ^= 1u << (t & 1);
-      ++n_s_waited;
+      ok = mbar_wait_bounded(&my_s[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns) && ok;
+      if (Gm::k16 && leave()) {
+        aborted = true;
+        break;
+      }
       tc::fence_after_sync();
 
       // scores of this row
+      const uint32_t t_s = t_row + D + 64 * (t & 1);
       uint32_t sv[64];
       {
         uint32_t a[32], c2[32];
-        tc::tmem_ld32(t_row + D + 64 * (t & 1), a);
-        tc::tmem_ld32(t_row + D + 64 * (t & 1) + 32, c2);
+        tc::tmem_ld32(t_s, a);
+        tc::tmem_ld32(t_s + 32, c2);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
           sv[i] = a[i];
@@ -641,14 +678,12 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         l += ((ra[0] + ra[1]) + (ra[2] + ra[3])) + ((rb[0] + rb[1]) + (rb[2] + rb[3]));
       }
 
-      // PV(t-1) must be done before O is rescaled or P is overwritten
-      if (t > 0) {
-        ok = mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns) && ok;
-        ph_pv ^= 1u;
-        ++n_pv_waited;
+
+      // O is rescaled once PV(t - 1) is done, before PV(t) is issued (which
+      // waits for this warp's P(t) below)
+      if (t > 0 && __any_sync(kFull, fo != 1.f)) {
+        ok = mbar_wait_bounded(&my_pv[(t - 1) & 1], (uint32_t)((t - 1) >> 1) & 1u, p.timeout_ns) && ok;
         tc::fence_after_sync();
-      }
-      if (pv_done > 0 && __any_sync(kFull, fo != 1.f)) {
 #pragma unroll 1
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -658,51 +693,24 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           tc::tmem_st32(t_row + c0, o);
         }
       }
-      // P row -> shared memory (K-major operand, 128-byte swizzle)
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        *reinterpret_cast<uint4*>(sP + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-        if constexpr (Gm::kSplitP)
-          *reinterpret_cast<uint4*>(sP + Gm::kPBytes + r * 128 + ((c ^ (r & 7)) << 4)) =
-              make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
-      }
-      tc::fence_smem_to_async();
+      // P row -> tensor memory over this row's S(t) (P_hi, then P_lo for bf16),
+      // then this warp's share of P(t) is handed to the MMA warp
+      tc::tmem_st32(t_s, pk);
+      if constexpr (Gm::kSplitP) tc::tmem_st32(t_s + 32, pl);
       tc::fence_before_sync();
-      // one barrier per tile: P complete and S read; for 16-bit caches it also
-      // decides on a timeout (quantized caches decide at the next dequantization)
-      if constexpr (Gm::k16) {
-        if (!wg_all(wg, ok)) {
-          aborted = true;
-          break;
-        }
-      } else {
-        wg_sync(wg);
-      }
-      if (r == 0) issue_pv(t, pv_done == 0);
-      ++pv_done;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&my_p[t & 1]);
     }
 
-    if (!aborted && pv_done > 0) {
-      ok = mbar_wait_bounded(bar_pv, ph_pv, p.timeout_ns) && ok;
-      if (!(Gm::k16 ? wg_all(wg, ok) : cta_all<NWG>(ok))) aborted = true;
-      else {
-        ph_pv ^= 1u;
-        ++n_pv_waited;
-      }
+    if (!aborted && T > 0) {
+      ok = mbar_wait_bounded(&my_pv[(T - 1) & 1], (uint32_t)((T - 1) >> 1) & 1u, p.timeout_ns) && ok;
+      if (leave()) aborted = true;
     }
     if (aborted) {
-      if (r == 0) {
+      if (lane == 0) {
         *abort_flag = 1;
         raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
       }
-      // let products still in flight finish (each wait bounded by the full limit)
-      bool drained = true;
-      for (int k = n_s_waited; k < n_s; ++k)
-        drained = mbar_wait_bounded(&bar_s[k & 1], (uint32_t)(k >> 1) & 1u, p.drain_ns) && drained;
-      for (int k = n_pv_waited; k < pv_done; ++k)
-        drained = mbar_wait_bounded(bar_pv, (uint32_t)k & 1u, p.drain_ns) && drained;
-      if (!drained) raise_flag(p.err, PQKV_DEVERR_DRAIN);
     } else {
       tc::fence_after_sync();
       const float inv = l > 0.f ? (Gm::kFp8 ? vref : 1.f) / l : 0.f;

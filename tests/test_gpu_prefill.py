@@ -139,3 +139,34 @@ def test_prefill_is_deterministic_and_layout_invariant():
     bt2[0, :n0] = free[:n0]
     c, _ = _run(g, q, cu, bt2, lens, 0.09)
     assert torch.equal(a, c)
+
+
+@pytest.mark.parametrize("case", [CASES[0], CASES[4], CASES[6]], ids=["bf16", "fp8", "fp4"])
+def test_prefill_wait_limit_runs_out_and_the_next_call_is_correct(case):
+    """With a 1 ns limit, the prefill's waits (on its copies, its tensor-core
+    products and the other warps) give up while the work is still on the way:
+    the call reports PQKV_DEVERR_TIMEOUT, lets every copy and product in flight
+    complete before its CTAs exit (no PQKV_DEVERR_DRAIN) and leaves the
+    context usable; the next call with the normal limit matches the oracle.
+    Nothing is dropped or corrupted to cause the timeout: only the limit is
+    short."""
+    lens, qlens = [1500, 700, 300], [512, 200, 300]
+    g, o, bt, cu, q = _build(case, lens, qlens, seed=77)
+    seen = 0
+    pq.set_decode_wait_limit_ns(1)
+    try:
+        for _ in range(5):
+            _, e = _run(g, q, cu, bt, lens, 0.088)  # synchronized: no fault, no hang
+            assert e & pq.DEVERR_DRAIN == 0, "work was still in flight when its CTA gave up draining"
+            assert e & ~pq.DEVERR_TIMEOUT == 0
+            seen += (e & pq.DEVERR_TIMEOUT) != 0
+            if seen:
+                break
+    finally:
+        pq.set_decode_wait_limit_ns(0)
+    assert seen, "no wait ran out with a 1 ns limit"
+    out, e = _run(g, q, cu, bt, lens, 0.088)
+    assert e == 0
+    ref, rerr = oracle.paged_prefill(o, q, cu, bt, np.array(lens, np.int32), 0.088)
+    assert rerr == 0
+    gh.assert_close(out, ref, case[0], tag="prefill after a timeout")
