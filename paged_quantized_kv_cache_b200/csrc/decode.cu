@@ -806,6 +806,9 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
   load_entry(lane, wid, wh);
   load_entry(32 + lane, nid, nh);
   uint32_t skip = 0;
+  // KV tiles are read once: evicted first, so that split partials stay in L2
+  // until they are merged
+  const uint64_t kv_policy = l2_evict_first_policy();
   auto issue = [&](int s, int v) {
     while (v - wbase >= 32) {
       wbase += 32;
@@ -830,7 +833,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
         constexpr int kElem = Gm::k16 ? 2 : 1;
 #pragma unroll
         for (int bx = 0; bx < Gm::kBoxes; ++bx)
-          tma_load_2d(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar);
+          tma_load_2d_hint(dst + bx * 32 * Gm::kBoxRow, &tmap, bx * (Gm::kBoxRow / kElem), coord, bar, kv_policy);
         const size_t pair = (size_t)id * Hkv + hh;
         uint8_t* side = wside + s * Gm::kSideStride;
         if constexpr (Gm::kFp8) {

@@ -185,6 +185,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* n_issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
+  volatile int* stage_mask = reinterpret_cast<volatile int*>(tmem_slot + 4);  // [kStages] blocks fetched
 
   asm volatile("griddepcontrol.wait;" ::: "memory");  // the chunk's K/V may come from the previous kernel
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -319,6 +320,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
             }
           }
         }
+        stage_mask[s] = mask;  // published to the consumers by the stage's barrier
         mbar_arrive_expect_tx(&bar_full[s], bytes);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -432,17 +434,10 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       const int s = t % kStages;
       ok = mbar_wait_bounded(&bar_full[s], (uint32_t)(t / kStages) & 1u, p.timeout_ns) && ok;
       ++n_prepared;
-      // blocks of the tile that were fetched (as the producer decided), from the
-      // block table itself so that every thread agrees even after a timeout
-      int mask = 0;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int blk = 4 * t + j;
-        if (blk * kBlock < n_kv) {
-          const int id = __ldg(table + blk);
-          if (id >= 0 && id < p.nb) mask |= 1 << j;
-        }
-      }
+      // blocks of the tile that were fetched, as the producer left them beside
+      // the stage (after a timeout the value may be stale: it is the same for
+      // every thread, and the results are not used then)
+      const int mask = stage_mask[s];
       const int base = t * kN;
       uint8_t* st = sStage + s * Gm::kStageBytes;
       if constexpr (Gm::k16) {
@@ -585,16 +580,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       // scores of this row
       const uint32_t t_s = t_row + D + 64 * (t & 1);
       uint32_t sv[64];
-      {
-        uint32_t a[32], c2[32];
-        tc::tmem_ld32(t_s, a);
-        tc::tmem_ld32(t_s + 32, c2);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          sv[i] = a[i];
-          sv[32 + i] = c2[i];
-        }
-      }
+      tc::tmem_ld64(t_s, sv);
       const int mask = mask_cur;
       // no column of this tile is masked for any row of the warpgroup: all 4
       // blocks valid and the tile ends at or before the first row's position
@@ -695,8 +681,17 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       }
       // P row -> tensor memory over this row's S(t) (P_hi, then P_lo for bf16),
       // then this warp's share of P(t) is handed to the MMA warp
-      tc::tmem_st32(t_s, pk);
-      if constexpr (Gm::kSplitP) tc::tmem_st32(t_s + 32, pl);
+      if constexpr (Gm::kSplitP) {
+        uint32_t pp[64];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          pp[i] = pk[i];
+          pp[32 + i] = pl[i];
+        }
+        tc::tmem_st64(t_s, pp);
+      } else {
+        tc::tmem_st32(t_s, pk);
+      }
       tc::fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&my_p[t & 1]);

@@ -220,8 +220,10 @@ __device__ __forceinline__ uint2 e2m1_codes16(const float (&x)[16], float d, flo
 // groups per token) for block rows tl, tl + TL, ... (tl = l / GPL, TL = 32 /
 // GPL): a token-group's absmax, scale and codes stay in one lane, and the two
 // rows of a V token pair (r, r ^ 1) sit in lanes l and l ^ GPL.
+// Four CTAs per SM (at most 128 registers a thread): the kernel is bound by
+// instruction issue, and 16 warps per SM hide more latency than 12.
 template <int D, bool INBF16>
-__global__ void __launch_bounds__(128) write_fp4_kernel(const WriteParams p) {
+__global__ void __launch_bounds__(128, 4) write_fp4_kernel(const WriteParams p) {
   // inputs may come from the previous kernel; let the next one start launching
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
