@@ -16,10 +16,11 @@
 //     tensor-memory lane r of the warpgroup's 256 columns): online softmax,
 //     and for quantized caches the dequantization of each tile (both together);
 //   a producer warp: refills each stage of a 4-deep ring as soon as it is
-//     released (by the MMA warp's commit after the last product reading it, or
+//     released (by the MMA warps' commits after the last products reading it, or
 //     once its raw codes are dequantized);
-//   an MMA warp: issues every tensor-core product and commits each to an
-//     mbarrier, so no compute warp waits on a barrier with the others.
+//   an MMA warp per warpgroup: issues its tensor-core products and commits
+//     each to an mbarrier, so no compute warp waits on a barrier with the
+//     others, and neither warpgroup's products wait for the other's P.
 // Per KV tile t of 64 tokens (4 cache blocks) and warpgroup:
 //   S(t) = Q K(t)^T        tcgen05.mma M=128 N=64 (A, B in shared memory),
 //                          into one of two S buffers in tensor memory
@@ -62,7 +63,7 @@ struct PrefillGeom {
   // rows). Quantized tiles are dequantized by both together.
   static constexpr int NWG = 2;
   static constexpr int kStages = 4;                // KV tiles in flight (shared memory)
-  static constexpr int kThreads = NWG * kWG + 64; // + one producer warp + one MMA warp
+  static constexpr int kThreads = NWG * kWG + 32 + 32 * NWG;  // + a producer warp + an MMA warp per warpgroup
   static constexpr int NB = D / 64;                // 128-byte boxes per operand row
   static constexpr int kQBytes = NB * kM * 128;    // Q operand of one warpgroup [box][128 rows][128 B]
   static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
@@ -179,8 +180,8 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   uint64_t* bar_p = bar_s + 2 * NWG;         // [NWG][2] P(t) in tensor memory (one arrival per warp)
   uint64_t* bar_pv = bar_p + 2 * NWG;        // [NWG][2] PV(t) computed
   uint64_t* bar_op = bar_pv + 2 * NWG;       // [2] quantized: operands of tile t dequantized
-  uint64_t* bar_drain = bar_op + 2;          // every product issued has completed
-  float* tile_sk = reinterpret_cast<float*>(bar_drain + 1);  // [2][4] FP8 K scales
+  uint64_t* bar_drain = bar_op + 2;          // [NWG] every product an MMA warp issued has completed
+  float* tile_sk = reinterpret_cast<float*>(bar_drain + NWG);  // [2][4] FP8 K scales
   float* tile_sv = tile_sk + 8;                              // [2][4] FP8 V scales
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -200,7 +201,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
   if (qn <= 0 || mt0 * TOK >= qn) return;
   const bool is_compute = tid < NWG * kWG;
-  const bool is_producer = warp == NWG * 4, is_mma = warp == NWG * 4 + 1;
+  const bool is_producer = warp == NWG * 4, is_mma = warp > NWG * 4;
   const int wg = is_compute ? tid / kWG : 0;
   const int r = tid % kWG;                           // row of this thread in its warpgroup's tile
   const int i0 = (mt0 + wg) * TOK;                   // first query token of the warpgroup's tile
@@ -227,7 +228,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   if (tid == 32) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&bar_full[s], 1);
-      mbar_init(&bar_empty[s], 1);  // 16-bit: the MMA warp's commit; else one arrival once dequantized
+      mbar_init(&bar_empty[s], Gm::k16 ? NWG : 1);  // 16-bit: each MMA warp's commit; else dequantized
     }
     for (int i = 0; i < 2 * NWG; ++i) {
       mbar_init(&bar_s[i], 1);
@@ -236,7 +237,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     }
     mbar_init(&bar_op[0], 1);
     mbar_init(&bar_op[1], 1);
-    mbar_init(bar_drain, 1);
+    for (int i = 0; i < NWG; ++i) mbar_init(&bar_drain[i], 1);
     *abort_flag = 0;
     *n_issued_slot = 0;
     fence_mbar_init();
@@ -350,11 +351,13 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       *n_issued_slot = t;
     }
   } else if (is_mma) {
-    // ================= MMA warp: every tensor-core product of both warpgroups =================
-    // Order per KV tile t: PV(t) of each warpgroup once its P(t) is in tensor
-    // memory, then S(t + 2) of each warpgroup into the buffer P(t) occupied,
-    // once PV(t) has read it. S(0) and S(1) are issued up front, so a
-    // warpgroup always finds the scores of its next tile computed.
+    // ================= MMA warp w: every tensor-core product of warpgroup w =================
+    // Order per KV tile t: PV(t) once the warpgroup's P(t) is in tensor memory,
+    // then S(t + 2) into the buffer P(t) occupied, once PV(t) has read it.
+    // S(0) and S(1) are issued up front, so the warpgroup finds the scores of
+    // its next tile computed. One MMA warp per warpgroup keeps the two chains
+    // independent: neither waits for the other's P (they share the tensor pipe).
+    const int w = warp - (NWG * 4 + 1);
     if (lane == 0) {
       bool good = true;
       // operands of tile t ready: 16-bit K/V landed; quantized tiles dequantized
@@ -364,7 +367,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         else
           return mbar_wait_bounded(&bar_op[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
       };
-      auto issue_s = [&](int t, int w) {
+      auto issue_s = [&](int t) {
         tc::fence_after_sync();
         const uint32_t d = tmem + 256u * w + D + 64 * (t & 1);
         const uint8_t* kop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes : sKop + (t & 1) * Gm::kOpBytes;
@@ -377,7 +380,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         }
         tc::commit(&bar_s[2 * w + (t & 1)]);
       };
-      auto issue_pv = [&](int t, int w) {
+      auto issue_pv = [&](int t) {
         tc::fence_after_sync();
         const uint8_t* vop = Gm::k16 ? sStage + (t % kStages) * Gm::kStageBytes + Gm::kOpBytes
                                      : sVop + (t % 3) * Gm::kOpBytes;
@@ -392,23 +395,19 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       };
       for (int t = 0; t < min(2, T) && good; ++t) {
         good = ready(t);
-        if (good)
-          for (int w = 0; w < NWG; ++w) issue_s(t, w);
+        if (good) issue_s(t);
       }
       for (int t = 0; t < T && good; ++t) {
-        for (int w = 0; w < NWG && good; ++w) {
-          good = mbar_wait_bounded(&bar_p[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
-          if (good) issue_pv(t, w);
-        }
+        good = mbar_wait_bounded(&bar_p[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
         if (!good) break;
-        // a 16-bit stage holds the operands themselves: free once S(t) and PV(t) are done
+        issue_pv(t);
+        // a 16-bit stage holds the operands themselves: free once S(t) and PV(t)
+        // of every warpgroup are done (one commit per MMA warp)
         if constexpr (Gm::k16) tc::commit(&bar_empty[t % kStages]);
         if (t + 2 < T) {
-          good = ready(t + 2);
-          for (int w = 0; w < NWG && good; ++w) {
-            good = mbar_wait_bounded(&bar_pv[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
-            if (good) issue_s(t + 2, w);
-          }
+          good = ready(t + 2) &&
+                 mbar_wait_bounded(&bar_pv[2 * w + (t & 1)], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
+          if (good) issue_s(t + 2);
         }
       }
       if (!good) {
@@ -416,8 +415,8 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
       }
       // every product issued completes before tensor memory is released
-      tc::commit(bar_drain);
-      if (!mbar_wait_bounded(bar_drain, 0, p.drain_ns)) raise_flag(p.err, PQKV_DEVERR_DRAIN);
+      tc::commit(&bar_drain[w]);
+      if (!mbar_wait_bounded(&bar_drain[w], 0, p.drain_ns)) raise_flag(p.err, PQKV_DEVERR_DRAIN);
     }
   } else if (is_compute) {
     // ================= compute warpgroup wg: one row per thread =================
