@@ -13,11 +13,13 @@
 // row is (query token, query head of the GQA group), so a tile holds 128 / G
 // query tokens. Warps have one role each:
 //   two compute warpgroups, one row per thread (its S, P and O rows live in
-//     tensor-memory lane r of the warpgroup's 256 columns): online softmax,
-//     and for quantized caches the dequantization of each tile (both together);
+//     tensor-memory lane r of the warpgroup's 256 columns): online softmax;
 //   a producer warp: refills each stage of a 4-deep ring as soon as it is
 //     released (by the MMA warps' commits after the last products reading it, or
 //     once its raw codes are dequantized);
+//   for quantized caches, a dequantization warpgroup: turns each tile's raw
+//     codes into f16 operands as soon as the products that read the previous
+//     contents of its operand buffers are done;
 //   an MMA warp per warpgroup: issues its tensor-core products and commits
 //     each to an mbarrier, so no compute warp waits on a barrier with the
 //     others, and neither warpgroup's products wait for the other's P.
@@ -63,7 +65,14 @@ struct PrefillGeom {
   // rows). Quantized tiles are dequantized by both together.
   static constexpr int NWG = 2;
   static constexpr int kStages = 4;                // KV tiles in flight (shared memory)
-  static constexpr int kThreads = NWG * kWG + 32 + 32 * NWG;  // + a producer warp + an MMA warp per warpgroup
+  // quantized caches: a dequantization warpgroup; 128 threads take the 64 x D/8
+  // operand chunks of a tile in a fixed number of rounds, unrolled so that the
+  // chains of several chunks overlap (16 warps in all: at most 4 per scheduler,
+  // so 128 registers a thread fit)
+  static constexpr int kDeqWarps = k16 ? 0 : 4;
+  static constexpr int kDeqThreads = 32 * kDeqWarps;
+  // compute warpgroups + a producer warp + an MMA warp per warpgroup (+ dequantization)
+  static constexpr int kThreads = NWG * kWG + 32 + 32 * NWG + kDeqThreads;
   static constexpr int NB = D / 64;                // 128-byte boxes per operand row
   static constexpr int kQBytes = NB * kM * 128;    // Q operand of one warpgroup [box][128 rows][128 B]
   static constexpr int kOpBytes = NB * kN * 128;   // one K or V operand tile [box][64 rows][128 B]
@@ -105,20 +114,21 @@ __device__ __forceinline__ uint32_t to_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// Barrier of all compute threads (named barrier 3), and its and-reduction.
-template <int NWG>
-__device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 3, %0;" ::"n"(NWG * 128) : "memory"); }
-template <int NWG>
-__device__ __forceinline__ bool cta_all(bool v) {
+// Barrier of the N dequantization threads (named barrier 1), and its and-reduction.
+template <int N>
+__device__ __forceinline__ void deq_sync() { asm volatile("bar.sync 1, %0;" ::"n"(N) : "memory"); }
+template <int N>
+__device__ __forceinline__ bool deq_all(bool v) {
   uint32_t r;
   asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 3, %2, p;\n\t"
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\tbar.red.and.pred q, 1, %2, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
-      : "r"((uint32_t)v), "n"(NWG * 128)
+      : "r"((uint32_t)v), "n"(N)
       : "memory");
   return r != 0;
 }
+
 // Packed pairs of fp32 operations (two lanes of IEEE fp32 arithmetic, rounded to
 // nearest, in one instruction): (d0, d1) = (a0, a1) op (b0, b1) [+ (c0, c1)].
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
@@ -179,11 +189,14 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   uint64_t* bar_s = bar_empty + kStages;     // [NWG][2] S(t) computed (buffer t % 2)
   uint64_t* bar_p = bar_s + 2 * NWG;         // [NWG][2] P(t) in tensor memory (one arrival per warp)
   uint64_t* bar_pv = bar_p + 2 * NWG;        // [NWG][2] PV(t) computed
-  uint64_t* bar_op = bar_pv + 2 * NWG;       // [2] quantized: operands of tile t dequantized
-  uint64_t* bar_drain = bar_op + 2;          // [NWG] every product an MMA warp issued has completed
-  float* tile_sk = reinterpret_cast<float*>(bar_drain + NWG);  // [2][4] FP8 K scales
-  float* tile_sv = tile_sk + 8;                              // [2][4] FP8 V scales
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tile_sv + 8);
+  uint64_t* bar_op = bar_pv + 2 * NWG;       // [4] quantized: operands, mask and scales of tile t ready
+  uint64_t* bar_kfree = bar_op + 4;          // [2] quantized: S(t) of every warpgroup done (kop[t % 2])
+  uint64_t* bar_vfree = bar_kfree + 2;       // [3] quantized: PV(t) of every warpgroup done (vop[t % 3])
+  uint64_t* bar_drain = bar_vfree + 3;       // [NWG] every product an MMA warp issued has completed
+  float* tile_sk = reinterpret_cast<float*>(bar_drain + NWG);  // [4][4] FP8 K scales of tile t % 4
+  float* tile_sv = tile_sk + 16;                               // [4][4] FP8 V scales
+  volatile int* op_mask = reinterpret_cast<volatile int*>(tile_sv + 16);  // [4] quantized: blocks of tile t % 4
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(const_cast<int*>(op_mask) + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* n_issued_slot = reinterpret_cast<int*>(tmem_slot + 2);
   volatile int* stage_mask = reinterpret_cast<volatile int*>(tmem_slot + 4);  // [kStages] blocks fetched
@@ -201,7 +214,8 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     raise_flag(p.err, PQKV_DEVERR_SEQ_LEN);  // rows past max_q_len are not computed
   if (qn <= 0 || mt0 * TOK >= qn) return;
   const bool is_compute = tid < NWG * kWG;
-  const bool is_producer = warp == NWG * 4, is_mma = warp > NWG * 4;
+  const bool is_producer = warp == NWG * 4;
+  const bool is_mma = warp > NWG * 4 && warp <= NWG * 4 + NWG, is_deq = warp > NWG * 4 + NWG;
   const int wg = is_compute ? tid / kWG : 0;
   const int r = tid % kWG;                           // row of this thread in its warpgroup's tile
   const int i0 = (mt0 + wg) * TOK;                   // first query token of the warpgroup's tile
@@ -235,8 +249,9 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       mbar_init(&bar_p[i], 4);
       mbar_init(&bar_pv[i], 1);
     }
-    mbar_init(&bar_op[0], 1);
-    mbar_init(&bar_op[1], 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&bar_op[i], 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&bar_kfree[i], NWG);
+    for (int i = 0; i < 3; ++i) mbar_init(&bar_vfree[i], NWG);
     for (int i = 0; i < NWG; ++i) mbar_init(&bar_drain[i], 1);
     *abort_flag = 0;
     *n_issued_slot = 0;
@@ -290,7 +305,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  int n_prepared = 0;  // KV tiles waited for by this thread (compute threads)
+  int n_prepared = 0;  // KV tiles this thread waited for, while no wait had given up
 
   if (is_producer) {
     // ================= producer warp: KV tiles into the stage ring =================
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         if constexpr (Gm::k16)
           return mbar_wait_bounded(&bar_full[t % kStages], (uint32_t)(t / kStages) & 1u, p.timeout_ns);
         else
-          return mbar_wait_bounded(&bar_op[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns);
+          return mbar_wait_bounded(&bar_op[t & 3], (uint32_t)(t >> 2) & 1u, p.timeout_ns);
       };
       auto issue_s = [&](int t) {
         tc::fence_after_sync();
@@ -379,6 +394,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           tc::mma_ss(d, a, bd, kIdescS, kk > 0);
         }
         tc::commit(&bar_s[2 * w + (t & 1)]);
+        if constexpr (!Gm::k16) tc::commit(&bar_kfree[t & 1]);  // the K operand buffer may be refilled
       };
       auto issue_pv = [&](int t) {
         tc::fence_after_sync();
@@ -392,6 +408,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           if constexpr (Gm::kSplitP) tc::mma_ts(o, pa + 32 + kk * 8, bd, kIdescPV, true);
         }
         tc::commit(&bar_pv[2 * w + (t & 1)]);
+        if constexpr (!Gm::k16) tc::commit(&bar_vfree[t % 3]);  // the V operand buffer may be refilled
       };
       for (int t = 0; t < min(2, T) && good; ++t) {
         good = ready(t);
@@ -418,51 +435,34 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       tc::commit(&bar_drain[w]);
       if (!mbar_wait_bounded(&bar_drain[w], 0, p.drain_ns)) raise_flag(p.err, PQKV_DEVERR_DRAIN);
     }
-  } else if (is_compute) {
-    // ================= compute warpgroup wg: one row per thread =================
-    const uint32_t t_row = tmem + 256u * wg + ((uint32_t)(32 * (warp & 3)) << 16);
-    uint64_t* my_s = bar_s + 2 * wg;
-    uint64_t* my_p = bar_p + 2 * wg;
-    uint64_t* my_pv = bar_pv + 2 * wg;
-    bool ok = true;  // no wait of this thread has timed out
-    bool aborted = false;
-    int mask_cur = 0, mask_next = 0;  // blocks of tile t / t + 1 holding data
-
-    // ---- make KV tile t's operands ready; returns its block mask ----
-    auto prepare = [&](int t) -> int {
-      const int s = t % kStages;
-      ok = mbar_wait_bounded(&bar_full[s], (uint32_t)(t / kStages) & 1u, p.timeout_ns) && ok;
-      ++n_prepared;
-      // blocks of the tile that were fetched, as the producer left them beside
-      // the stage (after a timeout the value may be stale: it is the same for
-      // every thread, and the results are not used then)
-      const int mask = stage_mask[s];
-      const int base = t * kN;
-      uint8_t* st = sStage + s * Gm::kStageBytes;
-      if constexpr (Gm::k16) {
-        // V rows without valid data (past the sequence, or a block not loaded)
-        // are zeroed: P is 0 there, and 0 x NaN would poison O. Each warpgroup
-        // zeroes before its own P(t) is handed over (the same zeros), so the
-        // product PV(t) of each warpgroup follows its own zeroing.
-        if (mask != 0xF || base + kN > L) {
-          for (int u = r; u < kN * Gm::NB * 8; u += kWG) {
-            const int rr = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
-            if (((mask >> (rr >> 4)) & 1) && base + rr < L) continue;
-            *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + rr * 128 + ((k & 7) << 4)) =
-                make_uint4(0, 0, 0, 0);
-          }
-          tc::fence_smem_to_async();
-        }
-      } else {
-        // both warpgroups are past the products that read the operand buffers
-        // written below (S(t - 2) and PV(t - 3), waited for by each before
-        // this barrier), then dequantize half of the tile each
-        cta_sync<NWG>();
-        const int gt = wg * kWG + r;
+  } else if (is_deq) {
+    // ================= dequantization warps (quantized caches) =================
+    // Tile t: raw codes landed, the operand buffers free again (S(t - 2) read
+    // kop[t % 2], PV(t - 3) read vop[t % 3], for both warpgroups), then the
+    // codes become f16 operands; bar_op[t % 4] hands them, the tile's block
+    // mask and FP8 scales to the MMA and compute warps, and the raw stage goes
+    // back to the producer. The dequantization warps leave together, at a consensus.
+    if constexpr (!Gm::k16) {
+      const int dq = tid - (NWG * 4 + 1 + NWG) * 32;  // 0 .. kDeqThreads - 1
+      bool ok = true;
+      for (int t = 0; t < T; ++t) {
+        const int s = t % kStages;
+        ok = mbar_wait_bounded(&bar_full[s], (uint32_t)(t / kStages) & 1u, p.timeout_ns) && ok;
+        if (ok) ++n_prepared;  // counted up to the first wait that gave up: the drain covers the rest
+        if (t >= 2) ok = mbar_wait_bounded(&bar_kfree[t & 1], (uint32_t)((t >> 1) - 1) & 1u, p.timeout_ns) && ok;
+        if (t >= 3) ok = mbar_wait_bounded(&bar_vfree[t % 3], (uint32_t)((t / 3) - 1) & 1u, p.timeout_ns) && ok;
+        ok = deq_all<Gm::kDeqThreads>(ok);
+        if (!ok) break;
+        // blocks of the tile that were fetched, as the producer left them beside the stage
+        const int mask = stage_mask[s];
+        const int base = t * kN;
+        uint8_t* st = sStage + s * Gm::kStageBytes;
         uint8_t* kop = sKop + (t & 1) * Gm::kOpBytes;
         uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
         constexpr int CPR = D / 8;  // 16-byte operand chunks per row
-        for (int u = gt; u < kN * CPR; u += NWG * kWG) {
+        static_assert(kN * CPR % Gm::kDeqThreads == 0, "whole rounds");
+#pragma unroll
+        for (int u = dq; u < kN * CPR; u += Gm::kDeqThreads) {
           const int rr = u / CPR, c = u % CPR, j = rr >> 4, tr = rr & 15;
           const bool okr = ((mask >> j) & 1) && base + rr < L;
           uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
@@ -507,42 +507,83 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         }
         if constexpr (Gm::kFp4) {
           // outlier channels (their codes are 0): write the fp16 values over them;
-          // thread = (block j, K|V, slot, eighth of the tokens)
-          cta_sync<NWG>();
-          const int j = gt >> 6, kv = (gt >> 5) & 1, slot = (gt >> 3) & 3, part = gt & 7;
-          if ((mask >> j) & 1) {
-            const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
-            const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
-            if (ch < D) {
-              const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes) + kv * 64;
-              uint8_t* op = kv ? vop : kop;
-              const int c = ch >> 3;
+          // item = (block j, K|V, slot, eighth of the tokens)
+          deq_sync<Gm::kDeqThreads>();
+          for (int gt = dq; gt < 256; gt += Gm::kDeqThreads) {
+            const int j = gt >> 6, kv = (gt >> 5) & 1, slot = (gt >> 3) & 3, part = gt & 7;
+            if ((mask >> j) & 1) {
+              const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
+              const int ch = side[Gm::kScaleBytes + Gm::kValBytes + 8 * kv + slot];
+              if (ch < D) {
+                const uint16_t* val = reinterpret_cast<const uint16_t*>(side + Gm::kScaleBytes) + kv * 64;
+                uint8_t* op = kv ? vop : kop;
+                const int c = ch >> 3;
 #pragma unroll
-              for (int q4 = 0; q4 < 2; ++q4) {
-                const int tr = 2 * part + q4, rr = 16 * j + tr;
-                if (base + rr < L)
-                  *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4) +
-                                               (ch & 7) * 2) = val[tr * 4 + slot];
+                for (int q4 = 0; q4 < 2; ++q4) {
+                  const int tr = 2 * part + q4, rr = 16 * j + tr;
+                  if (base + rr < L)
+                    *reinterpret_cast<uint16_t*>(op + (c >> 3) * (kN * 128) + rr * 128 + (((c & 7) ^ (rr & 7)) << 4) +
+                                                 (ch & 7) * 2) = val[tr * 4 + slot];
+                }
               }
             }
           }
         }
         if constexpr (Gm::kFp8) {
-          if (gt < 4) {
-            const bool okb = (mask >> gt) & 1;
-            const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + gt * Gm::kSide);
-            tile_sk[(t & 1) * 4 + gt] = okb ? sc[0] : 0.f;
-            tile_sv[(t & 1) * 4 + gt] = okb ? sc[1] : 0.f;
+          if (dq < 4) {
+            const bool okb = (mask >> dq) & 1;
+            const float* sc = reinterpret_cast<const float*>(st + 4 * Gm::kRawTile + dq * Gm::kSide);
+            tile_sk[(t & 3) * 4 + dq] = okb ? sc[0] : 0.f;
+            tile_sv[(t & 3) * 4 + dq] = okb ? sc[1] : 0.f;
           }
         }
+        if (dq == 0) op_mask[t & 3] = mask;
         tc::fence_smem_to_async();
-        // the products may read the operands once every thread wrote its part;
-        // the consensus over both warpgroups also carries timeouts (quantized
-        // caches abort only here, so that neither warpgroup is left waiting)
-        ok = cta_all<NWG>(ok);
-        if (gt == 0 && ok) {
+        deq_sync<Gm::kDeqThreads>();  // every thread's part is written
+        if (dq == 0) {
           mbar_arrive(&bar_empty[s]);  // a raw stage is free as soon as it is dequantized
-          mbar_arrive(&bar_op[t & 1]);
+          mbar_arrive(&bar_op[t & 3]);
+        }
+      }
+      if (!ok && dq == 0) {
+        *abort_flag = 1;
+        raise_flag(p.err, PQKV_DEVERR_TIMEOUT);
+      }
+    }
+  } else if (is_compute) {
+    // ================= compute warpgroup wg: one row per thread =================
+    const uint32_t t_row = tmem + 256u * wg + ((uint32_t)(32 * (warp & 3)) << 16);
+    uint64_t* my_s = bar_s + 2 * wg;
+    uint64_t* my_p = bar_p + 2 * wg;
+    uint64_t* my_pv = bar_pv + 2 * wg;
+    bool ok = true;  // no wait of this thread has timed out
+    bool aborted = false;
+    int mask_cur = 0, mask_next = 0;  // blocks of tile t / t + 1 holding data
+
+    // ---- 16-bit caches: KV tile t landed, V rows without data zeroed; returns its block mask ----
+    auto prepare = [&](int t) -> int {
+      const int s = t % kStages;
+      ok = mbar_wait_bounded(&bar_full[s], (uint32_t)(t / kStages) & 1u, p.timeout_ns) && ok;
+      if (ok) ++n_prepared;  // counted up to the first wait that gave up: the drain covers the rest
+      // blocks of the tile that were fetched, as the producer left them beside
+      // the stage (after a timeout the value may be stale: it is the same for
+      // every thread, and the results are not used then)
+      const int mask = stage_mask[s];
+      const int base = t * kN;
+      uint8_t* st = sStage + s * Gm::kStageBytes;
+      if constexpr (Gm::k16) {
+        // V rows without valid data (past the sequence, or a block not loaded)
+        // are zeroed: P is 0 there, and 0 x NaN would poison O. Each warpgroup
+        // zeroes before its own P(t) is handed over (the same zeros), so the
+        // product PV(t) of each warpgroup follows its own zeroing.
+        if (mask != 0xF || base + kN > L) {
+          for (int u = r; u < kN * Gm::NB * 8; u += kWG) {
+            const int rr = u / (Gm::NB * 8), k = u % (Gm::NB * 8);
+            if (((mask >> (rr >> 4)) & 1) && base + rr < L) continue;
+            *reinterpret_cast<uint4*>(st + Gm::kOpBytes + (k >> 3) * kN * 128 + rr * 128 + ((k & 7) << 4)) =
+                make_uint4(0, 0, 0, 0);
+          }
+          tc::fence_smem_to_async();
         }
       }
       return mask;
@@ -550,30 +591,29 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
 
     // ---- main loop ----
     // A warp leaves when one of its threads' waits gave up (tensor-memory loads
-    // and stores are collective over the warp, so the decision is too). 16-bit
-    // caches: at any wait, no barrier spans warps inside the loop. Quantized
-    // caches: at the consensus of a dequantization, which the whole CTA takes
-    // together (or after the last tile, where no barrier follows).
+    // and stores are collective over the warp, so the decision is too); no
+    // barrier spans warps inside the loop. S(t) done implies PV(t - 2) done
+    // (its MMA warp issues S(t) into the buffer P(t - 2) occupied only then).
     auto leave = [&]() -> bool { return !__all_sync(kFull, ok); };
     float m = -INFINITY, l = 0.f, vref = 0.f;
-    mask_next = prepare(0);
-    if (leave()) aborted = true;
+    if constexpr (Gm::k16) {
+      mask_next = prepare(0);
+      if (leave()) aborted = true;
+    }
 
     for (int t = 0; t < T && !aborted; ++t) {
-      mask_cur = mask_next;
-      // PV(t - 2) is done: its P (in the S buffer S(t) now holds) has been read,
-      // and, for quantized caches, the V operand buffer that tile t + 1 takes
-      if (t >= 2) ok = mbar_wait_bounded(&my_pv[t & 1], (uint32_t)((t - 2) >> 1) & 1u, p.timeout_ns) && ok;
-      if (t + 1 < T) mask_next = prepare(t + 1);
+      if constexpr (Gm::k16) {
+        mask_cur = mask_next;
+        if (t + 1 < T) mask_next = prepare(t + 1);
+      }
+      ok = mbar_wait_bounded(&my_s[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns) && ok;
+      // quantized: the tile's block mask and FP8 scales, left by the dequantization
+      if constexpr (!Gm::k16) ok = mbar_wait_bounded(&bar_op[t & 3], (uint32_t)(t >> 2) & 1u, p.timeout_ns) && ok;
       if (leave()) {
         aborted = true;
         break;
       }
-      ok = mbar_wait_bounded(&my_s[t & 1], (uint32_t)(t >> 1) & 1u, p.timeout_ns) && ok;
-      if (Gm::k16 && leave()) {
-        aborted = true;
-        break;
-      }
+      if constexpr (!Gm::k16) mask_cur = op_mask[t & 3];
       tc::fence_after_sync();
 
       // scores of this row
@@ -585,20 +625,24 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       // blocks valid and the tile ends at or before the first row's position
       // (rows past the chunk keep a zero query and are never stored)
       const bool full = mask == 0xF && t * kN + kN - 1 <= pos0 + i0;
+      // raw scores; the log2-domain scale of block j (softmax scale, times the
+      // FP8 K scale of the block) is applied in the exponent's FMA. A block
+      // with no data has K scale 0 and all its scores masked (-inf): it takes
+      // scale 1 so that no 0 x inf arises; an all-zero K block has scores of
+      // exactly 0, whose logit is 0 with any scale.
       float vs[4] = {1.f, 1.f, 1.f, 1.f};
-      float xs[64];  // FP8: scores in log2 units; otherwise raw scores (scale applied in the exponent)
+      float cj[4] = {sl2, sl2, sl2, sl2};
       if constexpr (Gm::kFp8) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const float cj = sl2 * tile_sk[(t & 1) * 4 + j];
-          vs[j] = tile_sv[(t & 1) * 4 + j];
-#pragma unroll
-          for (int c = 16 * j; c < 16 * j + 16; ++c) xs[c] = __uint_as_float(sv[c]) * cj;
+          const float k = tile_sk[(t & 3) * 4 + j];
+          cj[j] = sl2 * (k > 0.f ? k : 1.f);
+          vs[j] = tile_sv[(t & 3) * 4 + j];
         }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 64; ++c) xs[c] = __uint_as_float(sv[c]);
       }
+      float xs[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) xs[c] = __uint_as_float(sv[c]);
       if (!full) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
@@ -606,13 +650,20 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
       }
       float mx;
       {
+        // max of each half-block in 8 chains, then of each block times its scale
+        // (positive: the max commutes with it; -inf stays -inf)
         float mp[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mp[i] = xs[i];
+        for (int i = 0; i < 8; ++i) mp[i] = xs[8 * i];
 #pragma unroll
-        for (int c = 8; c < 64; ++c) mp[c & 7] = fmaxf(mp[c & 7], xs[c]);
-        mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])), fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-        if constexpr (!Gm::kFp8) mx *= sl2;  // -inf stays -inf (the scale is positive)
+        for (int c = 0; c < 64; ++c)
+          if (c & 7) mp[c >> 3] = fmaxf(mp[c >> 3], xs[c]);
+        mx = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float mb = fmaxf(mp[2 * j], mp[2 * j + 1]);
+          if (mb != -INFINITY) mx = fmaxf(mx, mb * cj[j]);
+        }
       }
       float fm = 1.f;  // rescale of l and O for a larger row max
       if (mx > m + kLazy) {
@@ -646,8 +697,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
           float ya, yb;
-          if constexpr (Gm::kFp8) sub2(ya, yb, xs[c], xs[c + 1], mu, mu);
-          else fma2(ya, yb, xs[c], xs[c + 1], sl2, sl2, -mu, -mu);
+          fma2(ya, yb, xs[c], xs[c + 1], cj[c >> 4], cj[c >> 4], -mu, -mu);
           const float pa = ex2(ya), pb = ex2(yb);
           const int i = (c >> 1) & 3;
           add2(ra[i], rb[i], ra[i], rb[i], pa, pb);
@@ -729,8 +779,10 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (tid == 0) {
-    // tiles issued but never consumed (only after a timeout) land before the CTA exits
+  if (tid == (Gm::k16 ? 0 : (NWG * 4 + 1 + NWG) * 32)) {
+    // tiles issued but never consumed by this thread (the first compute thread
+    // for 16-bit caches, the first dequantization thread otherwise; only after
+    // a timeout) land before the CTA exits
     const int issued = *n_issued_slot;
     bool drained = true;
     for (int k = n_prepared; k < issued; ++k)
