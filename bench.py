@@ -374,11 +374,12 @@ def decode_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def profiled_traffic(workload: str, kv_name: str, split_blocks: int) -> int | None:
+def profiled_traffic(workload: str, kv_name: str, split_blocks: int, q_len: int = 1) -> int | None:
     """DRAM bytes per decode launch from a committed ncu summary, if it was
-    taken from the current kernel source with the same split."""
+    taken from the current kernel source with the same split (one query token
+    per sequence: the summaries are of the single-token decode)."""
     p = os.path.join(ROOT, "profiles", "decode_traffic_%s_%s.txt" % (workload, kv_name))
-    if not os.path.exists(p):
+    if q_len != 1 or not os.path.exists(p):
         return None
     vals = {}
     for line in open(p):
@@ -612,7 +613,7 @@ def measure_decode(args, s: W.Spec, device, world: int, kv_list=None, keep_kv: b
     achieved = b["decode_total"] / (dec_ms * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"],
-                "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype], args.split_blocks),
+                "traffic": profiled_traffic(args.workload, DT_LABEL[s.kv_dtype], args.split_blocks, args.q_len),
                 "kernel": "paged_decode_kernel", "peak_source": peaks["source"] + " (MEASURED_PEAKS.json hbm_gbs, "
                 "a read+write copy)", "bytes_per_launch": b["decode_total"], "avg_launch_ms": dec_ms,
                 "timing": "CUDA events around each decode call (one decode kernel per pass, which also merges the "
