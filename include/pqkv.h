@@ -201,15 +201,18 @@ size_t pqkv_decode_workspace_bytes(int batch, int num_q_heads, int num_kv_heads,
  * GPU; > 0 = process the KV of all (sequence, head) pairs, laid end to end, in
  * chunks of exactly that many 16-token blocks. Results differ only by rounding.
  * workspace: device buffer of at least pqkv_decode_workspace_bytes(...) bytes,
- * scratch for the split pieces and one arrival word per chunk. Two kernels run
+ * scratch for the split pieces and one arrival word per chunk. One kernel runs
  * on `stream`: the split decode, whose warp that writes the last piece of a
  * pair split into at most 4 pieces merges the pieces by log-sum-exp in chunk
- * order, then (as a programmatic dependent) the merge of pairs split into more
- * pieces (few long sequences), whose warps exit at once when there are none.
- * The arrival words carry a 40-bit tag of the launch, so the buffer needs no
- * clearing between calls; on a buffer's first use its old bytes could match a
- * tag with probability 2^-40 per split pair, which pqkv_decode_workspace_init
- * (zero fill) removes. Calls that share a workspace must be ordered.
+ * order; pairs split into more pieces (long sequences) are merged by warps of
+ * the same grid after their own share of the KV. The arrival words carry a tag
+ * of the launch whose top byte is 0xFF, so the buffer needs no clearing
+ * between calls, also when its layout (batch, heads, q_len, blocks per
+ * sequence, split) changes: zero bytes and the partial outputs of earlier
+ * calls never match a tag. Other old contents (a buffer's first use) match a
+ * tag with probability about 2^-40 per split pair, which
+ * pqkv_decode_workspace_init (zero fill) removes. Calls that share a workspace
+ * must be ordered.
  * batch <= PQKV_MAX_BATCH.
  */
 int pqkv_paged_decode_attention(const void* q, int q_dtype, int batch, int num_q_heads,
@@ -364,8 +367,8 @@ int pqkv_swap_in(void* cache, void* scales, void* outliers_idx, void* outliers_v
                  int32_t* err_flag, pqkv_stream_t stream);
 
 /* Zero-fill a decode workspace on `stream`. Optional: it only removes the
- * 2^-40 chance per split pair that a never-used buffer's old bytes match a
- * launch tag (see pqkv_paged_decode_attention). */
+ * chance (about 2^-40 per split pair) that a never-used buffer's arbitrary old
+ * bytes match a launch tag (see pqkv_paged_decode_attention). */
 int pqkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
                                pqkv_stream_t stream);
 

@@ -224,13 +224,18 @@ static size_t decode_chunks(int batch, int num_kv_heads, int max_blocks_per_seq,
   return split_blocks > 0 ? (total_blocks + split_blocks - 1) / split_blocks + warps : warps;
 }
 
-// Launch tags of the decode's arrival words: 40 bits, never 0, so a zeroed
-// word never matches.
+// Launch tags of the decode's arrival words (40 bits): 0xFF, then a 31-bit
+// launch counter that is never 0. An arrival word is (tag << 24) | pieces, so a
+// word matches a tag only if its high 32 bits, read as a float, are at most
+// -2^127 or a negative NaN (the top byte 0xFF), and not -inf (whose low bits
+// would need the counter's bit 31). A zeroed word, or one left over from the
+// partial outputs of a call with another layout (finite values, -inf row
+// maxima), never matches; the counter repeats only after 2^31 - 1 launches.
 static unsigned long long next_decode_epoch() {
   static std::atomic<unsigned long long> n{0};
   for (;;) {
-    const unsigned long long e = (n.fetch_add(1) + 1) & ((1ull << 40) - 1);
-    if (e != 0) return e;
+    const unsigned long long c = (n.fetch_add(1) + 1) & 0x7FFFFFFFull;
+    if (c != 0) return (0xFFull << 32) | c;
   }
 }
 

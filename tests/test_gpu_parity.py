@@ -219,6 +219,36 @@ def test_arrival_words_left_by_other_split_plans_do_not_matter():
     gh.assert_close(a, ref, case[0])
 
 
+def test_partial_floats_left_in_a_workspace_are_never_read_as_arrival_words():
+    """A workspace reused with another layout has its arrival words where
+    partial outputs were: float pairs such as (+0.0 above 1.0f) or a -inf row
+    maximum. Launch tags start with the byte 0xFF and use a 31-bit counter, so
+    no such word is taken for a tag: every call on a workspace filled with
+    these patterns equals the same call on a fresh one, bit for bit."""
+    case = CASES[4]
+    lens = [1200, 17, 700, 5, 333]
+    g, o, bt, q = _scenario(case, lens, seed=511)
+    bt_d = torch.from_numpy(bt).cuda()
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    qd = q.cuda()
+    pairs = [(0.0, 1.0), (float("-inf"), 0.0), (float("-inf"), float("-inf")), (0.5, -2.0), (-0.0, 3.0e38)]
+    for split in (1, 3, 0):
+        need = pq.decode_workspace_bytes(len(lens), case[3], case[4], case[2], bt.shape[1], split)
+        fresh = torch.zeros(need, dtype=torch.uint8, device="cuda")
+        b = torch.empty_like(qd)
+        e2 = gh.err_flag()
+        pq.paged_decode_attention(qd, g, bt_d, sl, 0.1, b, fresh, e2, split_blocks=split)
+        for lo, hi in pairs:
+            words = torch.tensor([lo, hi], dtype=torch.float32).repeat((need + 7) // 8)
+            ws = words.view(torch.uint8)[:need].clone().cuda()
+            a = torch.empty_like(qd)
+            e1 = gh.err_flag()
+            pq.paged_decode_attention(qd, g, bt_d, sl, 0.1, a, ws, e1, split_blocks=split)
+            torch.cuda.synchronize()
+            assert int(e1.item()) == int(e2.item()) == 0
+            assert torch.equal(a, b), "split %d, words (%r, %r)" % (split, lo, hi)
+
+
 def test_edge_lengths_and_error_bits():
     case = CASES[1]
     kv_dtype, qdt, D, Hq, Hkv = case
