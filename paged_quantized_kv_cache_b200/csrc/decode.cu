@@ -59,6 +59,15 @@ __device__ __forceinline__ void store_out(void* out, size_t i, float v) {
     reinterpret_cast<__half*>(out)[i] = __float2half_rn(v);
 }
 
+// out[i], out[i + 1] = a, b in one 4-byte store (i even).
+template <bool QBF16>
+__device__ __forceinline__ void store_out2(void* out, size_t i, float a, float b) {
+  if constexpr (QBF16)
+    *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + i) = __floats2bfloat162_rn(a, b);
+  else
+    *reinterpret_cast<__half2*>(reinterpret_cast<__half*>(out) + i) = __floats2half2_rn(a, b);
+}
+
 // Four E4M3 codes -> f16x2 of bytes (0,1) and (2,3) by the hardware conversion.
 __device__ __forceinline__ void dec4_e4m3_cvt(uint32_t r, uint32_t& lo, uint32_t& hi) {
   asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
@@ -994,13 +1003,18 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt) {
             const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
-            if (n0 < G) {
-              store_out<QBF16>(p.out, ob0 + da, acc[nt][mt][0] * i0);
-              store_out<QBF16>(p.out, ob0 + db, acc[nt][mt][2] * i0);
-            }
-            if (n1 < G) {
-              store_out<QBF16>(p.out, ob1 + da, acc[nt][mt][1] * i1);
-              store_out<QBF16>(p.out, ob1 + db, acc[nt][mt][3] * i1);
+            if constexpr (!Gm::k16) {  // rows g, g + 8 of an m-tile are head dims da, da + 1: one 4-byte store
+              if (n0 < G) store_out2<QBF16>(p.out, ob0 + da, acc[nt][mt][0] * i0, acc[nt][mt][2] * i0);
+              if (n1 < G) store_out2<QBF16>(p.out, ob1 + da, acc[nt][mt][1] * i1, acc[nt][mt][3] * i1);
+            } else {
+              if (n0 < G) {
+                store_out<QBF16>(p.out, ob0 + da, acc[nt][mt][0] * i0);
+                store_out<QBF16>(p.out, ob0 + db, acc[nt][mt][2] * i0);
+              }
+              if (n1 < G) {
+                store_out<QBF16>(p.out, ob1 + da, acc[nt][mt][1] * i1);
+                store_out<QBF16>(p.out, ob1 + db, acc[nt][mt][3] * i1);
+              }
             }
           }
         }
@@ -1014,13 +1028,20 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
 #pragma unroll
         for (int mt = 0; mt < KT; ++mt) {
           const int da = dmap<KVF>(mt, g), db = dmap<KVF>(mt, g + 8);
-          if (n0 < G) {
-            base[n0 * D + da] = acc[nt][mt][0] * vs;
-            base[n0 * D + db] = acc[nt][mt][2] * vs;
-          }
-          if (n1 < G) {
-            base[n1 * D + da] = acc[nt][mt][1] * vs;
-            base[n1 * D + db] = acc[nt][mt][3] * vs;
+          if constexpr (!Gm::k16) {  // head dims da, da + 1 (da even): one 8-byte store
+            if (n0 < G)
+              *reinterpret_cast<float2*>(base + n0 * D + da) = make_float2(acc[nt][mt][0] * vs, acc[nt][mt][2] * vs);
+            if (n1 < G)
+              *reinterpret_cast<float2*>(base + n1 * D + da) = make_float2(acc[nt][mt][1] * vs, acc[nt][mt][3] * vs);
+          } else {
+            if (n0 < G) {
+              base[n0 * D + da] = acc[nt][mt][0] * vs;
+              base[n0 * D + db] = acc[nt][mt][2] * vs;
+            }
+            if (n1 < G) {
+              base[n1 * D + da] = acc[nt][mt][1] * vs;
+              base[n1 * D + db] = acc[nt][mt][3] * vs;
+            }
           }
         }
         if (g == 0) {
@@ -1271,7 +1292,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
         continue;
       }
       // pieces loaded at once: as many as the registers the main loop leaves allow
-      merge_column<D, QBF16, Gm::k16 ? 32 : 16>(p, cb, ch, cn, k0, np, lane);
+      merge_column<D, QBF16, Gm::k16 ? 32 : 24>(p, cb, ch, cn, k0, np, lane);
     }
   }
 
