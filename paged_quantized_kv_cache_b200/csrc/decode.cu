@@ -704,6 +704,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
   // multi-query: positions at the end of the sequence hidden from this lane's
   // columns n = 8nt + 2qd + c (query token q0 + n / Gh of k sits k - 1 - q0 -
   // n / Gh before the end)
+  const int hmax = p.k - 1 - p.q0;  // hidden positions of column 0, the most of any column
   int hid[NT][2];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
@@ -865,6 +866,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
   uint32_t qf[NT][KT][2];
   float acc[NT][KT][4];
   float mm[NT][2], ll[NT][2], vref;  // running max and sum of each of the lane's columns
+  float rvref = 0.f;                  // FP8: 1 / vref (0 while vref is 0)
   // softmax scale (log2 units) of each of the lane's columns, times the power
   // of two its query row was scaled down by before narrowing to f16
   // (quantized caches; 16-bit caches keep the query in its own type)
@@ -894,6 +896,7 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
         for (int mt = 0; mt < KT; ++mt) acc[nt][mt][0] = acc[nt][mt][1] = acc[nt][mt][2] = acc[nt][mt][3] = 0.f;
       }
       vref = 0.f;
+      rvref = 0.f;
       if (b == qb && h == qh) return;
       qb = b;
       qh = h;
@@ -1126,16 +1129,26 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
       float xA[NT][4], xB[NT][4], bm[NT][2];
       bool need_any = false;
       constexpr float kLazy = lazy_of<KVF>();
+      // both blocks full and visible to every column (the usual case): no mask
+      const bool full2 = useA && useB && remB - hmax >= kBlock;
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         const float mA0 = csc[nt][0] * skA, mA1 = csc[nt][1] * skA;
         const float mB0 = csc[nt][0] * skB, mB1 = csc[nt][1] * skB;
+        if (full2) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = g + 8 * (e >> 1), hd = hid[nt][e & 1];
-          // column n sees the tokens before the last hid ones (0 for one query token)
-          xA[nt][e] = (!useA || r >= remA - hd) ? kNegInf : scA[nt][e] * ((e & 1) ? mA1 : mA0);
-          xB[nt][e] = (!useB || r >= remB - hd) ? kNegInf : scB[nt][e] * ((e & 1) ? mB1 : mB0);
+          for (int e = 0; e < 4; ++e) {
+            xA[nt][e] = scA[nt][e] * ((e & 1) ? mA1 : mA0);
+            xB[nt][e] = scB[nt][e] * ((e & 1) ? mB1 : mB0);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int r = g + 8 * (e >> 1), hd = hid[nt][e & 1];
+            // column n sees the tokens before the last hid ones (0 for one query token)
+            xA[nt][e] = (!useA || r >= remA - hd) ? kNegInf : scA[nt][e] * ((e & 1) ? mA1 : mA0);
+            xB[nt][e] = (!useB || r >= remB - hd) ? kNegInf : scB[nt][e] * ((e & 1) ? mB1 : mB0);
+          }
         }
         bm[nt][0] = fmaxf(fmaxf(xA[nt][0], xA[nt][2]), fmaxf(xB[nt][0], xB[nt][2]));
         bm[nt][1] = fmaxf(fmaxf(xA[nt][1], xA[nt][3]), fmaxf(xB[nt][1], xB[nt][3]));
@@ -1175,10 +1188,11 @@ __global__ void __launch_bounds__(DecodeGeom<KVF, D, NT>::kWarps * 32, 1)
             fc[nt][1] *= rs;
           }
           vref = svm;
+          rvref = 1.f / svm;  // only when the largest scale grows
           rescale = true;
         }
-        prA = (useA && vref > 0.f) ? svA / vref : 0.f;
-        prB = (useB && vref > 0.f) ? svB / vref : 0.f;
+        prA = useA ? svA * rvref : 0.f;  // <= 1; differs from svA / vref by an ulp at most
+        prB = useB ? svB * rvref : 0.f;
       }
       if (rescale) {
 #pragma unroll
