@@ -596,6 +596,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
     // (its MMA warp issues S(t) into the buffer P(t - 2) occupied only then).
     auto leave = [&]() -> bool { return !__all_sync(kFull, ok); };
     float m = -INFINITY, l = 0.f, vref = 0.f;
+    float rvref = 0.f;  // FP8: 1 / vref (0 while vref is 0), recomputed only when vref grows
     if constexpr (Gm::k16) {
       mask_next = prepare(0);
       if (leave()) aborted = true;
@@ -679,6 +680,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         if (svm > vref) {
           fv = vref / svm;
           vref = svm;
+          rvref = 1.f / svm;
         }
       }
       l *= fm;
@@ -692,7 +694,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         float vr[4] = {1.f, 1.f, 1.f, 1.f};
         if constexpr (Gm::kFp8) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) vr[j] = vref > 0.f ? vs[j] / vref : 0.f;
+          for (int j = 0; j < 4; ++j) vr[j] = vs[j] * rvref;  // <= 1 up to an ulp
         }
 #pragma unroll
         for (int c = 0; c < 64; c += 2) {
