@@ -461,8 +461,10 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         uint8_t* vop = sVop + (t % 3) * Gm::kOpBytes;
         constexpr int CPR = D / 8;  // 16-byte operand chunks per row
         static_assert(kN * CPR % Gm::kDeqThreads == 0, "whole rounds");
+        constexpr int kRounds = kN * CPR / Gm::kDeqThreads;  // a compile-time count: fully unrolled
 #pragma unroll
-        for (int u = dq; u < kN * CPR; u += Gm::kDeqThreads) {
+        for (int k = 0; k < kRounds; ++k) {
+          const int u = dq + k * Gm::kDeqThreads;
           const int rr = u / CPR, c = u % CPR, j = rr >> 4, tr = rr & 15;
           const bool okr = ((mask >> j) & 1) && base + rr < L;
           uint32_t kf[4] = {0, 0, 0, 0}, vf[4] = {0, 0, 0, 0};
@@ -509,7 +511,9 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
           // outlier channels (their codes are 0): write the fp16 values over them;
           // item = (block j, K|V, slot, eighth of the tokens)
           deq_sync<Gm::kDeqThreads>();
-          for (int gt = dq; gt < 256; gt += Gm::kDeqThreads) {
+#pragma unroll
+          for (int k = 0; k < 256 / Gm::kDeqThreads; ++k) {
+            const int gt = dq + k * Gm::kDeqThreads;
             const int j = gt >> 6, kv = (gt >> 5) & 1, slot = (gt >> 3) & 3, part = gt & 7;
             if ((mask >> j) & 1) {
               const uint8_t* side = st + 4 * Gm::kRawTile + j * Gm::kSide;
