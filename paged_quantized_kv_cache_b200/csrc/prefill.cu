@@ -735,7 +735,7 @@ __global__ void __launch_bounds__(PrefillGeom<KVF, D>::kThreads, 1)
         }
       }
       // P row -> tensor memory over this row's S(t) (P_hi, then P_lo for bf16),
-      // then this warp's share of P(t) is handed to the MMA warp
+      // then this warp's share of P(t) is handed to its warpgroup's MMA warp
       if constexpr (Gm::kSplitP) {
         uint32_t pp[64];
 #pragma unroll

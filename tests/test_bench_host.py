@@ -86,3 +86,21 @@ def test_config_keys_and_byte_counts():
     # the FP4 chunk write of 512 tokens x 256 sequences: about 705 MB
     b = bench.write_call_bytes(W.DT_FP4, 131072, 8, 128, 131072 // 16)
     assert 700e6 < b < 710e6
+
+
+def test_profiled_traffic_only_for_its_source_split_and_query_length(tmp_path, monkeypatch):
+    """A committed ncu traffic figure is used only while it describes the kernel
+    being timed: same decode source, same split, one query token per sequence."""
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    good = "# comment\nsource_hash=%s\nsplit_blocks=32\ndram_bytes_per_launch=123456\n" % bench.decode_source_hash()
+    (prof / "decode_traffic_llama70b_bf16.txt").write_text(good)
+    (prof / "decode_traffic_llama70b_fp8_e4m3.txt").write_text(good.replace(bench.decode_source_hash(), "0" * 16))
+    h = bench.decode_source_hash()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "decode_source_hash", lambda: h)
+    assert bench.profiled_traffic("llama70b", "bf16", 32) == 123456
+    assert bench.profiled_traffic("llama70b", "bf16", 0) is None        # another split
+    assert bench.profiled_traffic("llama70b", "bf16", 32, q_len=4) is None  # multi-query decode
+    assert bench.profiled_traffic("llama70b", "fp8_e4m3", 32) is None   # taken from another source
+    assert bench.profiled_traffic("llama8b", "bf16", 32) is None        # no capture
